@@ -1,0 +1,452 @@
+"""Benchmark of the SmoothQuant W8A8 int8 linear layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload proj]
+                    [--impl ours|reference] [--no-e2e] [--no-cpu-baseline]
+
+A step is one pass of the whole path over one batch of seeded synthetic input:
+calibration (column max-abs of the calibration batch and of W, smoothing
+factor s), weight fold + int8 quantisation, per-token activation quantisation
+and the int8 tcgen05 GEMM with its dequant + bias epilogue.  The default
+workload is the projection-shaped layer: X[512x4096] bf16 with 41 outlier
+channels x50, W[4096x4096] bf16 ~N(0,0.02), no bias, alpha 0.5, calibration
+batch of 512 rows.
+
+Timing: every step is preceded by a 256 MiB write that evicts L2 (the inputs
+are smaller than L2); CUDA events on the launching stream bracket the step and
+each library call inside it; each call is replayed from its own CUDA graph so
+that host launch latency does not leak into the device timeline.  With N > 1
+(one process per GPU under torchrun) every rank runs an independent replica
+(the layer shards by tokens with no exchange): the value is the tokens all
+ranks processed divided by the slowest rank's time.
+
+The JSON line adds: `e2e` (the same step through the Python binding with the
+inputs copied from pinned host memory and Y copied back, every step),
+`roofline` of the dominant kernel, `cpu_baseline` (the CPU oracle timed on a
+bounded sample, rank 0 only), sampled `clocks`, and per-call `kernels` times.
+`--impl reference` times the CPU oracle itself as the reference arm.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "W8A8 linear int8 TOPS & tokens/s at 1 B200; % of INT8 tensor peak / HBM roofline"
+UNIT = "tokens/s"
+FLUSH_BYTES = 256 << 20
+# fallback peaks (only if MEASURED_PEAKS.json is absent)
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+INT8_OVER_BF16 = 2.0  # nominal dense int8 / bf16 ratio (4.5 / 2.25 PFLOP/s)
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default="proj", choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--settle-s", type=float, default=1.0,
+                    help="untimed replays after warm-up until this much wall time has passed (clock sampling)")
+    return ap.parse_args()
+
+
+def workload_config(wl):
+    return {
+        "workload": f"{wl.name}: X[{wl.M}x{wl.K}] W[{wl.N}x{wl.K}] bf16, alpha {wl.alpha_f32:g}, "
+                    f"{wl.outliers} outlier channels x{wl.outlier_scale:g}, calibration {wl.R} rows, "
+                    f"{'bias' if wl.has_bias else 'no bias'}",
+        "M": wl.M, "N": wl.N, "K": wl.K, "R": wl.R,
+        "l2": "flushed before every timed step (256 MiB write); inputs smaller than L2",
+    }
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d["hbm_gbs"], d["bf16_tflops"], d.get("bf16_tflops_sustained"), "measured"
+    return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, None, "fallback"
+
+
+def algorithmic_work(wl):
+    """Bytes (HBM-bound kernels) or int8 ops (GEMM) per launch, per call."""
+    M, N, K, R = wl.M, wl.N, wl.K, wl.R
+    return {
+        "sq_calibrate": ("hbm", 2 * R * K + 2 * N * K + 8 * K),
+        "sq_prepare_weight": ("hbm", 3 * N * K + 4 * N + 4 * K),
+        "sq_quantize_act": ("hbm", 3 * M * K + 4 * M + 4 * K),
+        "sq_linear": ("tensor", 2 * M * N * K),
+    }
+
+
+def source_sha():
+    h = hashlib.sha256()
+    cs = os.path.join(ROOT, "w8a8_smoothquant_int8_sq_b200", "csrc")
+    for f in sorted(os.listdir(cs)):
+        h.update(open(os.path.join(cs, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel_call, wl_name):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel sources."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        d = json.load(open(p))
+    except Exception:
+        return None
+    e = d.get(wl_name, {}).get(kernel_call)
+    if not e or e.get("source_sha") != source_sha():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+# ------------------------------------------------------------------- clocks
+class ClockSampler:
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,utilization.gpu,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        import tempfile
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 10:
+                continue
+            try:
+                rows.append(dict(sm=float(f[1]), max=float(f[2]), power=float(f[3]), util=float(f[4]),
+                                 hw=f[6], hwt=f[7], swt=f[8], pcap=f[9]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        load = [r for r in rows if r["util"] > 0] or rows
+        reasons = set()
+        for r in load:
+            for k, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"), ("swt", "sw_thermal_slowdown"),
+                            ("pcap", "sw_power_cap")):
+                if r[k].lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": float(np.median([r["sm"] for r in load])), "sm_max_mhz": load[0]["max"],
+                "reasons": sorted(reasons), "samples": len(load),
+                "power_w_max": max(r["power"] for r in load)}
+
+
+# --------------------------------------------------------------- CPU oracle
+def oracle_step(inp, wl, rows=None):
+    from oracle import smoothquant as O
+    s, _ = O.calibrate(inp["C"], inp["W"], wl.alpha_f32)
+    Wq, ws = O.fold_and_quantize_weight(inp["W"], s)
+    X = inp["X"] if rows is None else inp["X"][:rows]
+    Y, _, _, _ = O.forward(X, s, Wq, ws, inp["bias"])
+    return Y
+
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+def cpu_oracle_rate(wl, seconds, max_steps=None):
+    """Tokens/s of the oracle on whole steps, run until `seconds` pass."""
+    inp = workloads.make_inputs(wl)
+    oracle_step(inp, wl)  # warm (page-in, BLAS threads)
+    n, t0 = 0, time.perf_counter()
+    while True:
+        oracle_step(inp, wl)
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= seconds or (max_steps and n >= max_steps):
+            break
+    return wl.M * n / el, n, el
+
+
+def run_reference(args, wl, rank, world):
+    if rank != 0:
+        return
+    inp = workloads.make_inputs(wl)
+    for _ in range(args.warmup):
+        oracle_step(inp, wl)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_step(inp, wl)
+    el = time.perf_counter() - t0
+    v = wl.M * args.steps / el
+    cores = cpu_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * el / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64+fp32 (numpy)",
+        "data": "synthetic", "config": workload_config(wl),
+        "cpu_baseline": {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"{args.steps} whole {wl.name} steps (calibrate, fold+quantise W, forward)"},
+        "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# -------------------------------------------------------------------- GPU arm
+def run_ours(args, wl, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    import w8a8_smoothquant_int8_sq_b200 as sq
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    inp = workloads.make_inputs(wl)
+
+    def d(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    C, W, X = d(inp["C"]), d(inp["W"]), d(inp["X"])
+    b = d(inp["bias"]) if inp["bias"] is not None else None
+    K, N, M = wl.K, wl.N, wl.M
+    s = torch.empty(K, dtype=torch.float32, device=dev)
+    Wq = torch.empty(N, K, dtype=torch.int8, device=dev)
+    w_scale = torch.empty(N, dtype=torch.float32, device=dev)
+    Xq = torch.empty(M, K, dtype=torch.int8, device=dev)
+    x_scale = torch.empty(M, dtype=torch.float32, device=dev)
+    Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+    ws_cal = torch.empty(sq.sq_calibrate_workspace_bytes(K), dtype=torch.uint8, device=dev)
+    ws_fwd = torch.empty(max(sq.sq_forward_workspace_bytes(M, N, K), 16), dtype=torch.uint8, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    calls = {
+        "sq_calibrate": lambda: sq.sq_calibrate(C, W, wl.alpha_f32, s=s, workspace=ws_cal),
+        "sq_prepare_weight": lambda: sq.sq_prepare_weight(W, s, Wq=Wq, w_scale=w_scale),
+        "sq_quantize_act": lambda: sq.sq_quantize_act(X, s, Xq=Xq, x_scale=x_scale),
+        "sq_linear": lambda: sq.sq_linear(Xq, x_scale, Wq, w_scale, b, Y=Y),
+    }
+    launches_per_call = {"sq_calibrate": 2, "sq_prepare_weight": 1, "sq_quantize_act": 1, "sq_linear": 1}
+    names = list(calls)
+    # initialise library caches outside capture, then one graph per call
+    for f in calls.values():
+        f()
+    torch.cuda.synchronize()
+    graphs = {}
+    for n in names:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            calls[n]()
+        graphs[n] = g
+    torch.cuda.synchronize()
+
+    stream = torch.cuda.current_stream()
+
+    def step(evs=None):
+        flush.fill_(1)
+        if evs is not None:
+            evs[0].record(stream)
+        for i, n in enumerate(names):
+            graphs[n].replay()
+            if evs is not None:
+                evs[i + 1].record(stream)
+
+    sampler = ClockSampler(local_rank) if rank == 0 else None
+    if sampler:
+        sampler.start()
+    t_settle = time.perf_counter()
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    # keep the GPU under load briefly so the clock sampler sees steady clocks
+    while time.perf_counter() - t_settle < args.settle_s:
+        for _ in range(50):
+            step()
+        torch.cuda.synchronize()
+
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)] for _ in range(args.steps)]
+    t_wall = time.perf_counter()
+    for k in range(args.steps):
+        step(evs[k])
+    torch.cuda.synchronize()
+    wall = time.perf_counter() - t_wall
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop() if sampler else None
+
+    per_call = {n: 0.0 for n in names}
+    total_ms = 0.0
+    for e in evs:
+        total_ms += e[0].elapsed_time(e[-1])
+        for i, n in enumerate(names):
+            per_call[n] += e[i].elapsed_time(e[i + 1])
+    step_ms = total_ms / args.steps
+    per_call = {n: v / args.steps for n, v in per_call.items()}
+    if world > 1:
+        t = torch.tensor([step_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        step_ms = float(t.item())
+
+    # correctness guard on the timed buffers (cheap; sq_forward path equals these calls)
+    assert sq.sq_device_status() == 0, "device-side timeout flagged"
+
+    # ------------------------------------------------------------- e2e leg
+    e2e = None
+    if not args.no_e2e:
+        hC = torch.from_numpy(inp["C"].view(np.int16)).view(torch.bfloat16).pin_memory()
+        hW = torch.from_numpy(inp["W"].view(np.int16)).view(torch.bfloat16).pin_memory()
+        hX = torch.from_numpy(inp["X"].view(np.int16)).view(torch.bfloat16).pin_memory()
+        hb = torch.from_numpy(inp["bias"].view(np.int16)).view(torch.bfloat16).pin_memory() if b is not None else None
+        hY = torch.empty(M, N, dtype=torch.bfloat16).pin_memory()
+        dC, dW, dX = torch.empty_like(C), torch.empty_like(W), torch.empty_like(X)
+        db = torch.empty_like(b) if b is not None else None
+
+        def e2e_step():
+            dC.copy_(hC, non_blocking=True)
+            dW.copy_(hW, non_blocking=True)
+            dX.copy_(hX, non_blocking=True)
+            if db is not None:
+                db.copy_(hb, non_blocking=True)
+            sq.sq_calibrate(dC, dW, wl.alpha_f32, s=s, workspace=ws_cal)
+            sq.sq_prepare_weight(dW, s, Wq=Wq, w_scale=w_scale)
+            sq.sq_forward(dX, s, Wq, w_scale, db, Y=Y, workspace=ws_fwd)
+            hY.copy_(Y, non_blocking=True)
+
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
+        if world > 1:
+            t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        h2d = sum(t.numel() * t.element_size() for t in (hC, hW, hX) + ((hb,) if hb is not None else ()))
+        e2e = {"value": wl.M * world / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": hY.numel() * hY.element_size(), "ms_per_step": e2e_ms,
+               "call": "sq_calibrate + sq_prepare_weight + sq_forward"}
+
+    if rank != 0:
+        return
+
+    hbm_gbs, bf16_tf, bf16_tf_sus, peak_kind = peaks()
+    int8_peak_tops = bf16_tf * INT8_OVER_BF16
+    work = algorithmic_work(wl)
+    kernels = {}
+    for n in names:
+        bound, amount = work[n]
+        ms = per_call[n]
+        if bound == "hbm":
+            ach = amount / (ms * 1e-3) / 1e9
+            kernels[n] = {"ms": ms, "bound": "hbm", "algorithmic_bytes": amount, "achieved_gbs": ach,
+                          "frac_of_measured_hbm": ach / hbm_gbs, "launches": launches_per_call[n]}
+        else:
+            ach = amount / (ms * 1e-3) / 1e12
+            kernels[n] = {"ms": ms, "bound": "tensor", "int8_ops": amount, "achieved_tops": ach,
+                          "frac_of_int8_peak": ach / int8_peak_tops, "launches": launches_per_call[n]}
+    dom = max(names, key=lambda n: per_call[n])
+    kd = kernels[dom]
+    if kd["bound"] == "hbm":
+        roof = {"bound": "hbm", "achieved": kd["achieved_gbs"], "peak": hbm_gbs, "unit": "GB/s",
+                "frac": kd["achieved_gbs"] / hbm_gbs}
+    else:
+        roof = {"bound": "tensor", "achieved": kd["achieved_tops"], "peak": int8_peak_tops, "unit": "TFLOP/s",
+                "frac": kd["achieved_tops"] / int8_peak_tops}
+    roof["kernel"] = dom
+    roof["peak_source"] = (f"{peak_kind} {'HBM copy' if kd['bound'] == 'hbm' else 'cuBLAS bf16 burst x2 (nominal int8/bf16)'}")
+    roof["traffic"] = ncu_traffic(dom, wl.name)
+
+    cpu = None
+    if not args.no_cpu_baseline and world == 1:
+        v, n, el = cpu_oracle_rate(wl, args.cpu_seconds)
+        cpu = {"value": v, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+               "sample": f"{n} whole {wl.name} steps in {el:.1f} s (calibrate, fold+quantise W, forward)"}
+
+    value = wl.M * world / (step_ms * 1e-3)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "int8", "data": "synthetic", "config": workload_config(wl),
+        "tops_per_step": 2.0 * wl.M * wl.N * wl.K * world / (step_ms * 1e-3) / 1e12,
+        "gemm_tops": kernels["sq_linear"]["achieved_tops"],
+        "roofline": roof, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
+        "gpu_launches": args.steps * sum(launches_per_call.values()),
+        "clocks": clocks, "wall_s_timed": wall,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    wl = workloads.get(args.workload)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, wl, rank, world)
+        return
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        run_ours(args, wl, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

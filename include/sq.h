@@ -1,0 +1,185 @@
+/*
+ * sq.h -- C ABI of libsq, the SmoothQuant W8A8 int8 linear layer for B200 (sm_100a).
+ *
+ * The operations are those of the SmoothQuant page
+ * ("w8a8_smoothquant.py -- W8A8 com SmoothQuant e alpha APRENDIVEL (V5)"),
+ * restated as functions on caller-owned device buffers:
+ *
+ *   calibration    s_j  = max(mx_j,1e-8)^a / max(mw_j,1e-8)^(1-a), clamped at 1e-8
+ *                  (calibrate_smoothquant; running max of SmoothQuantW8A8.calibrate)
+ *   weight prep    W~ = W * s ; per-output-row symmetric int8 (freeze_quantization,
+ *                  quantize_per_channel_symmetric)
+ *   act quant      X~ = X / s ; per-token symmetric int8 (forward,
+ *                  quantize_per_token_symmetric)
+ *   int8 linear    acc = Xq Wq^T (int32) ; Y = bf16(acc * x_scale[m] * w_scale[n] + bias[n])
+ *                  (forward: "INT8 x INT8 -> INT32 -> fp32" on real hardware)
+ *
+ * Conventions shared by every entry point
+ *   - Layouts are row-major and dense: X[M][K], C[R][K], W[N][K] (nn.Linear
+ *     [d_out][d_in]), Xq[M][K], Wq[N][K], Y[M][N]; s[K], x_scale[M], w_scale[N],
+ *     bias[N].  bf16 values travel as their 16-bit patterns (sq_bf16).
+ *   - Every pointer is a DEVICE pointer owned by the caller; the library keeps no
+ *     reference after the call returns and allocates no device memory.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default stream)
+ *     and runs asynchronously: a returned SQ_OK means "validated and launched".
+ *     Output buffers must not alias inputs.
+ *   - Integer codes are symmetric: -127..127 (-128 is never produced); rounding
+ *     is to nearest, ties to even.
+ *   - Requirements: K % 16 == 0 (TMA rows are 16-byte multiples), every pointer
+ *     16-byte aligned, M, N, K >= 1 (R >= 0).  Violations return an error code
+ *     and launch nothing.  Inputs must be finite; NaN/Inf give unspecified codes.
+ *   - Errors: the return value is an sq_status; sq_last_error() gives a
+ *     human-readable message for the calling thread's last failure.
+ *     Device-side wait timeouts (never expected in correct use) are latched in a
+ *     per-process device word read by sq_device_status().
+ */
+#ifndef SQ_H_
+#define SQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define SQ_API __attribute__((visibility("default")))
+#else
+#define SQ_API
+#endif
+
+typedef uint16_t sq_bf16; /* bf16 bit pattern */
+
+typedef enum {
+  SQ_OK = 0,
+  SQ_ERR_NULL = 1,        /* a required pointer is NULL */
+  SQ_ERR_SHAPE = 2,       /* inconsistent or out-of-range sizes */
+  SQ_ERR_ALIGN = 3,       /* K % 16 != 0 or a pointer not 16-byte aligned */
+  SQ_ERR_ARG = 4,         /* alpha outside [0, 1], or another bad scalar */
+  SQ_ERR_UNSUPPORTED = 5, /* device is not sm_100 */
+  SQ_ERR_CUDA = 6,        /* a CUDA runtime/driver call failed */
+  SQ_ERR_TIMEOUT = 7,     /* a device-side wait ran out (see sq_device_status) */
+  SQ_ERR_WORKSPACE = 8    /* workspace NULL or smaller than required */
+} sq_status;
+
+/* Library version, e.g. 100 for 0.1.0. */
+SQ_API int sq_version(void);
+
+/* Message for the calling thread's most recent failing call ("" if none). */
+SQ_API const char* sq_last_error(void);
+
+/* Name of a status code. */
+SQ_API const char* sq_status_string(sq_status st);
+
+/* ------------------------------------------------------------ calibration
+ * sq_calibrate -- smoothing factor s from activation and weight statistics.
+ * Page: calibrate_smoothquant (formula for s_j, the 1e-8 clamps),
+ * SmoothQuantW8A8.calibrate (running per-channel max of |X| over batches) and
+ * freeze_quantization (s from the running max and the weight's per-input-
+ * channel max).
+ *
+ *   C[R][K]    calibration activations (bf16); may be NULL when R == 0
+ *   W[N][K]    layer weight (bf16)
+ *   alpha      smoothing strength in [0, 1]
+ *   s[K]       OUT: fp32 smoothing factor.  mx^a and mw^(1-a) are evaluated
+ *              in float64 and the quotient is rounded once to fp32.
+ *   mx_inout   NULL, or [K] fp32 running max-abs of activations: read, merged
+ *              with this batch's column max, written back (start from zeros).
+ *              With R == 0 it must be non-NULL and s comes from it alone.
+ *   workspace  device scratch of at least sq_calibrate_workspace_bytes(K)
+ *              bytes, 16-byte aligned; contents on entry are ignored.
+ * Launches: one memset of the workspace and two kernels (column max-abs over
+ * C and W, then the per-channel finalisation).
+ */
+SQ_API size_t sq_calibrate_workspace_bytes(int64_t K);
+SQ_API sq_status sq_calibrate(const sq_bf16* C, int64_t R, int64_t K,
+                       const sq_bf16* W, int64_t N, float alpha,
+                       float* s, float* mx_inout,
+                       void* workspace, size_t workspace_bytes, void* stream);
+
+/* --------------------------------------------------------- weight prepare
+ * sq_prepare_weight -- fold s into W and quantise per output channel.
+ * Page: freeze_quantization (W_smooth = weight_fp * s) and
+ * quantize_per_channel_symmetric(axis = 0).
+ *
+ *   W[N][K] bf16 in; s[K] fp32 in
+ *   Wq[N][K]  OUT int8 codes  q = clamp(round_half_even(fl(W*s) / w_scale), +-127)
+ *   w_scale[N] OUT fp32  fl( max(max_j |fl(W*s)|, 1e-8) / 127 )
+ * Every step is the page's fp32 operation (correctly rounded), so the result is
+ * bit-identical to an IEEE fp32 evaluation of the page's formulas.
+ */
+SQ_API sq_status sq_prepare_weight(const sq_bf16* W, int64_t N, int64_t K, const float* s,
+                            int8_t* Wq, float* w_scale, void* stream);
+
+/* ------------------------------------------------------- activation quant
+ * sq_quantize_act -- dynamic per-token quantisation of X / s.
+ * Page: forward (X_smooth = X / s) and quantize_per_token_symmetric.
+ *
+ *   X[M][K] bf16 in; s[K] fp32 in
+ *   Xq[M][K]   OUT int8  q = clamp(round_half_even(fl(X/s) / x_scale), +-127)
+ *   x_scale[M] OUT fp32  fl( max(max_j |fl(X/s)|, 1e-8) / 127 )
+ * Divisions are correctly rounded fp32 divisions, as on the page.
+ */
+SQ_API sq_status sq_quantize_act(const sq_bf16* X, int64_t M, int64_t K, const float* s,
+                          int8_t* Xq, float* x_scale, void* stream);
+
+/* ----------------------------------------------------------- int8 linear
+ * sq_linear -- Y = bf16( (Xq Wq^T)[m][n] * x_scale[m] * w_scale[n] + bias[n] ).
+ * Page: forward ("INT8 x INT8 -> INT32 -> fp32"; bias added after the product).
+ *
+ *   Xq[M][K], Wq[N][K] int8; x_scale[M], w_scale[N] fp32; bias[N] bf16 or NULL
+ *   Y[M][N]   OUT bf16.  The int32 accumulation is exact (|acc| <= 127^2 K,
+ *             K <= 133143); the epilogue runs in fp32 and rounds to bf16
+ *             (nearest even), i.e. within one bf16 ulp of the exact value.
+ *   workspace may be NULL when sq_workspace_bytes(M, N, K) == 0.
+ * Runs the tcgen05 (kind::i8) GEMM: TMA-fed shared-memory tiles, int32
+ * accumulators in tensor memory, fused dequant + bias epilogue.
+ */
+SQ_API size_t sq_workspace_bytes(int64_t M, int64_t N, int64_t K);
+SQ_API sq_status sq_linear(const int8_t* Xq, const float* x_scale, const int8_t* Wq,
+                    const float* w_scale, const sq_bf16* bias,
+                    int64_t M, int64_t N, int64_t K, sq_bf16* Y,
+                    void* workspace, size_t workspace_bytes, void* stream);
+
+/* --------------------------------------------------------- fused forward
+ * sq_forward -- the per-batch path: sq_quantize_act followed by sq_linear,
+ * Y from bf16 X.  Page: forward of SmoothQuantW8A8 once frozen.
+ *
+ *   X[M][K] bf16, s[K], Wq[N][K], w_scale[N], bias[N] or NULL -> Y[M][N] bf16
+ *   workspace  at least sq_forward_workspace_bytes(M, N, K) bytes (holds the
+ *              intermediate Xq and x_scale); contents on entry are ignored.
+ * The codes and scales are identical to those of sq_quantize_act.
+ */
+SQ_API size_t sq_forward_workspace_bytes(int64_t M, int64_t N, int64_t K);
+SQ_API sq_status sq_forward(const sq_bf16* X, const float* s, const int8_t* Wq,
+                     const float* w_scale, const sq_bf16* bias,
+                     int64_t M, int64_t N, int64_t K, sq_bf16* Y,
+                     void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------- test hook
+ * sq_gemm_s32 -- the same tcgen05 GEMM main loop with a raw int32 epilogue:
+ * acc[M][N] = Xq Wq^T, exposing the accumulator for bit-exact checks.
+ */
+SQ_API sq_status sq_gemm_s32(const int8_t* Xq, const int8_t* Wq, int64_t M, int64_t N, int64_t K,
+                      int32_t* acc, void* stream);
+
+/* ------------------------------------------------------ device status word
+ * sq_device_status -- read (and with clear != 0, reset) the device-side status
+ * flags of the current device: bit 0 = a pipeline wait in a GEMM kernel timed
+ * out.  Synchronises the device.  Returns SQ_ERR_TIMEOUT if any bit is set.
+ */
+SQ_API sq_status sq_device_status(uint32_t* flags, int clear);
+
+/* --------------------------------------------------------- fault injection
+ * sq_debug_fail_after -- host-side fault injection for tests: after `n` more
+ * successful launches, entry points return SQ_ERR_CUDA without touching the
+ * GPU.  n < 0 disables injection (the default).
+ */
+SQ_API void sq_debug_fail_after(int n);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SQ_H_ */

@@ -1,0 +1,74 @@
+"""The C ABI library without a GPU: it loads, exports every symbol that
+include/sq.h declares, and rejects bad arguments with status codes before it
+touches a device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def sq():
+    from w8a8_smoothquant_int8_sq_b200 import build
+    build.build()
+    import w8a8_smoothquant_int8_sq_b200 as m
+    return m
+
+
+def declared_symbols():
+    text = open(os.path.join(ROOT, "include", "sq.h")).read()
+    return sorted(set(re.findall(r"SQ_API\s+[\w\s\*]+?\b(sq_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_path():
+    names = declared_symbols()
+    for n in ("sq_calibrate", "sq_prepare_weight", "sq_quantize_act", "sq_linear", "sq_forward", "sq_gemm_s32"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(sq):
+    lib = ctypes.CDLL(sq.library_path)
+    missing = [n for n in declared_symbols() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_version_and_sizes(sq):
+    assert sq.sq_version() == 100
+    assert sq.sq_calibrate_workspace_bytes(4096) >= 2 * 4096 * 4
+    assert sq.sq_forward_workspace_bytes(512, 4096, 4096) >= 512 * 4096 + 512 * 4
+    assert sq.lib.sq_status_string(7) == b"SQ_ERR_TIMEOUT"
+
+
+def test_validation_before_device(sq):
+    lib = sq.lib
+    a = ctypes.c_void_p(1 << 20)          # 16-byte aligned, never dereferenced
+    mis = ctypes.c_void_p((1 << 20) + 4)
+    assert lib.sq_quantize_act(None, 4, 64, a, a, a, None) == 1
+    assert lib.sq_quantize_act(a, 4, 40, a, a, a, None) == 3
+    assert lib.sq_quantize_act(a, 4, 8, a, a, a, None) == 2
+    assert lib.sq_quantize_act(a, 0, 64, a, a, a, None) == 2
+    assert lib.sq_quantize_act(mis, 4, 64, a, a, a, None) == 3
+    assert b"not 16-byte aligned" in lib.sq_last_error()
+    assert lib.sq_prepare_weight(a, 4, 64, None, a, a, None) == 1
+    assert lib.sq_prepare_weight(a, 4, 32768, a, a, a, None) == 2        # above the on-chip K limit
+    assert lib.sq_calibrate(a, 4, 64, a, 8, ctypes.c_float(-0.1), a, None, a, 1024, None) == 4
+    assert lib.sq_calibrate(a, 4, 64, a, 8, ctypes.c_float(float("nan")), a, None, a, 1024, None) == 4
+    assert lib.sq_calibrate(a, 4, 64, a, 8, ctypes.c_float(0.5), a, None, a, 8, None) == 8
+    assert lib.sq_calibrate(None, 0, 64, a, 8, ctypes.c_float(0.5), a, None, a, 1024, None) == 1
+    assert lib.sq_linear(a, a, a, a, mis, 4, 8, 64, a, None, 0, None) == 3
+    assert lib.sq_linear(a, a, a, a, None, 4, 8, 200000, a, None, 0, None) == 2
+    assert lib.sq_forward(a, a, a, a, None, 4, 8, 64, a, a, 16, None) == 8
+    assert lib.sq_gemm_s32(a, a, 4, 0, 64, a, None) == 2
+
+
+def test_valid_call_without_gpu_fails_cleanly(sq):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    a = ctypes.c_void_p(1 << 20)
+    st = sq.lib.sq_quantize_act(a, 4, 64, a, a, a, None)
+    assert st in (5, 6)          # no sm_100 device: UNSUPPORTED or CUDA error, never a crash
+    assert sq.lib.sq_last_error()

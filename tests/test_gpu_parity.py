@@ -1,0 +1,193 @@
+"""CUDA path (through the C ABI) against the CPU oracle, stage by stage.
+
+Each stage is fed the GPU's own outputs of the previous stage, so a mismatch
+points at one kernel: s -> (Wq, w_scale) -> (Xq, x_scale) -> acc -> Y.  The
+end-to-end test then runs the pure oracle from the same seeded bf16 inputs.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import workloads
+from oracle import smoothquant as O
+from tests.helpers import (assert_codes, assert_scales_close, assert_y_close, dev, dev_bf16, host,
+                           host_bf16_bits)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def sq():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    import w8a8_smoothquant_int8_sq_b200 as m
+    return m
+
+
+def _stages(sq, C, W, X, bias, alpha, label, report):
+    """Run every stage on the GPU and compare with the oracle; returns GPU tensors."""
+    K = W.shape[1]
+    Cd, Wd, Xd = dev_bf16(C), dev_bf16(W), dev_bf16(X)
+    bd = dev_bf16(bias) if bias is not None else None
+    # a1 calibration (running max starts from zeros, as the page's buffer does)
+    mx = torch.zeros(K, dtype=torch.float32, device="cuda")
+    s_g = sq.sq_calibrate(Cd, Wd, alpha, mx_inout=mx)
+    s_o, mx_o = O.calibrate(C, W, alpha)
+    s_h = host(s_g)
+    assert np.array_equal(host(mx), mx_o), f"{label}: running max differs"
+    report["s_ulp"] = assert_scales_close(s_h, s_o, f"{label}: s")
+    # a2 fold + weight quantisation, from the GPU's s
+    Wq_g, ws_g = sq.sq_prepare_weight(Wd, s_g)
+    Wq_o, ws_o = O.fold_and_quantize_weight(W, s_h)
+    _, _, vw = O.fold_and_quantize_weight_f64(W, s_h)
+    report["w_scale_ulp"] = assert_scales_close(host(ws_g), ws_o, f"{label}: w_scale")
+    report["w_code_ties"] = assert_codes(host(Wq_g), Wq_o, vw, f"{label}: Wq")
+    # a3 activation quantisation
+    Xq_g, xs_g = sq.sq_quantize_act(Xd, s_g)
+    Xq_o, xs_o = O.quantize_activation(X, s_h)
+    _, _, vx = O.quantize_activation_f64(X, s_h)
+    report["x_scale_ulp"] = assert_scales_close(host(xs_g), xs_o, f"{label}: x_scale")
+    report["x_code_ties"] = assert_codes(host(Xq_g), Xq_o, vx, f"{label}: Xq")
+    # a4 int8 GEMM, raw accumulator
+    acc_g = host(sq.sq_gemm_s32(Xq_g, Wq_g))
+    acc_o = O.int8_gemm(host(Xq_g), host(Wq_g))
+    assert np.array_equal(acc_g.astype(np.int64), acc_o), f"{label}: int32 accumulators differ"
+    # a5 dequant epilogue
+    Y_g = sq.sq_linear(Xq_g, xs_g, Wq_g, ws_g, bd)
+    report["y_tol_ratio"] = assert_y_close(host_bf16_bits(Y_g), acc_o, host(xs_g), host(ws_g), bias, f"{label}: Y")
+    # fused forward = the two kernels above, bit for bit
+    Y_f = sq.sq_forward(Xd, s_g, Wq_g, ws_g, bd)
+    assert torch.equal(Y_f.view(torch.int16), Y_g.view(torch.int16)), f"{label}: sq_forward != sq_linear(quantize_act)"
+    torch.cuda.synchronize()
+    return dict(s=s_g, Wq=Wq_g, ws=ws_g, Xq=Xq_g, xs=xs_g, Y=Y_g, Yf=Y_f)
+
+
+@pytest.mark.parametrize("name", ["tiny", "proj", "mlp", "decode"])
+def test_workload_stage_parity(sq, name):
+    wl = workloads.get(name)
+    inp = workloads.make_inputs(wl)
+    report = {}
+    g = _stages(sq, inp["C"], inp["W"], inp["X"], inp["bias"], wl.alpha_f32, name, report)
+    # end to end against the pure oracle (its own s, codes and scales)
+    s_o, _ = O.calibrate(inp["C"], inp["W"], wl.alpha_f32)
+    Wq_o, ws_o = O.fold_and_quantize_weight(inp["W"], s_o)
+    Y_o, Xq_o, xs_o, acc_o = O.forward(inp["X"], s_o, Wq_o, ws_o, inp["bias"])
+    if np.array_equal(host(g["s"]), s_o):
+        assert_y_close(host_bf16_bits(g["Yf"]), acc_o, xs_o, ws_o, inp["bias"], f"{name}: end-to-end Y")
+    yfp = O.reference_linear_f64(inp["X"], inp["W"], inp["bias"])
+    report["rel_err_vs_fp"] = O.quantization_error(yfp, O.widen_bf16(host_bf16_bits(g["Yf"])).astype(np.float64))
+    print(f"\n[parity] {name}: {report}")
+    assert report["rel_err_vs_fp"] < 0.05
+
+
+@pytest.mark.parametrize("M,N,K,with_bias", [
+    (1, 256, 256, True),        # single token
+    (100, 200, 48, False),      # K below one 128-byte stage, ragged M and N
+    (130, 36, 16, True),        # K = 16 (smallest), N not a multiple of 8 (scalar stores)
+    (257, 520, 4112, True),     # ragged K block (4112 = 32*128 + 16), M just past two tiles
+    (3, 8, 4096, False),        # tiny N
+    (384, 768, 1024, True),     # several full tiles in both dimensions
+    (129, 4104, 512, False),    # N just past a 256-wide tile boundary
+])
+def test_ragged_shapes(sq, M, N, K, with_bias):
+    rng = np.random.default_rng(M * 7919 + N * 31 + K)
+    oc = rng.choice(K, size=max(1, K // 100), replace=False)
+    X = workloads.random_bf16((M, K), seed=M + 1, outlier_cols=oc, outlier_scale=50.0)
+    C = workloads.random_bf16((64, K), seed=M + 2, outlier_cols=oc, outlier_scale=50.0)
+    W = workloads.random_bf16((N, K), seed=M + 3, scale=0.02)
+    b = workloads.random_bf16((N,), seed=M + 4, scale=0.01) if with_bias else None
+    report = {}
+    _stages(sq, C, W, X, b, np.float32(0.5).item(), f"{M}x{N}x{K}", report)
+    print(f"\n[parity] {M}x{N}x{K}: {report}")
+
+
+def test_zero_rows_and_floor(sq):
+    K, M, N = 64, 4, 32
+    X = workloads.random_bf16((M, K), seed=5)
+    X[1] = 0
+    W = workloads.random_bf16((N, K), seed=6, scale=0.02)
+    W[3] = 0
+    s = dev(np.ones(K, np.float32))
+    Xq, xs = sq.sq_quantize_act(dev_bf16(X), s)
+    Wq, ws = sq.sq_prepare_weight(dev_bf16(W), s)
+    floor_scale = np.float32(np.float32(1e-8) / np.float32(127))
+    assert host(xs)[1] == floor_scale and not host(Xq)[1].any()
+    assert host(ws)[3] == floor_scale and not host(Wq)[3].any()
+    Xq_o, xs_o = O.quantize_activation(X, np.ones(K, np.float32))
+    assert np.array_equal(host(Xq), Xq_o) and np.array_equal(host(xs), xs_o)
+
+
+def test_accumulator_extremes(sq):
+    K = 8192
+    Xq = np.full((3, K), 127, np.int8)
+    Xq[1] = -127
+    Xq[2, ::2] = -127
+    Wq = np.full((5, K), 127, np.int8)
+    acc = host(sq.sq_gemm_s32(dev(Xq), dev(Wq)))
+    assert acc[0, 0] == 132128768 and acc[1, 0] == -132128768 and acc[2, 0] == 0
+    assert np.array_equal(acc.astype(np.int64), O.int8_gemm(Xq, Wq))
+
+
+def test_running_max_two_batches(sq):
+    wl = workloads.get("tiny")
+    inp = workloads.make_inputs(wl, ("C", "W"))
+    C, W = inp["C"], inp["W"]
+    mx = torch.zeros(wl.K, dtype=torch.float32, device="cuda")
+    sq.sq_calibrate(dev_bf16(C[:20]), dev_bf16(W), wl.alpha_f32, mx_inout=mx)
+    s2 = sq.sq_calibrate(dev_bf16(C[20:]), dev_bf16(W), wl.alpha_f32, mx_inout=mx)
+    s_one = sq.sq_calibrate(dev_bf16(C), dev_bf16(W), wl.alpha_f32)
+    assert torch.equal(s2, s_one)
+    # R == 0: s from the running max alone
+    s3 = sq.sq_calibrate(None, dev_bf16(W), wl.alpha_f32, mx_inout=mx)
+    assert torch.equal(s3, s_one)
+
+
+def test_alpha_special_cases(sq):
+    wl = workloads.get("tiny")
+    inp = workloads.make_inputs(wl, ("C", "W"))
+    for a in (0.0, 1.0):
+        s = host(sq.sq_calibrate(dev_bf16(inp["C"]), dev_bf16(inp["W"]), a))
+        s_o, _ = O.calibrate(inp["C"], inp["W"], a)
+        assert_scales_close(s, s_o, f"alpha={a}")
+
+
+def test_status_codes(sq):
+    lib = sq.lib
+    X = torch.zeros(4, 64, dtype=torch.bfloat16, device="cuda")
+    s = torch.ones(64, dtype=torch.float32, device="cuda")
+    Xq = torch.empty(4, 64, dtype=torch.int8, device="cuda")
+    xs = torch.empty(4, dtype=torch.float32, device="cuda")
+    p = lambda t, off=0: ctypes.c_void_p(t.data_ptr() + off)  # noqa: E731
+    assert lib.sq_quantize_act(p(X, 2), 4, 64, p(s), p(Xq), p(xs), None) == 3      # misaligned
+    assert lib.sq_quantize_act(p(X), 4, 40, p(s), p(Xq), p(xs), None) == 3         # K % 16
+    assert lib.sq_quantize_act(p(X), 0, 64, p(s), p(Xq), p(xs), None) == 2         # M = 0
+    assert lib.sq_quantize_act(None, 4, 64, p(s), p(Xq), p(xs), None) == 1
+    W = torch.zeros(8, 64, dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(16, dtype=torch.uint8, device="cuda")
+    assert lib.sq_calibrate(p(X), 4, 64, p(W), 8, ctypes.c_float(1.5), p(s), None, p(ws), 16, None) == 4
+    assert lib.sq_calibrate(p(X), 4, 64, p(W), 8, ctypes.c_float(0.5), p(s), None, p(ws), 16, None) == 8
+    Wq = torch.zeros(8, 64, dtype=torch.int8, device="cuda")
+    w_scale = torch.ones(8, dtype=torch.float32, device="cuda")
+    Y = torch.empty(4, 8, dtype=torch.bfloat16, device="cuda")
+    assert lib.sq_forward(p(X), p(s), p(Wq), p(w_scale), None, 4, 8, 64, p(Y), p(ws), 16, None) == 8
+    with pytest.raises(ValueError):
+        sq.sq_forward(X, s, Wq, w_scale, workspace=ws)
+
+
+def test_fault_injection(sq):
+    X = torch.zeros(4, 64, dtype=torch.bfloat16, device="cuda")
+    s = torch.ones(64, dtype=torch.float32, device="cuda")
+    try:
+        sq.sq_debug_fail_after(1)
+        sq.sq_quantize_act(X, s)                       # the one allowed launch
+        with pytest.raises(sq.SqError) as ei:
+            sq.sq_quantize_act(X, s)
+        assert ei.value.status == 6 and "injected" in str(ei.value)
+    finally:
+        sq.sq_debug_fail_after(-1)
+    sq.sq_quantize_act(X, s)
+
+
+def test_device_status_clean(sq):
+    assert sq.sq_device_status() == 0

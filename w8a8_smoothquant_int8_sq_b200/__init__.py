@@ -1,0 +1,268 @@
+"""SmoothQuant W8A8 int8 linear layer on B200 (sm_100a): Python binding of libsq.
+
+This module is argument marshalling only: it checks tensor dtypes, devices and
+shapes, allocates output tensors when the caller passes none, and calls the C
+ABI declared in ``include/sq.h`` (``libsq.so``, built next to this file by
+``build.py``).  Every step of the computation runs in the library's CUDA
+kernels; there is no Python or CPU fallback -- importing this package without
+the built library raises ImportError.
+
+Tensors: bf16 inputs are ``torch.bfloat16``, codes ``torch.int8``, scales
+``torch.float32``; all on the current CUDA device, contiguous, 16-byte aligned.
+Work is enqueued on the current torch CUDA stream (or ``stream=``).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+__all__ = [
+    "SqError", "lib", "library_path",
+    "sq_version", "sq_calibrate", "sq_calibrate_workspace_bytes", "sq_prepare_weight",
+    "sq_quantize_act", "sq_linear", "sq_workspace_bytes", "sq_forward",
+    "sq_forward_workspace_bytes", "sq_gemm_s32", "sq_device_status", "sq_debug_fail_after",
+    "STATUS",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+library_path = os.path.join(_HERE, "libsq.so")
+
+STATUS = {
+    0: "SQ_OK", 1: "SQ_ERR_NULL", 2: "SQ_ERR_SHAPE", 3: "SQ_ERR_ALIGN", 4: "SQ_ERR_ARG",
+    5: "SQ_ERR_UNSUPPORTED", 6: "SQ_ERR_CUDA", 7: "SQ_ERR_TIMEOUT", 8: "SQ_ERR_WORKSPACE",
+}
+
+if not os.path.exists(library_path):
+    raise ImportError(
+        f"libsq.so not found at {library_path}; build it with "
+        "`python -m w8a8_smoothquant_int8_sq_b200.build` (nvcc, sm_100a)")
+lib = ctypes.CDLL(library_path)
+
+_P = ctypes.c_void_p
+_I64 = ctypes.c_int64
+_SZ = ctypes.c_size_t
+
+
+def _sig(name, res, *args):
+    f = getattr(lib, name)
+    f.restype = res
+    f.argtypes = list(args)
+    return f
+
+
+_sig("sq_version", ctypes.c_int)
+_sig("sq_last_error", ctypes.c_char_p)
+_sig("sq_status_string", ctypes.c_char_p, ctypes.c_int)
+_sig("sq_calibrate_workspace_bytes", _SZ, _I64)
+_sig("sq_calibrate", ctypes.c_int, _P, _I64, _I64, _P, _I64, ctypes.c_float, _P, _P, _P, _SZ, _P)
+_sig("sq_prepare_weight", ctypes.c_int, _P, _I64, _I64, _P, _P, _P, _P)
+_sig("sq_quantize_act", ctypes.c_int, _P, _I64, _I64, _P, _P, _P, _P)
+_sig("sq_workspace_bytes", _SZ, _I64, _I64, _I64)
+_sig("sq_linear", ctypes.c_int, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _SZ, _P)
+_sig("sq_forward_workspace_bytes", _SZ, _I64, _I64, _I64)
+_sig("sq_forward", ctypes.c_int, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _SZ, _P)
+_sig("sq_gemm_s32", ctypes.c_int, _P, _P, _I64, _I64, _I64, _P, _P)
+_sig("sq_device_status", ctypes.c_int, ctypes.POINTER(ctypes.c_uint32), ctypes.c_int)
+_sig("sq_debug_fail_after", None, ctypes.c_int)
+
+
+class SqError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS.get(status, status)}: {message}")
+        self.status = status
+
+
+def _check(st: int) -> None:
+    if st != 0:
+        msg = lib.sq_last_error()
+        raise SqError(st, msg.decode() if msg else "")
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+def _want(t: torch.Tensor, name: str, dtype: torch.dtype, ndim: int) -> torch.Tensor:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims, got shape {tuple(t.shape)}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+def _out(t, shape, dtype, device, name):
+    if t is None:
+        return torch.empty(shape, dtype=dtype, device=device)
+    _want(t, name, dtype, len(shape))
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    return t
+
+
+def sq_version() -> int:
+    return int(lib.sq_version())
+
+
+def sq_calibrate_workspace_bytes(K: int) -> int:
+    return int(lib.sq_calibrate_workspace_bytes(K))
+
+
+def sq_workspace_bytes(M: int, N: int, K: int) -> int:
+    return int(lib.sq_workspace_bytes(M, N, K))
+
+
+def sq_forward_workspace_bytes(M: int, N: int, K: int) -> int:
+    return int(lib.sq_forward_workspace_bytes(M, N, K))
+
+
+def _workspace(ws, nbytes, device):
+    if ws is None:
+        return torch.empty(max(nbytes, 16), dtype=torch.uint8, device=device)
+    if ws.dtype != torch.uint8 or ws.numel() < nbytes:
+        raise ValueError(f"workspace must be a uint8 tensor of at least {nbytes} bytes")
+    return ws
+
+
+def sq_calibrate(C: Optional[torch.Tensor], W: torch.Tensor, alpha: float, s: Optional[torch.Tensor] = None,
+                 mx_inout: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                 stream=None) -> torch.Tensor:
+    """Smoothing factor s[K] (fp32) from calibration activations C[R,K] (or
+    only the running max ``mx_inout``) and the weight W[N,K]."""
+    _want(W, "W", torch.bfloat16, 2)
+    N, K = W.shape
+    if C is not None:
+        _want(C, "C", torch.bfloat16, 2)
+        if C.shape[1] != K:
+            raise ValueError(f"C has {C.shape[1]} columns, W has {K}")
+        R = C.shape[0]
+    else:
+        R = 0
+    if mx_inout is not None:
+        _want(mx_inout, "mx_inout", torch.float32, 1)
+        if mx_inout.shape[0] != K:
+            raise ValueError("mx_inout must have K entries")
+    s = _out(s, (K,), torch.float32, W.device, "s")
+    ws = _workspace(workspace, sq_calibrate_workspace_bytes(K), W.device)
+    _check(lib.sq_calibrate(_ptr(C), R, K, _ptr(W), N, float(alpha), _ptr(s), _ptr(mx_inout), _ptr(ws),
+                            ws.numel(), _stream(stream)))
+    return s
+
+
+def sq_prepare_weight(W: torch.Tensor, s: torch.Tensor, Wq: Optional[torch.Tensor] = None,
+                      w_scale: Optional[torch.Tensor] = None, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """(Wq[N,K] int8, w_scale[N] fp32) from W[N,K] bf16 and s[K]."""
+    _want(W, "W", torch.bfloat16, 2)
+    _want(s, "s", torch.float32, 1)
+    N, K = W.shape
+    if s.shape[0] != K:
+        raise ValueError("s must have K entries")
+    Wq = _out(Wq, (N, K), torch.int8, W.device, "Wq")
+    w_scale = _out(w_scale, (N,), torch.float32, W.device, "w_scale")
+    _check(lib.sq_prepare_weight(_ptr(W), N, K, _ptr(s), _ptr(Wq), _ptr(w_scale), _stream(stream)))
+    return Wq, w_scale
+
+
+def sq_quantize_act(X: torch.Tensor, s: torch.Tensor, Xq: Optional[torch.Tensor] = None,
+                    x_scale: Optional[torch.Tensor] = None, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """(Xq[M,K] int8, x_scale[M] fp32) from X[M,K] bf16 and s[K]."""
+    _want(X, "X", torch.bfloat16, 2)
+    _want(s, "s", torch.float32, 1)
+    M, K = X.shape
+    if s.shape[0] != K:
+        raise ValueError("s must have K entries")
+    Xq = _out(Xq, (M, K), torch.int8, X.device, "Xq")
+    x_scale = _out(x_scale, (M,), torch.float32, X.device, "x_scale")
+    _check(lib.sq_quantize_act(_ptr(X), M, K, _ptr(s), _ptr(Xq), _ptr(x_scale), _stream(stream)))
+    return Xq, x_scale
+
+
+def sq_linear(Xq: torch.Tensor, x_scale: torch.Tensor, Wq: torch.Tensor, w_scale: torch.Tensor,
+              bias: Optional[torch.Tensor] = None, Y: Optional[torch.Tensor] = None,
+              workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Y[M,N] bf16 = bf16((Xq Wq^T) * x_scale[m] * w_scale[n] + bias[n])."""
+    _want(Xq, "Xq", torch.int8, 2)
+    _want(Wq, "Wq", torch.int8, 2)
+    _want(x_scale, "x_scale", torch.float32, 1)
+    _want(w_scale, "w_scale", torch.float32, 1)
+    M, K = Xq.shape
+    N = Wq.shape[0]
+    if Wq.shape[1] != K or x_scale.shape[0] != M or w_scale.shape[0] != N:
+        raise ValueError("inconsistent shapes")
+    if bias is not None:
+        _want(bias, "bias", torch.bfloat16, 1)
+        if bias.shape[0] != N:
+            raise ValueError("bias must have N entries")
+    Y = _out(Y, (M, N), torch.bfloat16, Xq.device, "Y")
+    nbytes = sq_workspace_bytes(M, N, K)
+    ws = _workspace(workspace, nbytes, Xq.device) if nbytes else workspace
+    _check(lib.sq_linear(_ptr(Xq), _ptr(x_scale), _ptr(Wq), _ptr(w_scale), _ptr(bias), M, N, K, _ptr(Y),
+                         _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)))
+    return Y
+
+
+def sq_forward(X: torch.Tensor, s: torch.Tensor, Wq: torch.Tensor, w_scale: torch.Tensor,
+               bias: Optional[torch.Tensor] = None, Y: Optional[torch.Tensor] = None,
+               workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Y[M,N] bf16 from X[M,K] bf16: per-token quantisation of X/s, int8 GEMM,
+    dequant + bias, all in the library's kernels."""
+    _want(X, "X", torch.bfloat16, 2)
+    _want(s, "s", torch.float32, 1)
+    _want(Wq, "Wq", torch.int8, 2)
+    _want(w_scale, "w_scale", torch.float32, 1)
+    M, K = X.shape
+    N = Wq.shape[0]
+    if Wq.shape[1] != K or s.shape[0] != K or w_scale.shape[0] != N:
+        raise ValueError("inconsistent shapes")
+    if bias is not None:
+        _want(bias, "bias", torch.bfloat16, 1)
+        if bias.shape[0] != N:
+            raise ValueError("bias must have N entries")
+    Y = _out(Y, (M, N), torch.bfloat16, X.device, "Y")
+    ws = _workspace(workspace, sq_forward_workspace_bytes(M, N, K), X.device)
+    _check(lib.sq_forward(_ptr(X), _ptr(s), _ptr(Wq), _ptr(w_scale), _ptr(bias), M, N, K, _ptr(Y), _ptr(ws),
+                          ws.numel(), _stream(stream)))
+    return Y
+
+
+def sq_gemm_s32(Xq: torch.Tensor, Wq: torch.Tensor, acc: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """acc[M,N] int32 = Xq Wq^T on the tensor cores (accumulator exposed for tests)."""
+    _want(Xq, "Xq", torch.int8, 2)
+    _want(Wq, "Wq", torch.int8, 2)
+    M, K = Xq.shape
+    N = Wq.shape[0]
+    if Wq.shape[1] != K:
+        raise ValueError("inconsistent K")
+    acc = _out(acc, (M, N), torch.int32, Xq.device, "acc")
+    _check(lib.sq_gemm_s32(_ptr(Xq), _ptr(Wq), M, N, K, _ptr(acc), _stream(stream)))
+    return acc
+
+
+def sq_device_status(clear: bool = False) -> int:
+    """Device status flags (bit 0: a GEMM pipeline wait timed out).  Syncs the device."""
+    v = ctypes.c_uint32(0)
+    st = lib.sq_device_status(ctypes.byref(v), 1 if clear else 0)
+    if st not in (0, 7):
+        _check(st)
+    return int(v.value)
+
+
+def sq_debug_fail_after(n: int) -> None:
+    """Host-side fault injection: after n more launches, entry points fail with SQ_ERR_CUDA."""
+    lib.sq_debug_fail_after(int(n))

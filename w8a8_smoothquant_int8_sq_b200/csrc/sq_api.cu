@@ -1,0 +1,295 @@
+// sq_api.cu -- the C ABI of libsq: argument validation, workspace carving,
+// launch, status codes.  Declarations and contracts: include/sq.h.
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstdio>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "../../include/sq.h"
+#include "sq_internal.h"
+
+namespace sq {
+
+// ------------------------------------------------------------ device info
+cudaError_t current_device_info(DeviceInfo* out) {
+  static std::mutex mu;
+  static std::vector<DeviceInfo> cache;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lk(mu);
+  if (dev < static_cast<int>(cache.size()) && cache[dev].device == dev) {
+    *out = cache[dev];
+    return cudaSuccess;
+  }
+  DeviceInfo d;
+  d.device = dev;
+  if ((e = cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&d.major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&d.minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess) return e;
+  int smem = 0;
+  if ((e = cudaDeviceGetAttribute(&smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess) return e;
+  d.max_smem_optin = static_cast<size_t>(smem);
+  if (static_cast<int>(cache.size()) <= dev) cache.resize(dev + 1);
+  cache[dev] = d;
+  *out = d;
+  return cudaSuccess;
+}
+
+}  // namespace sq
+
+namespace {
+
+thread_local std::string g_last_error;
+std::atomic<int> g_fail_after{-1};
+
+constexpr int64_t kMaxGemmK = 133143;  // 127^2 * K must stay below 2^31
+
+sq_status fail(sq_status st, const std::string& msg) {
+  g_last_error = std::string(sq_status_string(st)) + ": " + msg;
+  return st;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Host-side fault injection: consume one "launch credit".
+bool injected_failure() {
+  int cur = g_fail_after.load();
+  while (cur >= 0) {
+    if (cur == 0) return true;
+    if (g_fail_after.compare_exchange_weak(cur, cur - 1)) return false;
+  }
+  return false;
+}
+
+sq_status prologue(sq::DeviceInfo* dev) {
+  cudaError_t e = sq::current_device_info(dev);
+  if (e != cudaSuccess) return fail(SQ_ERR_CUDA, std::string("device query: ") + cudaGetErrorString(e));
+  if (dev->major != 10)
+    return fail(SQ_ERR_UNSUPPORTED, "libsq needs an sm_100 device (compute capability 10.x); found " +
+                                        std::to_string(dev->major) + "." + std::to_string(dev->minor));
+  if (injected_failure()) return fail(SQ_ERR_CUDA, "injected failure (sq_debug_fail_after)");
+  return SQ_OK;
+}
+
+sq_status cuda_status(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return SQ_OK;
+  return fail(SQ_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
+}
+
+sq_status check_k(int64_t K, int64_t kmax) {
+  if (K < 16 || K > kmax) return fail(SQ_ERR_SHAPE, "K=" + std::to_string(K) + " outside [16, " + std::to_string(kmax) + "]");
+  if (K % 16 != 0) return fail(SQ_ERR_ALIGN, "K=" + std::to_string(K) + " is not a multiple of 16");
+  return SQ_OK;
+}
+
+sq_status check_rows(int64_t v, const char* name, int64_t lo = 1) {
+  if (v < lo || v > INT32_MAX) return fail(SQ_ERR_SHAPE, std::string(name) + "=" + std::to_string(v) + " out of range");
+  return SQ_OK;
+}
+
+#define SQ_TRY(x)                 \
+  do {                            \
+    sq_status _st = (x);          \
+    if (_st != SQ_OK) return _st; \
+  } while (0)
+
+#define SQ_NONNULL(p)                                                       \
+  do {                                                                      \
+    if ((p) == nullptr) return fail(SQ_ERR_NULL, #p " is NULL");            \
+    if (!aligned16(p)) return fail(SQ_ERR_ALIGN, #p " is not 16-byte aligned"); \
+  } while (0)
+
+size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+}  // namespace
+
+extern "C" {
+
+int sq_version(void) { return 100; }
+
+const char* sq_last_error(void) { return g_last_error.c_str(); }
+
+const char* sq_status_string(sq_status st) {
+  switch (st) {
+    case SQ_OK: return "SQ_OK";
+    case SQ_ERR_NULL: return "SQ_ERR_NULL";
+    case SQ_ERR_SHAPE: return "SQ_ERR_SHAPE";
+    case SQ_ERR_ALIGN: return "SQ_ERR_ALIGN";
+    case SQ_ERR_ARG: return "SQ_ERR_ARG";
+    case SQ_ERR_UNSUPPORTED: return "SQ_ERR_UNSUPPORTED";
+    case SQ_ERR_CUDA: return "SQ_ERR_CUDA";
+    case SQ_ERR_TIMEOUT: return "SQ_ERR_TIMEOUT";
+    case SQ_ERR_WORKSPACE: return "SQ_ERR_WORKSPACE";
+  }
+  return "SQ_ERR_UNKNOWN";
+}
+
+void sq_debug_fail_after(int n) { g_fail_after.store(n < 0 ? -1 : n); }
+
+// ------------------------------------------------------------ calibration
+size_t sq_calibrate_workspace_bytes(int64_t K) {
+  if (K <= 0) return 0;
+  return round_up(static_cast<size_t>(2 * K) * sizeof(uint32_t), 256);
+}
+
+sq_status sq_calibrate(const sq_bf16* C, int64_t R, int64_t K, const sq_bf16* W, int64_t N, float alpha, float* s,
+                       float* mx_inout, void* workspace, size_t workspace_bytes, void* stream) {
+  SQ_TRY(check_k(K, INT32_MAX - 15));
+  SQ_TRY(check_rows(N, "N"));
+  SQ_TRY(check_rows(R, "R", 0));
+  if (!(alpha >= 0.0f && alpha <= 1.0f)) return fail(SQ_ERR_ARG, "alpha must lie in [0, 1]");
+  if (R > 0) SQ_NONNULL(C);
+  if (R == 0 && mx_inout == nullptr) return fail(SQ_ERR_NULL, "R == 0 needs the running max mx_inout");
+  SQ_NONNULL(W);
+  SQ_NONNULL(s);
+  if (mx_inout != nullptr && !aligned16(mx_inout)) return fail(SQ_ERR_ALIGN, "mx_inout is not 16-byte aligned");
+  if (workspace == nullptr || workspace_bytes < sq_calibrate_workspace_bytes(K))
+    return fail(SQ_ERR_WORKSPACE, "workspace must hold sq_calibrate_workspace_bytes(K) = " +
+                                      std::to_string(sq_calibrate_workspace_bytes(K)) + " bytes");
+  if (!aligned16(workspace)) return fail(SQ_ERR_ALIGN, "workspace is not 16-byte aligned");
+  sq::DeviceInfo dev;
+  SQ_TRY(prologue(&dev));
+  return cuda_status(sq::launch_calibrate(C, R, K, W, N, alpha, s, mx_inout, workspace,
+                                          static_cast<cudaStream_t>(stream), dev),
+                     "calibrate launch");
+}
+
+// ---------------------------------------------------------- weight prepare
+sq_status sq_prepare_weight(const sq_bf16* W, int64_t N, int64_t K, const float* s, int8_t* Wq, float* w_scale,
+                            void* stream) {
+  SQ_TRY(check_k(K, sq::kMaxQuantK));
+  SQ_TRY(check_rows(N, "N"));
+  SQ_NONNULL(W);
+  SQ_NONNULL(s);
+  SQ_NONNULL(Wq);
+  SQ_NONNULL(w_scale);
+  sq::DeviceInfo dev;
+  SQ_TRY(prologue(&dev));
+  return cuda_status(sq::launch_row_quant(true, W, N, K, s, Wq, w_scale, static_cast<cudaStream_t>(stream), dev),
+                     "prepare_weight launch");
+}
+
+// -------------------------------------------------------- activation quant
+sq_status sq_quantize_act(const sq_bf16* X, int64_t M, int64_t K, const float* s, int8_t* Xq, float* x_scale,
+                          void* stream) {
+  SQ_TRY(check_k(K, sq::kMaxQuantK));
+  SQ_TRY(check_rows(M, "M"));
+  SQ_NONNULL(X);
+  SQ_NONNULL(s);
+  SQ_NONNULL(Xq);
+  SQ_NONNULL(x_scale);
+  sq::DeviceInfo dev;
+  SQ_TRY(prologue(&dev));
+  return cuda_status(sq::launch_row_quant(false, X, M, K, s, Xq, x_scale, static_cast<cudaStream_t>(stream), dev),
+                     "quantize_act launch");
+}
+
+// ------------------------------------------------------------- int8 linear
+size_t sq_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  (void)M;
+  (void)N;
+  (void)K;
+  return 0;
+}
+
+static sq_status gemm_common(const int8_t* Xq, const float* x_scale, const int8_t* Wq, const float* w_scale,
+                             const sq_bf16* bias, int64_t M, int64_t N, int64_t K, void* out, sq::Epilogue epi,
+                             void* stream, const sq::DeviceInfo& dev) {
+  sq::GemmArgs a;
+  a.A = Xq;
+  a.B = Wq;
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.x_scale = x_scale;
+  a.w_scale = w_scale;
+  a.bias = bias;
+  a.out = out;
+  a.epi = epi;
+  const char* why = "kernel launch";
+  cudaError_t e = sq::launch_gemm(a, static_cast<cudaStream_t>(stream), dev, &why);
+  return cuda_status(e, why);
+}
+
+sq_status sq_linear(const int8_t* Xq, const float* x_scale, const int8_t* Wq, const float* w_scale,
+                    const sq_bf16* bias, int64_t M, int64_t N, int64_t K, sq_bf16* Y, void* workspace,
+                    size_t workspace_bytes, void* stream) {
+  SQ_TRY(check_k(K, kMaxGemmK));
+  SQ_TRY(check_rows(M, "M"));
+  SQ_TRY(check_rows(N, "N"));
+  SQ_NONNULL(Xq);
+  SQ_NONNULL(x_scale);
+  SQ_NONNULL(Wq);
+  SQ_NONNULL(w_scale);
+  SQ_NONNULL(Y);
+  if (bias != nullptr && !aligned16(bias)) return fail(SQ_ERR_ALIGN, "bias is not 16-byte aligned");
+  if (workspace_bytes < sq_workspace_bytes(M, N, K))
+    return fail(SQ_ERR_WORKSPACE, "workspace smaller than sq_workspace_bytes(M, N, K)");
+  (void)workspace;
+  sq::DeviceInfo dev;
+  SQ_TRY(prologue(&dev));
+  return gemm_common(Xq, x_scale, Wq, w_scale, bias, M, N, K, Y, sq::Epilogue::kBf16Dequant, stream, dev);
+}
+
+// ----------------------------------------------------------- fused forward
+static size_t forward_xq_bytes(int64_t M, int64_t K) { return round_up(static_cast<size_t>(M * K), 256); }
+
+size_t sq_forward_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  if (M <= 0 || K <= 0) return 0;
+  return forward_xq_bytes(M, K) + round_up(static_cast<size_t>(M) * sizeof(float), 256) + sq_workspace_bytes(M, N, K);
+}
+
+sq_status sq_forward(const sq_bf16* X, const float* s, const int8_t* Wq, const float* w_scale, const sq_bf16* bias,
+                     int64_t M, int64_t N, int64_t K, sq_bf16* Y, void* workspace, size_t workspace_bytes,
+                     void* stream) {
+  SQ_TRY(check_k(K, sq::kMaxQuantK));
+  SQ_TRY(check_rows(M, "M"));
+  SQ_TRY(check_rows(N, "N"));
+  SQ_NONNULL(X);
+  SQ_NONNULL(s);
+  SQ_NONNULL(Wq);
+  SQ_NONNULL(w_scale);
+  SQ_NONNULL(Y);
+  if (bias != nullptr && !aligned16(bias)) return fail(SQ_ERR_ALIGN, "bias is not 16-byte aligned");
+  if (workspace == nullptr || workspace_bytes < sq_forward_workspace_bytes(M, N, K))
+    return fail(SQ_ERR_WORKSPACE, "workspace must hold sq_forward_workspace_bytes(M, N, K) = " +
+                                      std::to_string(sq_forward_workspace_bytes(M, N, K)) + " bytes");
+  if (!aligned16(workspace)) return fail(SQ_ERR_ALIGN, "workspace is not 16-byte aligned");
+  sq::DeviceInfo dev;
+  SQ_TRY(prologue(&dev));
+  int8_t* Xq = static_cast<int8_t*>(workspace);
+  float* xs = reinterpret_cast<float*>(static_cast<char*>(workspace) + forward_xq_bytes(M, K));
+  sq_status st = cuda_status(
+      sq::launch_row_quant(false, X, M, K, s, Xq, xs, static_cast<cudaStream_t>(stream), dev), "quantize_act launch");
+  if (st != SQ_OK) return st;
+  return gemm_common(Xq, xs, Wq, w_scale, bias, M, N, K, Y, sq::Epilogue::kBf16Dequant, stream, dev);
+}
+
+// ---------------------------------------------------------------- test hook
+sq_status sq_gemm_s32(const int8_t* Xq, const int8_t* Wq, int64_t M, int64_t N, int64_t K, int32_t* acc,
+                      void* stream) {
+  SQ_TRY(check_k(K, kMaxGemmK));
+  SQ_TRY(check_rows(M, "M"));
+  SQ_TRY(check_rows(N, "N"));
+  SQ_NONNULL(Xq);
+  SQ_NONNULL(Wq);
+  SQ_NONNULL(acc);
+  sq::DeviceInfo dev;
+  SQ_TRY(prologue(&dev));
+  return gemm_common(Xq, nullptr, Wq, nullptr, nullptr, M, N, K, acc, sq::Epilogue::kS32, stream, dev);
+}
+
+// ------------------------------------------------------------ device status
+sq_status sq_device_status(uint32_t* flags, int clear) {
+  if (flags == nullptr) return fail(SQ_ERR_NULL, "flags is NULL");
+  cudaError_t e = sq::read_device_status(flags, clear != 0);
+  if (e != cudaSuccess) return cuda_status(e, "device status read");
+  if (*flags != 0u) return fail(SQ_ERR_TIMEOUT, "a device-side pipeline wait timed out");
+  return SQ_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,411 @@
+// sq_gemm.cu -- int8 x int8 -> int32 GEMM on the sm_100a tensor cores with the
+// SmoothQuant dequantising epilogue.
+//
+// Page: "w8a8_smoothquant.py -- W8A8 com SmoothQuant e alpha APRENDIVEL (V5)",
+// SmoothQuantW8A8.forward: the product of the quantised activations and
+// weights plus the bias, which on hardware is "INT8 x INT8 -> INT32 -> fp32":
+//     acc[m][n] = sum_k Xq[m][k] * Wq[n][k]
+//     Y[m][n]   = bf16( acc * x_scale[m] * w_scale[n] + bias[n] )
+//
+// Design (one CTA per SM, persistent over output tiles of 128 x BN):
+//   warp 0      TMA producer: 128 x 128-byte K slices of Xq and BN x 128-byte
+//               slices of Wq into a STAGES-deep shared-memory ring (128-byte
+//               swizzle), completion counted on per-stage mbarriers.
+//   warp 1      allocates 2*BN TMEM columns (two int32 accumulators) and issues
+//               tcgen05.mma kind::i8 (M=128, N=BN, K=32) from one thread;
+//               tcgen05.commit frees ring slots and publishes finished tiles.
+//   warps 2..5  epilogue: tcgen05.ld of 32 columns at a time, fp32
+//               dequantisation + bias, bf16 pack, 16-byte stores.  The two TMEM
+//               accumulators let the epilogue of tile i overlap the main loop of
+//               tile i+1.
+// Every mbarrier wait is bounded in time; a timeout latches bit 0 of the device
+// status word, the CTA drains the copies and MMAs it issued, frees its TMEM and
+// returns.
+#include <algorithm>
+#include <cstdint>
+#include <mutex>
+
+#include "sq_device.cuh"
+#include "sq_internal.h"
+
+namespace sq {
+
+__device__ unsigned int g_sq_device_status = 0u;
+
+namespace {
+
+constexpr int kBM = 128;         // MMA M (tile rows of Xq / Y)
+constexpr int kBK = 128;         // K bytes per stage = one 128-byte swizzle row
+constexpr int kUmmaK = 32;       // K per tcgen05.mma kind::i8
+constexpr int kThreads = 192;    // 6 warps
+constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // 2 s per wait
+
+struct KParams {
+  int M, N, K;
+  int num_m_blocks, num_n_blocks, num_k_blocks;
+  const float* x_scale;
+  const float* w_scale;
+  const uint16_t* bias;
+  void* out;
+  int vec_ok;  // 16-byte stores allowed (row pitch and base aligned)
+};
+
+template <int BN, int STAGES>
+struct SmemLayout {
+  static constexpr int kABytes = kBM * kBK;
+  static constexpr int kBBytes = BN * kBK;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kRingBytes = STAGES * kStageBytes;
+  // barriers after the ring
+  static constexpr int kBarOffset = kRingBytes;
+  static constexpr int kNumBars = 2 * STAGES + 4 + 1;  // full, empty, tfull[2], tempty[2], drain
+  static constexpr int kMiscOffset = kBarOffset + kNumBars * 8;
+  static constexpr int kBytes = kMiscOffset + 16;
+  static constexpr int kAlloc = kBytes + 1024;  // manual 1024-byte alignment
+};
+
+__device__ __forceinline__ void flag_timeout(volatile int* abort_flag) {
+  *abort_flag = 1;
+  atomicOr(&g_sq_device_status, 1u);
+}
+
+template <int BN, int STAGES, int EPI>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const KParams p) {
+  using L = SmemLayout<BN, STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOffset);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + STAGES;
+  uint64_t* tfull = bars + 2 * STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOffset);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOffset + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  constexpr uint32_t kTmemCols = 2 * BN;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < STAGES; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&tfull[i], 1);
+      mbar_init(&tempty[i], 4);  // one arrive per epilogue warp
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    __syncwarp();
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int num_tiles = p.num_m_blocks * p.num_n_blocks;
+  const int nk = p.num_k_blocks;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued[STAGES];
+      uint32_t issued_phase[STAGES];
+#pragma unroll
+      for (int i = 0; i < STAGES; ++i) issued[i] = 0, issued_phase[i] = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+        const int m_blk = tile % p.num_m_blocks;
+        const int n_blk = tile / p.num_m_blocks;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (*abort_flag || !mbar_wait_bounded(&empty[stage], phase ^ 1u, kWaitTimeoutNs)) {
+            if (!*abort_flag) flag_timeout(abort_flag);
+            ok = false;
+            break;
+          }
+          uint8_t* sa = smem + stage * L::kStageBytes;
+          uint8_t* sb = sa + L::kABytes;
+          mbar_arrive_expect_tx(&full[stage], L::kStageBytes);
+          tma_load_2d(sa, &tmA, kb * kBK, m_blk * kBM, &full[stage]);
+          tma_load_2d(sb, &tmB, kb * kBK, n_blk * BN, &full[stage]);
+          issued[stage] = 1;
+          issued_phase[stage] = phase;
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        // drain: every copy this thread issued must land before the CTA exits
+#pragma unroll
+        for (int i = 0; i < STAGES; ++i)
+          if (issued[i]) (void)mbar_wait_bounded(&full[i], issued_phase[i], kWaitTimeoutNs);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_i8(kBM, BN);
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x, ++it) {
+        const int acc = it & 1;
+        const uint32_t acc_phase = (it >> 1) & 1;
+        if (*abort_flag || !mbar_wait_bounded(&tempty[acc], acc_phase ^ 1u, kWaitTimeoutNs)) {
+          if (!*abort_flag) flag_timeout(abort_flag);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        for (int kb = 0; kb < nk; ++kb) {
+          if (*abort_flag || !mbar_wait_bounded(&full[stage], phase, kWaitTimeoutNs)) {
+            if (!*abort_flag) flag_timeout(abort_flag);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + stage * L::kStageBytes);
+          const uint32_t sb = sa + L::kABytes;
+          const uint64_t adesc = smem_desc_k_sw128(sa);
+          const uint64_t bdesc = smem_desc_k_sw128(sb);
+#pragma unroll
+          for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
+            // advance the start address by kk * 32 bytes (encoded >> 4) inside the swizzle atom
+            mma_i8(d_tmem, adesc + static_cast<uint64_t>(kk * 2), bdesc + static_cast<uint64_t>(kk * 2), idesc,
+                   (kb | kk) != 0 ? 1u : 0u);
+          }
+          mma_commit(&empty[stage]);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        mma_commit(&tfull[acc]);
+      }
+      // drain: wait until every MMA this thread issued has completed
+      mma_commit(drain);
+      (void)mbar_wait_bounded(drain, 0, kWaitTimeoutNs);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int quarter = warp & 3;  // TMEM lanes [32*quarter, 32*quarter + 32) for this warp
+    int it = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
+      const int acc = it & 1;
+      const uint32_t acc_phase = (it >> 1) & 1;
+      // every lane observes the phase itself; the vote keeps the warp uniform
+      // for the warp-collective tcgen05.ld even if lanes disagree on a timeout
+      const bool mine = !*abort_flag && mbar_wait_bounded(&tfull[acc], acc_phase, kWaitTimeoutNs);
+      if (!__all_sync(0xFFFFFFFFu, mine)) {
+        if (lane == 0 && !*abort_flag) flag_timeout(abort_flag);
+        break;
+      }
+      tc_fence_after();
+      const int m_blk = tile % p.num_m_blocks;
+      const int n_blk = tile / p.num_m_blocks;
+      const int row = m_blk * kBM + quarter * 32 + lane;
+      const bool row_ok = row < p.M;
+      const float xs = (EPI == 0 && row_ok) ? __ldg(p.x_scale + row) : 0.0f;
+      const uint32_t t_base = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * BN);
+#pragma unroll 1
+      for (int c0 = 0; c0 < BN; c0 += 32) {
+        uint32_t r[32];
+        tmem_ld_32cols(t_base + static_cast<uint32_t>(c0), r);
+        tmem_ld_wait();
+        const int n0 = n_blk * BN + c0;
+        if (n0 >= p.N) continue;  // tile overhang past N (warp-uniform)
+        const bool full_chunk = (n0 + 32 <= p.N);
+        const bool vec = full_chunk && p.vec_ok;
+        if (EPI == 0) {
+          float ws[32], bs[32];
+          if (vec) {
+#pragma unroll
+            for (int j = 0; j < 32; j += 4) {
+              const float4 w4 = __ldg(reinterpret_cast<const float4*>(p.w_scale + n0 + j));
+              ws[j] = w4.x, ws[j + 1] = w4.y, ws[j + 2] = w4.z, ws[j + 3] = w4.w;
+            }
+            if (p.bias != nullptr) {
+#pragma unroll
+              for (int j = 0; j < 32; j += 8) {
+                const uint4 b8 = __ldg(reinterpret_cast<const uint4*>(p.bias + n0 + j));
+                bs[j] = bf16_lo(b8.x), bs[j + 1] = bf16_hi(b8.x), bs[j + 2] = bf16_lo(b8.y), bs[j + 3] = bf16_hi(b8.y);
+                bs[j + 4] = bf16_lo(b8.z), bs[j + 5] = bf16_hi(b8.z), bs[j + 6] = bf16_lo(b8.w), bs[j + 7] = bf16_hi(b8.w);
+              }
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j) bs[j] = 0.0f;
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const bool in = n0 + j < p.N;
+              ws[j] = in ? __ldg(p.w_scale + n0 + j) : 0.0f;
+              bs[j] = (in && p.bias != nullptr) ? __uint_as_float(static_cast<uint32_t>(__ldg(p.bias + n0 + j)) << 16)
+                                                : 0.0f;
+            }
+          }
+          uint32_t packed[16];
+#pragma unroll
+          for (int j = 0; j < 32; j += 2) {
+            const float y0 = __fmaf_rn(__int2float_rn(static_cast<int>(r[j])), __fmul_rn(xs, ws[j]), bs[j]);
+            const float y1 = __fmaf_rn(__int2float_rn(static_cast<int>(r[j + 1])), __fmul_rn(xs, ws[j + 1]), bs[j + 1]);
+            packed[j / 2] = pack_bf16x2(y0, y1);
+          }
+          if (row_ok) {
+            uint16_t* yrow = static_cast<uint16_t*>(p.out) + static_cast<int64_t>(row) * p.N + n0;
+            if (vec) {
+              uint4* dst = reinterpret_cast<uint4*>(yrow);
+#pragma unroll
+              for (int j = 0; j < 4; ++j)
+                dst[j] = make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (n0 + j < p.N) yrow[j] = static_cast<uint16_t>(packed[j / 2] >> ((j & 1) * 16));
+            }
+          }
+        } else {
+          if (row_ok) {
+            int32_t* arow = static_cast<int32_t*>(p.out) + static_cast<int64_t>(row) * p.N + n0;
+            if (vec) {
+              uint4* dst = reinterpret_cast<uint4*>(arow);
+#pragma unroll
+              for (int j = 0; j < 8; ++j) dst[j] = make_uint4(r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]);
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (n0 + j < p.N) arow[j] = static_cast<int32_t>(r[j]);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
+    }
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+// ----------------------------------------------------------- host helpers
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// 2-D int8 tensor map over a row-major [rows][K] matrix, box = box_rows x 128 bytes,
+// 128-byte swizzle, zero fill outside the matrix.
+bool make_tmap_i8(CUtensorMap* map, const int8_t* base, int64_t rows, int64_t K, int box_rows) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(K)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(kBK), static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<int8_t*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int BN, int STAGES, int EPI>
+cudaError_t run_gemm(const GemmArgs& a, cudaStream_t st, const DeviceInfo& dev, const char** why) {
+  using L = SmemLayout<BN, STAGES>;
+  CUtensorMap tmA, tmB;
+  if (!make_tmap_i8(&tmA, a.A, a.M, a.K, kBM) || !make_tmap_i8(&tmB, a.B, a.N, a.K, BN)) {
+    *why = "cuTensorMapEncodeTiled failed or unavailable";
+    return cudaErrorInvalidValue;
+  }
+  KParams p;
+  p.M = static_cast<int>(a.M);
+  p.N = static_cast<int>(a.N);
+  p.K = static_cast<int>(a.K);
+  p.num_m_blocks = static_cast<int>((a.M + kBM - 1) / kBM);
+  p.num_n_blocks = static_cast<int>((a.N + BN - 1) / BN);
+  p.num_k_blocks = static_cast<int>((a.K + kBK - 1) / kBK);
+  p.x_scale = a.x_scale;
+  p.w_scale = a.w_scale;
+  p.bias = a.bias;
+  p.out = a.out;
+  const int elem = (EPI == 0) ? 2 : 4;
+  p.vec_ok = ((a.N * elem) % 16 == 0) && (reinterpret_cast<uintptr_t>(a.out) % 16 == 0) &&
+             (reinterpret_cast<uintptr_t>(a.w_scale) % 16 == 0 || EPI != 0) &&
+             (a.bias == nullptr || reinterpret_cast<uintptr_t>(a.bias) % 16 == 0);
+  auto kern = gemm_i8_kernel<BN, STAGES, EPI>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+  if (e != cudaSuccess) {
+    *why = "cudaFuncSetAttribute(MaxDynamicSharedMemorySize) failed";
+    return e;
+  }
+  const int tiles = p.num_m_blocks * p.num_n_blocks;
+  const int grid = std::min(tiles, dev.sm_count);
+  kern<<<grid, kThreads, L::kAlloc, st>>>(tmA, tmB, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t st, const DeviceInfo& dev, const char** why) {
+  // Tile width: 256-column tiles when they still fill the machine, else 128.
+  const int64_t mb = (a.M + kBM - 1) / kBM;
+  const int64_t tiles256 = mb * ((a.N + 255) / 256);
+  const bool wide = tiles256 >= dev.sm_count;
+  if (a.epi == Epilogue::kBf16Dequant) {
+    return wide ? run_gemm<256, 4, 0>(a, st, dev, why) : run_gemm<128, 6, 0>(a, st, dev, why);
+  }
+  return wide ? run_gemm<256, 4, 1>(a, st, dev, why) : run_gemm<128, 6, 1>(a, st, dev, why);
+}
+
+cudaError_t read_device_status(uint32_t* flags, bool clear) {
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return e;
+  unsigned int v = 0;
+  e = cudaMemcpyFromSymbol(&v, g_sq_device_status, sizeof(v));
+  if (e != cudaSuccess) return e;
+  if (clear) {
+    const unsigned int z = 0;
+    e = cudaMemcpyToSymbol(g_sq_device_status, &z, sizeof(z));
+    if (e != cudaSuccess) return e;
+  }
+  *flags = v;
+  return cudaSuccess;
+}
+
+}  // namespace sq

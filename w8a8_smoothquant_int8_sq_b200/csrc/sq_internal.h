@@ -1,0 +1,53 @@
+// sq_internal.h -- launchers shared between the libsq translation units.
+// Arguments are validated by the C ABI layer (sq_api.cu) before these run.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace sq {
+
+// Largest K the row quantisers keep on chip (s and 1/s staged in shared memory,
+// one row per thread block held in registers).
+constexpr int64_t kMaxQuantK = 16384;
+
+struct DeviceInfo {
+  int device = -1;
+  int sm_count = 0;
+  int major = 0, minor = 0;
+  size_t max_smem_optin = 0;
+};
+
+// Cached properties of the current device.
+cudaError_t current_device_info(DeviceInfo* out);
+
+// ---- calibration (sq_quant.cu)
+cudaError_t launch_calibrate(const uint16_t* C, int64_t R, int64_t K, const uint16_t* W, int64_t N, float alpha,
+                             float* s, float* mx_inout, void* ws, cudaStream_t st, const DeviceInfo& dev);
+
+// ---- row quantisers (sq_quant.cu)
+// multiply == true : weight path,   t = fl(w * s_j)
+// multiply == false: activation path, t = fl(x / s_j)
+cudaError_t launch_row_quant(bool multiply, const uint16_t* src, int64_t rows, int64_t K, const float* s,
+                             int8_t* q, float* scale, cudaStream_t st, const DeviceInfo& dev);
+
+// ---- GEMM (sq_gemm.cu)
+enum class Epilogue { kBf16Dequant = 0, kS32 = 1 };
+
+struct GemmArgs {
+  const int8_t* A;          // Xq [M][K]
+  const int8_t* B;          // Wq [N][K]
+  int64_t M, N, K;
+  const float* x_scale;     // [M]   (bf16 epilogue)
+  const float* w_scale;     // [N]   (bf16 epilogue)
+  const uint16_t* bias;     // [N] or null
+  void* out;                // Y bf16 [M][N] or acc int32 [M][N]
+  Epilogue epi;
+};
+cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t st, const DeviceInfo& dev, const char** why);
+
+// Device status word (bit 0: pipeline wait timeout).
+cudaError_t read_device_status(uint32_t* flags, bool clear);
+
+}  // namespace sq
