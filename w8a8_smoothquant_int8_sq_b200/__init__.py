@@ -35,38 +35,52 @@ STATUS = {
     5: "SQ_ERR_UNSUPPORTED", 6: "SQ_ERR_CUDA", 7: "SQ_ERR_TIMEOUT", 8: "SQ_ERR_WORKSPACE",
 }
 
-if not os.path.exists(library_path):
-    raise ImportError(
-        f"libsq.so not found at {library_path}; build it with "
-        "`python -m w8a8_smoothquant_int8_sq_b200.build` (nvcc, sm_100a)")
-lib = ctypes.CDLL(library_path)
-
 _P = ctypes.c_void_p
 _I64 = ctypes.c_int64
 _SZ = ctypes.c_size_t
 
+# (name, restype, argtypes) of every entry point of include/sq.h
+_SIGNATURES = [
+    ("sq_version", ctypes.c_int, ()),
+    ("sq_last_error", ctypes.c_char_p, ()),
+    ("sq_status_string", ctypes.c_char_p, (ctypes.c_int,)),
+    ("sq_calibrate_workspace_bytes", _SZ, (_I64,)),
+    ("sq_calibrate", ctypes.c_int, (_P, _I64, _I64, _P, _I64, ctypes.c_float, _P, _P, _P, _SZ, _P)),
+    ("sq_prepare_weight", ctypes.c_int, (_P, _I64, _I64, _P, _P, _P, _P)),
+    ("sq_quantize_act", ctypes.c_int, (_P, _I64, _I64, _P, _P, _P, _P)),
+    ("sq_workspace_bytes", _SZ, (_I64, _I64, _I64)),
+    ("sq_linear", ctypes.c_int, (_P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _SZ, _P)),
+    ("sq_forward_workspace_bytes", _SZ, (_I64, _I64, _I64)),
+    ("sq_forward", ctypes.c_int, (_P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _SZ, _P)),
+    ("sq_gemm_s32", ctypes.c_int, (_P, _P, _I64, _I64, _I64, _P, _P)),
+    ("sq_device_status", ctypes.c_int, (ctypes.POINTER(ctypes.c_uint32), ctypes.c_int)),
+    ("sq_debug_fail_after", None, (ctypes.c_int,)),
+]
 
-def _sig(name, res, *args):
-    f = getattr(lib, name)
-    f.restype = res
-    f.argtypes = list(args)
-    return f
+_LIB = None
 
 
-_sig("sq_version", ctypes.c_int)
-_sig("sq_last_error", ctypes.c_char_p)
-_sig("sq_status_string", ctypes.c_char_p, ctypes.c_int)
-_sig("sq_calibrate_workspace_bytes", _SZ, _I64)
-_sig("sq_calibrate", ctypes.c_int, _P, _I64, _I64, _P, _I64, ctypes.c_float, _P, _P, _P, _SZ, _P)
-_sig("sq_prepare_weight", ctypes.c_int, _P, _I64, _I64, _P, _P, _P, _P)
-_sig("sq_quantize_act", ctypes.c_int, _P, _I64, _I64, _P, _P, _P, _P)
-_sig("sq_workspace_bytes", _SZ, _I64, _I64, _I64)
-_sig("sq_linear", ctypes.c_int, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _SZ, _P)
-_sig("sq_forward_workspace_bytes", _SZ, _I64, _I64, _I64)
-_sig("sq_forward", ctypes.c_int, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _SZ, _P)
-_sig("sq_gemm_s32", ctypes.c_int, _P, _P, _I64, _I64, _I64, _P, _P)
-_sig("sq_device_status", ctypes.c_int, ctypes.POINTER(ctypes.c_uint32), ctypes.c_int)
-_sig("sq_debug_fail_after", None, ctypes.c_int)
+def _load():
+    """Load libsq.so on first use.  There is no fallback: a missing library is an error."""
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(library_path):
+            raise ImportError(
+                f"libsq.so not found at {library_path}; build it with "
+                "`python -m w8a8_smoothquant_int8_sq_b200.build` (nvcc, sm_100a)")
+        handle = ctypes.CDLL(library_path)
+        for name, res, args in _SIGNATURES:
+            f = getattr(handle, name)
+            f.restype = res
+            f.argtypes = list(args)
+        _LIB = handle
+    return _LIB
+
+
+def __getattr__(name):
+    if name == "lib":
+        return _load()
+    raise AttributeError(name)
 
 
 class SqError(RuntimeError):
@@ -77,7 +91,7 @@ class SqError(RuntimeError):
 
 def _check(st: int) -> None:
     if st != 0:
-        msg = lib.sq_last_error()
+        msg = _load().sq_last_error()
         raise SqError(st, msg.decode() if msg else "")
 
 
@@ -117,19 +131,19 @@ def _out(t, shape, dtype, device, name):
 
 
 def sq_version() -> int:
-    return int(lib.sq_version())
+    return int(_load().sq_version())
 
 
 def sq_calibrate_workspace_bytes(K: int) -> int:
-    return int(lib.sq_calibrate_workspace_bytes(K))
+    return int(_load().sq_calibrate_workspace_bytes(K))
 
 
 def sq_workspace_bytes(M: int, N: int, K: int) -> int:
-    return int(lib.sq_workspace_bytes(M, N, K))
+    return int(_load().sq_workspace_bytes(M, N, K))
 
 
 def sq_forward_workspace_bytes(M: int, N: int, K: int) -> int:
-    return int(lib.sq_forward_workspace_bytes(M, N, K))
+    return int(_load().sq_forward_workspace_bytes(M, N, K))
 
 
 def _workspace(ws, nbytes, device):
@@ -160,7 +174,7 @@ def sq_calibrate(C: Optional[torch.Tensor], W: torch.Tensor, alpha: float, s: Op
             raise ValueError("mx_inout must have K entries")
     s = _out(s, (K,), torch.float32, W.device, "s")
     ws = _workspace(workspace, sq_calibrate_workspace_bytes(K), W.device)
-    _check(lib.sq_calibrate(_ptr(C), R, K, _ptr(W), N, float(alpha), _ptr(s), _ptr(mx_inout), _ptr(ws),
+    _check(_load().sq_calibrate(_ptr(C), R, K, _ptr(W), N, float(alpha), _ptr(s), _ptr(mx_inout), _ptr(ws),
                             ws.numel(), _stream(stream)))
     return s
 
@@ -175,7 +189,7 @@ def sq_prepare_weight(W: torch.Tensor, s: torch.Tensor, Wq: Optional[torch.Tenso
         raise ValueError("s must have K entries")
     Wq = _out(Wq, (N, K), torch.int8, W.device, "Wq")
     w_scale = _out(w_scale, (N,), torch.float32, W.device, "w_scale")
-    _check(lib.sq_prepare_weight(_ptr(W), N, K, _ptr(s), _ptr(Wq), _ptr(w_scale), _stream(stream)))
+    _check(_load().sq_prepare_weight(_ptr(W), N, K, _ptr(s), _ptr(Wq), _ptr(w_scale), _stream(stream)))
     return Wq, w_scale
 
 
@@ -189,7 +203,7 @@ def sq_quantize_act(X: torch.Tensor, s: torch.Tensor, Xq: Optional[torch.Tensor]
         raise ValueError("s must have K entries")
     Xq = _out(Xq, (M, K), torch.int8, X.device, "Xq")
     x_scale = _out(x_scale, (M,), torch.float32, X.device, "x_scale")
-    _check(lib.sq_quantize_act(_ptr(X), M, K, _ptr(s), _ptr(Xq), _ptr(x_scale), _stream(stream)))
+    _check(_load().sq_quantize_act(_ptr(X), M, K, _ptr(s), _ptr(Xq), _ptr(x_scale), _stream(stream)))
     return Xq, x_scale
 
 
@@ -212,7 +226,7 @@ def sq_linear(Xq: torch.Tensor, x_scale: torch.Tensor, Wq: torch.Tensor, w_scale
     Y = _out(Y, (M, N), torch.bfloat16, Xq.device, "Y")
     nbytes = sq_workspace_bytes(M, N, K)
     ws = _workspace(workspace, nbytes, Xq.device) if nbytes else workspace
-    _check(lib.sq_linear(_ptr(Xq), _ptr(x_scale), _ptr(Wq), _ptr(w_scale), _ptr(bias), M, N, K, _ptr(Y),
+    _check(_load().sq_linear(_ptr(Xq), _ptr(x_scale), _ptr(Wq), _ptr(w_scale), _ptr(bias), M, N, K, _ptr(Y),
                          _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)))
     return Y
 
@@ -236,7 +250,7 @@ def sq_forward(X: torch.Tensor, s: torch.Tensor, Wq: torch.Tensor, w_scale: torc
             raise ValueError("bias must have N entries")
     Y = _out(Y, (M, N), torch.bfloat16, X.device, "Y")
     ws = _workspace(workspace, sq_forward_workspace_bytes(M, N, K), X.device)
-    _check(lib.sq_forward(_ptr(X), _ptr(s), _ptr(Wq), _ptr(w_scale), _ptr(bias), M, N, K, _ptr(Y), _ptr(ws),
+    _check(_load().sq_forward(_ptr(X), _ptr(s), _ptr(Wq), _ptr(w_scale), _ptr(bias), M, N, K, _ptr(Y), _ptr(ws),
                           ws.numel(), _stream(stream)))
     return Y
 
@@ -250,14 +264,14 @@ def sq_gemm_s32(Xq: torch.Tensor, Wq: torch.Tensor, acc: Optional[torch.Tensor] 
     if Wq.shape[1] != K:
         raise ValueError("inconsistent K")
     acc = _out(acc, (M, N), torch.int32, Xq.device, "acc")
-    _check(lib.sq_gemm_s32(_ptr(Xq), _ptr(Wq), M, N, K, _ptr(acc), _stream(stream)))
+    _check(_load().sq_gemm_s32(_ptr(Xq), _ptr(Wq), M, N, K, _ptr(acc), _stream(stream)))
     return acc
 
 
 def sq_device_status(clear: bool = False) -> int:
     """Device status flags (bit 0: a GEMM pipeline wait timed out).  Syncs the device."""
     v = ctypes.c_uint32(0)
-    st = lib.sq_device_status(ctypes.byref(v), 1 if clear else 0)
+    st = _load().sq_device_status(ctypes.byref(v), 1 if clear else 0)
     if st not in (0, 7):
         _check(st)
     return int(v.value)
@@ -265,4 +279,4 @@ def sq_device_status(clear: bool = False) -> int:
 
 def sq_debug_fail_after(n: int) -> None:
     """Host-side fault injection: after n more launches, entry points fail with SQ_ERR_CUDA."""
-    lib.sq_debug_fail_after(int(n))
+    _load().sq_debug_fail_after(int(n))
