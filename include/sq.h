@@ -98,6 +98,28 @@ SQ_API sq_status sq_calibrate(const sq_bf16* C, int64_t R, int64_t K,
                        float* s, float* mx_inout,
                        void* workspace, size_t workspace_bytes, void* stream);
 
+/* sq_calibrate_noalloc -- sq_calibrate without a workspace argument.
+ * The SmoothQuant page has no counterpart: this is a library convenience.
+ * It is for callers that cannot hand the library scratch memory: code
+ * embedded in a host engine that owns every device byte through its own
+ * fixed pool and gives plugins no way to call cudaMalloc, or loops where an
+ * allocation (which may block or synchronise the device) is not allowed.
+ *   Arguments and results are those of sq_calibrate, minus the workspace.
+ *   Limit: K <= 16384 (SQ_ERR_SHAPE with a message beyond that).
+ *   Scratch: a fixed 128 KiB device array inside libsq, held by every GPU that
+ *   loads the library until the process exits.  Nothing is allocated per call.
+ *   The first call on each device looks up that array's device address (a
+ *   one-time set-up, made with that device current); make that first call
+ *   before any stream capture on the device.
+ *   All calls on a device share the array: calls that may run at the same time
+ *   on the GPU (different streams without ordering) race and give wrong s.
+ *   Each call clears the part it uses before reducing into it, so one call's
+ *   leftovers never reach the next.
+ */
+SQ_API sq_status sq_calibrate_noalloc(const sq_bf16* C, int64_t R, int64_t K,
+                                      const sq_bf16* W, int64_t N, float alpha,
+                                      float* s, float* mx_inout, void* stream);
+
 /* --------------------------------------------------------- weight prepare
  * sq_prepare_weight -- fold s into W and quantise per output channel.
  * Page: freeze_quantization (W_smooth = weight_fp * s) and

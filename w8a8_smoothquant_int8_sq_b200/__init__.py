@@ -21,7 +21,7 @@ import torch
 
 __all__ = [
     "SqError", "lib", "library_path",
-    "sq_version", "sq_calibrate", "sq_calibrate_workspace_bytes", "sq_prepare_weight",
+    "sq_version", "sq_calibrate", "sq_calibrate_workspace_bytes", "sq_calibrate_noalloc", "sq_prepare_weight",
     "sq_quantize_act", "sq_linear", "sq_workspace_bytes", "sq_forward",
     "sq_forward_workspace_bytes", "sq_gemm_s32", "sq_device_status", "sq_debug_fail_after",
     "STATUS",
@@ -46,6 +46,7 @@ _SIGNATURES = [
     ("sq_status_string", ctypes.c_char_p, (ctypes.c_int,)),
     ("sq_calibrate_workspace_bytes", _SZ, (_I64,)),
     ("sq_calibrate", ctypes.c_int, (_P, _I64, _I64, _P, _I64, ctypes.c_float, _P, _P, _P, _SZ, _P)),
+    ("sq_calibrate_noalloc", ctypes.c_int, (_P, _I64, _I64, _P, _I64, ctypes.c_float, _P, _P, _P)),
     ("sq_prepare_weight", ctypes.c_int, (_P, _I64, _I64, _P, _P, _P, _P)),
     ("sq_quantize_act", ctypes.c_int, (_P, _I64, _I64, _P, _P, _P, _P)),
     ("sq_workspace_bytes", _SZ, (_I64, _I64, _I64)),
@@ -176,6 +177,29 @@ def sq_calibrate(C: Optional[torch.Tensor], W: torch.Tensor, alpha: float, s: Op
     ws = _workspace(workspace, sq_calibrate_workspace_bytes(K), W.device)
     _check(_load().sq_calibrate(_ptr(C), R, K, _ptr(W), N, float(alpha), _ptr(s), _ptr(mx_inout), _ptr(ws),
                             ws.numel(), _stream(stream)))
+    return s
+
+
+def sq_calibrate_noalloc(C: Optional[torch.Tensor], W: torch.Tensor, alpha: float,
+                         s: Optional[torch.Tensor] = None, mx_inout: Optional[torch.Tensor] = None,
+                         stream=None) -> torch.Tensor:
+    """sq_calibrate without scratch from the caller (K <= 16384): for code that
+    cannot give the library device memory.  The library uses a fixed device
+    array of its own; calls that overlap on the GPU race (see include/sq.h).
+    Only ``s`` is allocated here when the caller passes none."""
+    _want(W, "W", torch.bfloat16, 2)
+    N, K = W.shape
+    R = 0
+    if C is not None:
+        _want(C, "C", torch.bfloat16, 2)
+        if C.shape[1] != K:
+            raise ValueError(f"C has {C.shape[1]} columns, W has {K}")
+        R = C.shape[0]
+    if mx_inout is not None:
+        _want(mx_inout, "mx_inout", torch.float32, 1)
+    s = _out(s, (K,), torch.float32, W.device, "s")
+    _check(_load().sq_calibrate_noalloc(_ptr(C), R, K, _ptr(W), N, float(alpha), _ptr(s), _ptr(mx_inout),
+                                    _stream(stream)))
     return s
 
 

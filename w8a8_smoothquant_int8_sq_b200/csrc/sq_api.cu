@@ -158,6 +158,30 @@ sq_status sq_calibrate(const sq_bf16* C, int64_t R, int64_t K, const sq_bf16* W,
                      "calibrate launch");
 }
 
+// For callers that cannot pass scratch memory: the column maxima live in a
+// fixed array inside the library (see include/sq.h for the limits and the
+// sharing rule); nothing is allocated.
+sq_status sq_calibrate_noalloc(const sq_bf16* C, int64_t R, int64_t K, const sq_bf16* W, int64_t N, float alpha,
+                               float* s, float* mx_inout, void* stream) {
+  SQ_TRY(check_k(K, INT32_MAX - 15));
+  if (K > sq::kNoAllocMaxK)
+    return fail(SQ_ERR_SHAPE, "sq_calibrate_noalloc supports K <= " + std::to_string(sq::kNoAllocMaxK) + " (got " +
+                                  std::to_string(K) + "); use sq_calibrate with a workspace");
+  SQ_TRY(check_rows(N, "N"));
+  SQ_TRY(check_rows(R, "R", 0));
+  if (!(alpha >= 0.0f && alpha <= 1.0f)) return fail(SQ_ERR_ARG, "alpha must lie in [0, 1]");
+  if (R > 0) SQ_NONNULL(C);
+  if (R == 0 && mx_inout == nullptr) return fail(SQ_ERR_NULL, "R == 0 needs the running max mx_inout");
+  SQ_NONNULL(W);
+  SQ_NONNULL(s);
+  if (mx_inout != nullptr && !aligned16(mx_inout)) return fail(SQ_ERR_ALIGN, "mx_inout is not 16-byte aligned");
+  sq::DeviceInfo dev;
+  SQ_TRY(prologue(&dev));
+  return cuda_status(sq::launch_calibrate_noalloc(C, R, K, W, N, alpha, s, mx_inout,
+                                                  static_cast<cudaStream_t>(stream), dev),
+                     "calibrate (no-alloc) launch");
+}
+
 // ---------------------------------------------------------- weight prepare
 sq_status sq_prepare_weight(const sq_bf16* W, int64_t N, int64_t K, const float* s, int8_t* Wq, float* w_scale,
                             void* stream) {

@@ -26,6 +26,14 @@ cudaError_t current_device_info(DeviceInfo* out);
 cudaError_t launch_calibrate(const uint16_t* C, int64_t R, int64_t K, const uint16_t* W, int64_t N, float alpha,
                              float* s, float* mx_inout, void* ws, cudaStream_t st, const DeviceInfo& dev);
 
+// Largest K accepted by sq_calibrate_noalloc (its fixed scratch holds 2*K words).
+constexpr int64_t kNoAllocMaxK = 16384;
+
+// Same as launch_calibrate, with the scratch in a fixed device array instead
+// of a caller workspace; looks up that array's address on a device's first call.
+cudaError_t launch_calibrate_noalloc(const uint16_t* C, int64_t R, int64_t K, const uint16_t* W, int64_t N,
+                                     float alpha, float* s, float* mx_inout, cudaStream_t st, const DeviceInfo& dev);
+
 // ---- row quantisers (sq_quant.cu)
 // multiply == true : weight path,   t = fl(w * s_j)
 // multiply == false: activation path, t = fl(x / s_j)

@@ -12,6 +12,7 @@
 // SmoothQuantW8A8.calibrate / freeze_quantization / forward.
 #include <algorithm>
 #include <cstdint>
+#include <mutex>
 
 #include "sq_device.cuh"
 #include "sq_internal.h"
@@ -120,6 +121,37 @@ cudaError_t launch_calibrate(const uint16_t* C, int64_t R, int64_t K, const uint
                                                                                 static_cast<double>(alpha),
                                                                                 mx_inout, s);
   return cudaGetLastError();
+}
+
+// ============================================ calibration without allocation
+// Scratch for sq_calibrate_noalloc: the same 2*K words of column maxima that
+// sq_calibrate keeps in the caller's workspace, here in a fixed array that
+// every device loading the library holds until the process exits (128 KiB).
+// Host code must not pass the symbol itself to a kernel (on the host it only
+// names a stand-in object); the device address comes from cudaGetSymbolAddress.
+static __device__ __align__(256) uint32_t g_calib_noalloc_scratch[2 * kNoAllocMaxK];
+
+cudaError_t launch_calibrate_noalloc(const uint16_t* C, int64_t R, int64_t K, const uint16_t* W, int64_t N,
+                                     float alpha, float* s, float* mx_inout, cudaStream_t st, const DeviceInfo& dev) {
+  // One-time set-up per device, done on that device's first call: look up the
+  // device address of the scratch array while the device is current.
+  static std::mutex mu;
+  static void* addr[64] = {};
+  void* ws = nullptr;
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    if (dev.device < 0 || dev.device >= 64) return cudaErrorInvalidDevice;
+    if (addr[dev.device] == nullptr) {
+      void* p = nullptr;
+      cudaError_t e = cudaGetSymbolAddress(&p, g_calib_noalloc_scratch);
+      if (e != cudaSuccess) return e;
+      addr[dev.device] = p;
+    }
+    ws = addr[dev.device];
+  }
+  // launch_calibrate clears the 2*K words it uses before the reduction, so the
+  // previous call's contents never leak into this one.
+  return launch_calibrate(C, R, K, W, N, alpha, s, mx_inout, ws, st, dev);
 }
 
 // ===================================================== row quantisers (K2/K3)
