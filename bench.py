@@ -11,8 +11,10 @@ workload is the projection-shaped layer: X[512x4096] bf16 with 41 outlier
 channels x50, W[4096x4096] bf16 ~N(0,0.02), no bias, alpha 0.5, calibration
 batch of 512 rows.
 
-Timing: every step is preceded by a 256 MiB write that evicts L2 (the inputs
-are smaller than L2); CUDA events on the launching stream bracket the step and
+Timing: every step is preceded by an L2 flush (the inputs are smaller than
+L2): a 256 MiB write, then a 512 MiB read, so that L2 holds neither the
+step's inputs nor dirty lines whose write-back would land inside the timed
+step.  CUDA events on the launching stream bracket the step and
 each library call inside it; each call is replayed from its own CUDA graph so
 that host launch latency does not leak into the device timeline.  With N > 1
 (one process per GPU under torchrun) every rank runs an independent replica
@@ -45,7 +47,8 @@ import workloads  # noqa: E402
 
 METRIC = "W8A8 linear int8 TOPS & tokens/s at 1 B200; % of INT8 tensor peak / HBM roofline"
 UNIT = "tokens/s"
-FLUSH_BYTES = 256 << 20
+FLUSH_BYTES = 256 << 20        # written before each step
+FLUSH_READ_BYTES = 512 << 20   # then read, leaving L2 clean
 # fallback peaks (only if MEASURED_PEAKS.json is absent)
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
@@ -74,7 +77,7 @@ def workload_config(wl):
                     f"{wl.outliers} outlier channels x{wl.outlier_scale:g}, calibration {wl.R} rows, "
                     f"{'bias' if wl.has_bias else 'no bias'}",
         "M": wl.M, "N": wl.N, "K": wl.K, "R": wl.R,
-        "l2": "flushed before every timed step (256 MiB write); inputs smaller than L2",
+        "l2": "flushed before every timed step (256 MiB write, then 512 MiB read); inputs smaller than L2",
     }
 
 
@@ -260,6 +263,7 @@ def run_ours(args, wl, rank, world, local_rank):
     ws_cal = torch.empty(sq.sq_calibrate_workspace_bytes(K), dtype=torch.uint8, device=dev)
     ws_fwd = torch.empty(max(sq.sq_forward_workspace_bytes(M, N, K), 16), dtype=torch.uint8, device=dev)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush_read = torch.ones(FLUSH_READ_BYTES // 4, dtype=torch.int32, device=dev)
 
     calls = {
         "sq_calibrate": lambda: sq.sq_calibrate(C, W, wl.alpha_f32, s=s, workspace=ws_cal),
@@ -285,6 +289,7 @@ def run_ours(args, wl, rank, world, local_rank):
 
     def step(evs=None):
         flush.fill_(1)
+        flush_read.max()
         if evs is not None:
             evs[0].record(stream)
         for i, n in enumerate(names):

@@ -89,8 +89,8 @@ SQ_API const char* sq_status_string(sq_status st);
  *              With R == 0 it must be non-NULL and s comes from it alone.
  *   workspace  device scratch of at least sq_calibrate_workspace_bytes(K)
  *              bytes, 16-byte aligned; contents on entry are ignored.
- * Launches: one memset of the workspace and two kernels (column max-abs over
- * C and W, then the per-channel finalisation).
+ * Launches: one memset of the workspace and one kernel (column max-abs over
+ * C and W; the last block to finish each 256-column stripe computes s there).
  */
 SQ_API size_t sq_calibrate_workspace_bytes(int64_t K);
 SQ_API sq_status sq_calibrate(const sq_bf16* C, int64_t R, int64_t K,
@@ -106,7 +106,7 @@ SQ_API sq_status sq_calibrate(const sq_bf16* C, int64_t R, int64_t K,
  * allocation (which may block or synchronise the device) is not allowed.
  *   Arguments and results are those of sq_calibrate, minus the workspace.
  *   Limit: K <= 16384 (SQ_ERR_SHAPE with a message beyond that).
- *   Scratch: a fixed 128 KiB device array inside libsq, held by every GPU that
+ *   Scratch: a fixed device array of about 128 KiB inside libsq, held by every GPU that
  *   loads the library until the process exits.  Nothing is allocated per call.
  *   The first call on each device looks up that array's device address (a
  *   one-time set-up, made with that device current); make that first call

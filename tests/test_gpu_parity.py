@@ -89,6 +89,10 @@ def test_workload_stage_parity(sq, name):
     (3, 8, 4096, False),        # tiny N
     (384, 768, 1024, True),     # several full tiles in both dimensions
     (129, 4104, 512, False),    # N just past a 256-wide tile boundary
+    (17, 520, 4112, True),      # few tokens, 32-wide token tile, one split-K rank with no k-blocks
+    (32, 4104, 1024, False),    # largest few-token case, ragged last weight block
+    (8, 4096, 4096, True),      # few tokens, four-way split-K cluster
+    (33, 256, 512, True),       # just above the few-token path
 ])
 def test_ragged_shapes(sq, M, N, K, with_bias):
     rng = np.random.default_rng(M * 7919 + N * 31 + K)

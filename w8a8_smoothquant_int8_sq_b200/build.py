@@ -18,7 +18,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libsq.so")
 SOURCES = ["sq_api.cu", "sq_quant.cu", "sq_gemm.cu"]
-HEADERS = ["sq_device.cuh", "sq_internal.h", os.path.join("..", "..", "include", "sq.h")]
+HEADERS = ["sq_device.cuh", "sq_internal.h", "sq_gemm_small.cuh", os.path.join("..", "..", "include", "sq.h")]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
@@ -40,12 +40,15 @@ def _stale() -> bool:
     return any(os.path.getmtime(d) > t for d in deps if os.path.exists(d))
 
 
-def build(force: bool = False, verbose_ptxas: bool = False) -> str:
-    """Compile every CUDA source into libsq.so (sm_100a).  Returns its path."""
-    if not force and not verbose_ptxas and not _stale():
+def build(force: bool = False, verbose_ptxas: bool = False, out: str = LIB, defines=()) -> str:
+    """Compile every CUDA source into a shared library for sm_100a (libsq.so
+    next to this file by default).  ``defines`` are extra -D tuning macros.
+    Returns the library path."""
+    if out == LIB and not defines and not force and not verbose_ptxas and not _stale():
         return LIB
-    tmp = LIB + ".tmp"
-    cmd = [nvcc()] + ARCH + FLAGS + ["-shared", "-o", tmp] + [os.path.join(CSRC, s) for s in SOURCES]
+    tmp = out + ".tmp"
+    cmd = [nvcc()] + ARCH + FLAGS + [f"-D{d}" for d in defines] + ["-shared", "-o", tmp] + \
+        [os.path.join(CSRC, s) for s in SOURCES]
     if verbose_ptxas:
         cmd[1:1] = ["-Xptxas", "-v"]
     res = subprocess.run(cmd, cwd=CSRC, capture_output=True, text=True)
@@ -53,8 +56,8 @@ def build(force: bool = False, verbose_ptxas: bool = False) -> str:
         raise RuntimeError("nvcc failed:\n" + " ".join(cmd) + "\n" + res.stdout + res.stderr)
     if verbose_ptxas:
         sys.stderr.write(res.stdout + res.stderr)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, out)
+    return out
 
 
 if __name__ == "__main__":

@@ -133,7 +133,7 @@ void sq_debug_fail_after(int n) { g_fail_after.store(n < 0 ? -1 : n); }
 // ------------------------------------------------------------ calibration
 size_t sq_calibrate_workspace_bytes(int64_t K) {
   if (K <= 0) return 0;
-  return round_up(static_cast<size_t>(2 * K) * sizeof(uint32_t), 256);
+  return round_up(sq::calibrate_workspace_words(K) * sizeof(uint32_t), 256);
 }
 
 sq_status sq_calibrate(const sq_bf16* C, int64_t R, int64_t K, const sq_bf16* W, int64_t N, float alpha, float* s,
@@ -256,6 +256,12 @@ sq_status sq_linear(const int8_t* Xq, const float* x_scale, const int8_t* Wq, co
   (void)workspace;
   sq::DeviceInfo dev;
   SQ_TRY(prologue(&dev));
+  if (M <= sq::kSmallMaxM) {  // few tokens: weight-streaming split-K kernel
+    sq::SmallArgs a{nullptr, nullptr, Xq, x_scale, Wq, w_scale, bias, M, N, K, Y};
+    const char* why = "small-M kernel";
+    cudaError_t e = sq::launch_small_m(a, static_cast<cudaStream_t>(stream), dev, &why);
+    if (e != cudaErrorNotSupported) return cuda_status(e, why);
+  }
   return gemm_common(Xq, x_scale, Wq, w_scale, bias, M, N, K, Y, sq::Epilogue::kBf16Dequant, stream, dev);
 }
 
@@ -285,6 +291,12 @@ sq_status sq_forward(const sq_bf16* X, const float* s, const int8_t* Wq, const f
   if (!aligned16(workspace)) return fail(SQ_ERR_ALIGN, "workspace is not 16-byte aligned");
   sq::DeviceInfo dev;
   SQ_TRY(prologue(&dev));
+  if (M <= sq::kSmallMaxM) {  // few tokens: quantisation fused into the weight-streaming kernel
+    sq::SmallArgs a{X, s, nullptr, nullptr, Wq, w_scale, bias, M, N, K, Y};
+    const char* why = "fused small-M kernel";
+    cudaError_t e = sq::launch_small_m(a, static_cast<cudaStream_t>(stream), dev, &why);
+    if (e != cudaErrorNotSupported) return cuda_status(e, why);
+  }
   int8_t* Xq = static_cast<int8_t*>(workspace);
   float* xs = reinterpret_cast<float*>(static_cast<char*>(workspace) + forward_xq_bytes(M, K));
   sq_status st = cuda_status(

@@ -45,6 +45,73 @@ __device__ __forceinline__ int rne_clamp_q(float v) {
   return __float_as_int(t) - 0x4B400000;
 }
 
+// round_half_even(v) as an int, for |v| < 2^22 (the fp32 add of 1.5 * 2^23
+// rounds to an integer, ties to even); callers guarantee |v| < 127.5.
+__device__ __forceinline__ int rne_q(float v) {
+  const float t = __fadd_rn(v, 12582912.0f);
+  return __float_as_int(t) - 0x4B400000;
+}
+
+// ------------------------------------------------- packed fp32 pairs (f32x2)
+// sm_100 executes two fp32 lanes per instruction (add/mul/fma .rn.f32x2); each
+// lane rounds exactly like the scalar IEEE operation.  A pair travels as one
+// 64-bit value: low word = first element.
+using f2x = unsigned long long;
+
+__device__ __forceinline__ f2x f2_pack(float lo, float hi) {
+  f2x d;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(lo), "f"(hi));
+  return d;
+}
+__device__ __forceinline__ float f2_lo(f2x v) { return __uint_as_float(static_cast<uint32_t>(v)); }
+__device__ __forceinline__ float f2_hi(f2x v) { return __uint_as_float(static_cast<uint32_t>(v >> 32)); }
+__device__ __forceinline__ f2x f2_mul(f2x a, f2x b) {
+  f2x d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ f2x f2_fma(f2x a, f2x b, f2x c) {
+  f2x d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ f2x f2_add(f2x a, f2x b) {
+  f2x d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+// the two bf16 values of a 32-bit word, widened exactly to an fp32 pair
+__device__ __forceinline__ f2x f2_from_bf16x2(uint32_t w) {
+  return (static_cast<f2x>(w & 0xFFFF0000u) << 32) | static_cast<f2x>(w << 16);
+}
+// a / b per lane, correctly rounded, given nb = -b and rb = RN(1/b) (div_rn)
+__device__ __forceinline__ f2x f2_div_rn(f2x a, f2x nb, f2x rb) {
+  const f2x q0 = f2_mul(a, rb);
+  const f2x r = f2_fma(q0, nb, a);  // a - b*q0, exact
+  return f2_fma(r, rb, q0);
+}
+// max(m, |lo|, |hi|) in one three-input max
+__device__ __forceinline__ float f2_absmax(float m, f2x v) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(m), "f"(fabsf(f2_lo(v))), "f"(fabsf(f2_hi(v))));
+  return d;
+}
+// Round both lanes half-to-even to integers (|v| < 127.5) by adding 1.5*2^23;
+// the low byte of each lane's bit pattern is then its int8 code.
+__device__ __forceinline__ f2x f2_round_codes(f2x v) {
+  return f2_add(v, 0x4B4000004B400000ull);
+}
+// int8 codes of four rounded pairs -> two words of packed bytes (byte permutes)
+__device__ __forceinline__ uint2 pack8_codes(f2x a, f2x b, f2x c, f2x d) {
+  const uint32_t ab = __byte_perm(__byte_perm(static_cast<uint32_t>(a), static_cast<uint32_t>(a >> 32), 0x0040),
+                                  __byte_perm(static_cast<uint32_t>(b), static_cast<uint32_t>(b >> 32), 0x0040),
+                                  0x5410);
+  const uint32_t cd = __byte_perm(__byte_perm(static_cast<uint32_t>(c), static_cast<uint32_t>(c >> 32), 0x0040),
+                                  __byte_perm(static_cast<uint32_t>(d), static_cast<uint32_t>(d >> 32), 0x0040),
+                                  0x5410);
+  return make_uint2(ab, cd);
+}
+
 // pack four int codes (each in -127..127) into one little-endian word of int8
 __device__ __forceinline__ uint32_t pack4_i8(int a, int b, int c, int d) {
   return (uint32_t(a) & 0xFFu) | ((uint32_t(b) & 0xFFu) << 8) | ((uint32_t(c) & 0xFFu) << 16) |
@@ -60,6 +127,17 @@ __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
   return v;
+}
+
+// named barrier `id` (1..15) over `nthreads` threads (a multiple of 32)
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+__device__ __forceinline__ uint32_t cluster_nctarank() {
+  uint32_t n;
+  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(n));
+  return n;
 }
 
 // ------------------------------------------------------------ smem address
@@ -133,6 +211,14 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* m
           smem_u32(smem_dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
       : "memory");
+}
+
+// Prefetch a 2-D tile of a tensor map into L2 (no shared memory, no barrier).
+__device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap* map, int32_t x, int32_t y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(x), "r"(y)
+               : "memory");
 }
 
 // ----------------------------------------------------------------- tcgen05

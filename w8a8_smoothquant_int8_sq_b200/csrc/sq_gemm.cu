@@ -39,6 +39,42 @@ constexpr int kBK = 128;         // K bytes per stage = one 128-byte swizzle row
 constexpr int kUmmaK = 32;       // K per tcgen05.mma kind::i8
 constexpr int kThreads = 192;    // 6 warps
 constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // 2 s per wait
+// Build-time tuning knobs (defaults are the measured best on B200):
+//   SQ_GEMM_PF     k-blocks of L2 prefetch ahead of the shared-memory ring (0: none)
+//   SQ_GEMM_PF_A   1: prefetch the Xq slices too, 0: only the Wq slices
+//   SQ_GEMM_ROTATE 1: start each tile's K loop at a tile-dependent k-block, so
+//                  CTAs that share an operand slice do not all request the same
+//                  lines at the same moment (int32 sums are exact in any order)
+//   SQ_GEMM_BN     0: choose the tile width per problem, else force 128 or 256
+#ifndef SQ_GEMM_PF
+#define SQ_GEMM_PF 0
+#endif
+#ifndef SQ_GEMM_PF_A
+#define SQ_GEMM_PF_A 0
+#endif
+#ifndef SQ_GEMM_ROTATE
+#define SQ_GEMM_ROTATE 0
+#endif
+#ifndef SQ_GEMM_BN
+#define SQ_GEMM_BN 0
+#endif
+#ifndef SQ_GEMM_CHAINS128  // accumulator chains for 128-wide tiles (1 or 2)
+#define SQ_GEMM_CHAINS128 2
+#endif
+constexpr int kPrefetchAhead = SQ_GEMM_PF;
+
+// First k-block of a tile's K loop.
+__device__ __forceinline__ int k_start(int m_blk, int n_blk, int nk) {
+#if SQ_GEMM_ROTATE
+  return static_cast<int>((static_cast<unsigned>(n_blk) * 3u + static_cast<unsigned>(m_blk) * 5u) %
+                          static_cast<unsigned>(nk));
+#else
+  (void)m_blk;
+  (void)n_blk;
+  (void)nk;
+  return 0;
+#endif
+}
 
 struct KParams {
   int M, N, K;
@@ -69,7 +105,7 @@ __device__ __forceinline__ void flag_timeout(volatile int* abort_flag) {
   atomicOr(&g_sq_device_status, 1u);
 }
 
-template <int BN, int STAGES, int EPI>
+template <int BN, int STAGES, int EPI, int CHAINS>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const KParams p) {
@@ -87,7 +123,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  constexpr uint32_t kTmemCols = 2 * BN;
+  // Two accumulator buffers (epilogue of one tile overlaps the next tile's
+  // main loop), each split into CHAINS int32 accumulators that alternate
+  // between consecutive MMAs of a k-block so that they do not wait on each
+  // other's accumulation; the epilogue adds the chains (exact).
+  constexpr uint32_t kTmemCols = 2 * CHAINS * BN;
+  static_assert(kTmemCols <= 512, "TMEM holds 512 columns");
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < STAGES; ++i) {
@@ -130,10 +171,33 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int i = 0; i < STAGES; ++i) issued[i] = 0, issued_phase[i] = 0;
       bool ok = true;
+      // L2 prefetch runs kPrefetchAhead k-blocks ahead of the shared-memory
+      // ring along this CTA's (tile, k-block) sequence, so the ring's loads hit
+      // L2 instead of waiting on DRAM.
+      const int my_tiles = (num_tiles - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) /
+                           static_cast<int>(gridDim.x);
+      const int64_t total = static_cast<int64_t>(my_tiles) * nk;
+      int64_t pf = 0;
+      auto prefetch_upto = [&](int64_t limit) {
+        for (; pf < limit && pf < total; ++pf) {
+          const int t = static_cast<int>(blockIdx.x) + static_cast<int>(pf / nk) * static_cast<int>(gridDim.x);
+          const int mb = t % p.num_m_blocks, nb = t / p.num_m_blocks;
+          int k = static_cast<int>(pf % nk) + k_start(mb, nb, nk);
+          if (k >= nk) k -= nk;
+          if (SQ_GEMM_PF_A) tma_prefetch_l2_2d(&tmA, k * kBK, mb * kBM);
+          tma_prefetch_l2_2d(&tmB, k * kBK, nb * BN);
+        }
+      };
+      if (kPrefetchAhead > 0) prefetch_upto(kPrefetchAhead);
+      int64_t seq = 0;
       for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
         const int m_blk = tile % p.num_m_blocks;
         const int n_blk = tile / p.num_m_blocks;
-        for (int kb = 0; kb < nk; ++kb) {
+        const int k0 = k_start(m_blk, n_blk, nk);
+        for (int kb = 0; kb < nk; ++kb, ++seq) {
+          if (kPrefetchAhead > 0) prefetch_upto(seq + 1 + kPrefetchAhead);
+          int kk = kb + k0;
+          if (kk >= nk) kk -= nk;
           if (*abort_flag || !mbar_wait_bounded(&empty[stage], phase ^ 1u, kWaitTimeoutNs)) {
             if (!*abort_flag) flag_timeout(abort_flag);
             ok = false;
@@ -142,8 +206,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint8_t* sa = smem + stage * L::kStageBytes;
           uint8_t* sb = sa + L::kABytes;
           mbar_arrive_expect_tx(&full[stage], L::kStageBytes);
-          tma_load_2d(sa, &tmA, kb * kBK, m_blk * kBM, &full[stage]);
-          tma_load_2d(sb, &tmB, kb * kBK, n_blk * BN, &full[stage]);
+          tma_load_2d(sa, &tmA, kk * kBK, m_blk * kBM, &full[stage]);
+          tma_load_2d(sb, &tmB, kk * kBK, n_blk * BN, &full[stage]);
           issued[stage] = 1;
           issued_phase[stage] = phase;
           if (++stage == STAGES) {
@@ -175,7 +239,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * CHAINS * BN);
         for (int kb = 0; kb < nk; ++kb) {
           if (*abort_flag || !mbar_wait_bounded(&full[stage], phase, kWaitTimeoutNs)) {
             if (!*abort_flag) flag_timeout(abort_flag);
@@ -190,8 +254,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
             // advance the start address by kk * 32 bytes (encoded >> 4) inside the swizzle atom
-            mma_i8(d_tmem, adesc + static_cast<uint64_t>(kk * 2), bdesc + static_cast<uint64_t>(kk * 2), idesc,
-                   (kb | kk) != 0 ? 1u : 0u);
+            mma_i8(d_tmem + static_cast<uint32_t>((kk % CHAINS) * BN), adesc + static_cast<uint64_t>(kk * 2),
+                   bdesc + static_cast<uint64_t>(kk * 2), idesc, (kb != 0 || kk >= CHAINS) ? 1u : 0u);
           }
           mma_commit(&empty[stage]);
           if (++stage == STAGES) {
@@ -226,12 +290,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int row = m_blk * kBM + quarter * 32 + lane;
       const bool row_ok = row < p.M;
       const float xs = (EPI == 0 && row_ok) ? __ldg(p.x_scale + row) : 0.0f;
-      const uint32_t t_base = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * BN);
+      const uint32_t t_base =
+          tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * CHAINS * BN);
 #pragma unroll 1
       for (int c0 = 0; c0 < BN; c0 += 32) {
         uint32_t r[32];
         tmem_ld_32cols(t_base + static_cast<uint32_t>(c0), r);
         tmem_ld_wait();
+#pragma unroll
+        for (int ch = 1; ch < CHAINS; ++ch) {
+          uint32_t r2[32];
+          tmem_ld_32cols(t_base + static_cast<uint32_t>(ch * BN + c0), r2);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) r[j] += r2[j];
+        }
         const int n0 = n_blk * BN + c0;
         if (n0 >= p.N) continue;  // tile overhang past N (warp-uniform)
         const bool full_chunk = (n0 + 32 <= p.N);
@@ -312,6 +385,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+}  // namespace
+}  // namespace sq
+
+#include "sq_gemm_small.cuh"
+
+namespace sq {
+namespace {
+
 // ----------------------------------------------------------- host helpers
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -345,7 +426,7 @@ bool make_tmap_i8(CUtensorMap* map, const int8_t* base, int64_t rows, int64_t K,
   return r == CUDA_SUCCESS;
 }
 
-template <int BN, int STAGES, int EPI>
+template <int BN, int STAGES, int EPI, int CHAINS>
 cudaError_t run_gemm(const GemmArgs& a, cudaStream_t st, const DeviceInfo& dev, const char** why) {
   using L = SmemLayout<BN, STAGES>;
   CUtensorMap tmA, tmB;
@@ -368,10 +449,12 @@ cudaError_t run_gemm(const GemmArgs& a, cudaStream_t st, const DeviceInfo& dev, 
   p.vec_ok = ((a.N * elem) % 16 == 0) && (reinterpret_cast<uintptr_t>(a.out) % 16 == 0) &&
              (reinterpret_cast<uintptr_t>(a.w_scale) % 16 == 0 || EPI != 0) &&
              (a.bias == nullptr || reinterpret_cast<uintptr_t>(a.bias) % 16 == 0);
-  auto kern = gemm_i8_kernel<BN, STAGES, EPI>;
+  auto kern = gemm_i8_kernel<BN, STAGES, EPI, CHAINS>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, kCarveoutMaxShared);
   if (e != cudaSuccess) {
-    *why = "cudaFuncSetAttribute(MaxDynamicSharedMemorySize) failed";
+    *why = "cudaFuncSetAttribute failed";
     return e;
   }
   const int tiles = p.num_m_blocks * p.num_n_blocks;
@@ -380,18 +463,108 @@ cudaError_t run_gemm(const GemmArgs& a, cudaStream_t st, const DeviceInfo& dev, 
   return cudaGetLastError();
 }
 
+template <int NT, bool kFused>
+cudaError_t run_small(const SmallArgs& a, cudaStream_t st, const DeviceInfo& dev, const char** why) {
+  const int nrb = static_cast<int>((a.N + kSmallRows - 1) / kSmallRows);
+  const int nk = static_cast<int>((a.K + kBK - 1) / kBK);
+  const int smem_cap = static_cast<int>(dev.max_smem_optin) - 1024;
+  const int part_bytes = kSmallRows * NT * 4;
+  const int stage_bytes = kSmallABytes + (kFused ? 0 : NT * kBK);
+  const int fixed = part_bytes + 128 + 9 * NT * 4 + 256 + 16;
+  // split K over a cluster of S CTAs: as many splits as keep one wave of CTAs
+  // (S <= 8, at least two k-blocks each), more if the fused codes would not fit
+  int S = 1;
+  while (S < 8 && static_cast<int64_t>(nrb) * S * 2 <= dev.sm_count && (nk + 2 * S - 1) / (2 * S) >= 2) S *= 2;
+  auto b_bytes_for = [&](int splits) { return kFused ? ((nk + splits - 1) / splits) * NT * kBK : 0; };
+  while (S < 8 && b_bytes_for(S) + fixed + 2 * stage_bytes > smem_cap) S *= 2;
+  const int kps = (nk + S - 1) / S;
+  const int b_bytes = b_bytes_for(S);
+  const int stages = std::min(kSmallMaxStages, (smem_cap - b_bytes - fixed) / stage_bytes);
+  if (stages < 2) {
+    *why = "small-M kernel: K too large for shared memory";
+    return cudaErrorNotSupported;
+  }
+  SmallParams p{};
+  p.M = static_cast<int>(a.M);
+  p.N = static_cast<int>(a.N);
+  p.K = static_cast<int>(a.K);
+  p.nk = nk;
+  p.kb_per_split = kps;
+  p.stages = stages;
+  p.stage_bytes = stage_bytes;
+  p.X = a.X;
+  p.s = a.s;
+  p.x_scale = a.x_scale;
+  p.w_scale = a.w_scale;
+  p.bias = a.bias;
+  p.Y = a.Y;
+  p.b_off = stages * stage_bytes;
+  p.part_off = p.b_off + b_bytes;
+  p.xs_off = p.part_off + part_bytes;
+  p.red_off = p.xs_off + 128;
+  p.bar_off = p.red_off + 9 * NT * 4;
+  p.misc_off = p.bar_off + 256;
+  const int alloc = p.misc_off + 16 + 1024;
+  CUtensorMap tmW, tmX;
+  if (!make_tmap_i8(&tmW, a.Wq, a.N, a.K, kSmallRows) ||
+      (!kFused && !make_tmap_i8(&tmX, a.Xq, a.M, a.K, NT))) {
+    *why = "cuTensorMapEncodeTiled failed or unavailable";
+    return cudaErrorInvalidValue;
+  }
+  if (kFused) tmX = tmW;  // unused
+  auto kern = gemm_small_m_kernel<NT, kFused>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, alloc);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, kCarveoutMaxShared);
+  if (e != cudaSuccess) {
+    *why = "cudaFuncSetAttribute failed";
+    return e;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(S), static_cast<unsigned>(nrb), 1);
+  cfg.blockDim = dim3(kSmallThreads, 1, 1);
+  cfg.dynamicSmemBytes = static_cast<size_t>(alloc);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(S);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, kern, tmW, tmX, p);
+  if (e != cudaSuccess) *why = "cluster launch of the small-M kernel failed";
+  return e;
+}
+
 }  // namespace
+
+cudaError_t launch_small_m(const SmallArgs& a, cudaStream_t st, const DeviceInfo& dev, const char** why) {
+  if (a.M < 1 || a.M > kSmallMaxM) return cudaErrorNotSupported;
+  const bool fused = a.X != nullptr;
+  if (a.M <= 16) return fused ? run_small<16, true>(a, st, dev, why) : run_small<16, false>(a, st, dev, why);
+  return fused ? run_small<32, true>(a, st, dev, why) : run_small<32, false>(a, st, dev, why);
+}
 
 cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t st, const DeviceInfo& dev, const char** why) {
   // Tile width: 256-column tiles when they still fill the machine, else 128.
   const int64_t mb = (a.M + kBM - 1) / kBM;
   const int64_t tiles256 = mb * ((a.N + 255) / 256);
-  const bool wide = tiles256 >= dev.sm_count;
+  const bool wide = SQ_GEMM_BN == 256 || (SQ_GEMM_BN == 0 && tiles256 >= dev.sm_count);
   if (a.epi == Epilogue::kBf16Dequant) {
-    return wide ? run_gemm<256, 4, 0>(a, st, dev, why) : run_gemm<128, 6, 0>(a, st, dev, why);
+    return wide ? run_gemm<256, 4, 0, 1>(a, st, dev, why) : run_gemm<128, 6, 0, SQ_GEMM_CHAINS128>(a, st, dev, why);
   }
-  return wide ? run_gemm<256, 4, 1>(a, st, dev, why) : run_gemm<128, 6, 1>(a, st, dev, why);
+  return wide ? run_gemm<256, 4, 1, 1>(a, st, dev, why) : run_gemm<128, 6, 1, SQ_GEMM_CHAINS128>(a, st, dev, why);
 }
+
+#ifdef SQ_TRACE
+extern "C" __attribute__((visibility("default"))) int sq_trace_read(unsigned long long* host, int n) {
+  return cudaMemcpyFromSymbol(host, g_small_trace, sizeof(unsigned long long) * 8 * static_cast<size_t>(n)) ==
+                 cudaSuccess
+             ? 0
+             : 1;
+}
+#endif
 
 cudaError_t read_device_status(uint32_t* flags, bool clear) {
   cudaError_t e = cudaDeviceSynchronize();

@@ -1,0 +1,454 @@
+// sq_gemm_small.cuh -- the int8 linear for few tokens (M <= 32), optionally with
+// the per-token activation quantisation fused in.  Included by sq_gemm.cu (one
+// translation unit: it shares the device status word and the host helpers).
+//
+// Page: "w8a8_smoothquant.py -- W8A8 com SmoothQuant e alpha APRENDIVEL (V5)",
+// SmoothQuantW8A8.forward (X / s, per-token quantisation, int8 product,
+// dequantisation and bias).  With few tokens the layer is a stream of the int8
+// weight: the kernel is built to read Wq from HBM once, at full bandwidth.
+//
+//   * swap-AB: the MMA's M = 128 rows of Wq, its N = the tokens padded to
+//     NT = 16 or 32 (tcgen05.mma kind::i8, M=128, N=NT, K=32).  A CTA owns
+//     256 rows of Wq, fetched as one 256-row x 128-byte TMA box per stage
+//     (large boxes stream HBM markedly faster than 128-row ones) and fed to the
+//     tensor core as two 128-row halves with their own accumulators.  An M=128
+//     int8 MMA costs about the same whatever its N, so the tensor core takes
+//     about 4 KB of Wq per MMA; spreading the rows over ~128 CTAs keeps that
+//     above the HBM rate.
+//   * split-K over a thread-block cluster of S CTAs: each CTA streams its
+//     share of the row block's K; the S partial int32 accumulators are summed
+//     through distributed shared memory at the end, every rank reducing a
+//     share of the rows (exact, no global scratch).
+//   * prequantised codes (sq_linear): the codes travel by TMA in the same
+//     stage as the weight box (NT-row box, rows past M zero-filled), so the
+//     first MMA waits only for the first stage.
+//   * fused quantisation (sq_forward): eight warps quantise this CTA's K-slice
+//     of X / s (correctly rounded fp32 division, as sq_quantize_act).  The
+//     per-token maxima over the whole row are assembled from the S ranks'
+//     slice maxima through distributed shared memory at a mid-kernel cluster
+//     barrier; the codes then go straight into the shared-memory B operand in
+//     the 128-byte-swizzled K-major layout the tensor core reads.
+//
+// Warps: 0 TMA producer, 1 TMEM owner + MMA issuer, 2..9 quantisation and
+// reduction (2..5 also drain TMEM: lane quarters 2, 3, 0, 1).  Every mbarrier
+// wait is bounded; every thread reaches every cluster barrier.
+
+namespace sq {
+namespace {
+
+constexpr int kSmallThreads = 320;
+constexpr int kSmallQuantThreads = 256;  // warps 2..9
+constexpr int kSmallMaxStages = 8;
+constexpr int kSmallRows = 2 * kBM;             // Wq rows per CTA (two MMA halves)
+constexpr int kSmallABytes = kSmallRows * kBK;  // 256 rows of Wq x 128 bytes of K
+
+struct SmallParams {
+  int M, N, K;
+  int nk;            // k-blocks of 128 bytes over K
+  int kb_per_split;  // k-blocks per cluster rank
+  int stages;
+  int stage_bytes;   // Wq box (+ codes box when prequantised)
+  const uint16_t* X;     // fused: bf16 activations [M][K]
+  const float* s;        // fused: smoothing factor [K]
+  const float* x_scale;  // prequantised scales [M]
+  const float* w_scale;  // [N]
+  const uint16_t* bias;  // [N] or null
+  uint16_t* Y;           // [M][N]
+  // shared-memory layout (bytes from the 1024-aligned base)
+  int b_off, part_off, xs_off, red_off, bar_off, misc_off;
+};
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire;" ::: "memory"); }
+__device__ __forceinline__ uint32_t map_cluster_rank(uint32_t smem_addr, uint32_t rank) {
+  uint32_t d;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(d) : "r"(smem_addr), "r"(rank));
+  return d;
+}
+__device__ __forceinline__ uint4 ld_cluster_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared::cluster.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
+__device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
+}
+
+// Byte offset of code (token m, local column c) in the B operand: k-block
+// c/128 holds NT rows of 128 bytes in 8-row atoms of 1024 bytes, each row's
+// 16-byte chunks permuted by XOR with (row % 8) -- the layout a TMA load with
+// 128-byte swizzle produces and the descriptor's 128-byte swizzle mode reads.
+template <int NT>
+__device__ __forceinline__ uint32_t b_code_offset(int m, int c) {
+  const int j = c >> 7, b = c & 127;
+  return static_cast<uint32_t>(j * (NT * 128) + (m >> 3) * 1024 + (m & 7) * 128 + (((b >> 4) ^ (m & 7)) << 4) +
+                               (b & 15));
+}
+
+#ifdef SQ_TRACE
+// Optional phase timestamps (build with -DSQ_TRACE): per CTA, globaltimer at
+// 0 start, 1 codes ready, 2 first stage consumed, 3 last MMA issued,
+// 4 accumulators read, 5 after the reduction barrier, 6 end.
+__device__ unsigned long long g_small_trace[1024][8];
+#define SQ_TRACE_MARK(i)                                        \
+  do {                                                          \
+    const int cta_ = blockIdx.y * gridDim.x + blockIdx.x;       \
+    if (cta_ < 1024) g_small_trace[cta_][i] = globaltimer_ns(); \
+  } while (0)
+#else
+#define SQ_TRACE_MARK(i) \
+  do {                   \
+  } while (0)
+#endif
+
+// fl(x / s) for the 8 columns of one 16-byte bf16 vector, as four fp32 pairs
+__device__ __forceinline__ void smooth8(const uint4 w, const f2x (&ns)[4], const f2x (&rs)[4], f2x (&t)[4]) {
+  t[0] = f2_div_rn(f2_from_bf16x2(w.x), ns[0], rs[0]);
+  t[1] = f2_div_rn(f2_from_bf16x2(w.y), ns[1], rs[1]);
+  t[2] = f2_div_rn(f2_from_bf16x2(w.z), ns[2], rs[2]);
+  t[3] = f2_div_rn(f2_from_bf16x2(w.w), ns[3], rs[3]);
+}
+// -s and RN(1/s) for the 8 columns of vector v, as fp32 pairs
+__device__ __forceinline__ void load_s8(const float4* s4, int v, f2x (&ns)[4], f2x (&rs)[4]) {
+  const float4 a = __ldg(s4 + 2 * v), b = __ldg(s4 + 2 * v + 1);
+  ns[0] = f2_pack(-a.x, -a.y), ns[1] = f2_pack(-a.z, -a.w), ns[2] = f2_pack(-b.x, -b.y), ns[3] = f2_pack(-b.z, -b.w);
+  rs[0] = f2_pack(__frcp_rn(a.x), __frcp_rn(a.y)), rs[1] = f2_pack(__frcp_rn(a.z), __frcp_rn(a.w));
+  rs[2] = f2_pack(__frcp_rn(b.x), __frcp_rn(b.y)), rs[3] = f2_pack(__frcp_rn(b.z), __frcp_rn(b.w));
+}
+
+template <int NT, bool kFused>
+__global__ void __launch_bounds__(kSmallThreads, 1)
+    gemm_small_m_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
+                        const SmallParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* bsm = smem + p.b_off;  // fused: the codes of this CTA's K-slice
+  int32_t* part = reinterpret_cast<int32_t*>(smem + p.part_off);
+  float* xs_s = reinterpret_cast<float*>(smem + p.xs_off);
+  float* red = reinterpret_cast<float*>(smem + p.red_off);  // [8 warps][NT], then the slice maxima [NT]
+  float* cmax = red + 8 * NT;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + p.bar_off);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + kSmallMaxStages;
+  uint64_t* b_ready = bars + 2 * kSmallMaxStages;
+  uint64_t* acc_full = b_ready + 1;
+  uint64_t* drain = b_ready + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + p.misc_off);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + p.misc_off + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const int S = static_cast<int>(cluster_nctarank());
+  const int rb = blockIdx.y;  // 256-row block of Wq (= 256 outputs)
+  const int kb0 = static_cast<int>(rank) * p.kb_per_split;
+  const int kb1 = min(p.nk, kb0 + p.kb_per_split);
+  const int my_nkb = max(0, kb1 - kb0);
+  const int stages = p.stages;
+  // The four K=32 steps of a k-block write four separate TMEM accumulators
+  // (NT columns each) per 128-row half; the epilogue adds them (exact int32).
+  constexpr int kChains = 4;
+  constexpr int kHalfCols = kChains * NT;
+  constexpr uint32_t kTmemCols = 2 * kHalfCols;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < stages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    mbar_init(b_ready, 1);
+    mbar_init(acc_full, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmW);
+    if (!kFused) tma_prefetch_desc(&tmX);
+  }
+  if (warp == 1) {
+    __syncwarp();
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  if (threadIdx.x == 0) SQ_TRACE_MARK(0);
+  // fused: warps 0 and 1 take no part in the mid-kernel exchange of row maxima;
+  // they arrive now and complete that phase at the end
+  if (kFused && warp < 2) cluster_arrive_relaxed();
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0 && my_nkb > 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued = 0;
+      bool ok = true;
+      for (int kb = kb0; kb < kb1; ++kb) {
+        if (*abort_flag || !mbar_wait_bounded(&empty[stage], phase ^ 1u, kWaitTimeoutNs)) {
+          if (!*abort_flag) flag_timeout(abort_flag);
+          ok = false;
+          break;
+        }
+        uint8_t* dst = smem + stage * p.stage_bytes;
+        mbar_arrive_expect_tx(&full[stage], static_cast<uint32_t>(p.stage_bytes));
+        tma_load_2d(dst, &tmW, kb * kBK, rb * kSmallRows, &full[stage]);
+        if (!kFused) tma_load_2d(dst + kSmallABytes, &tmX, kb * kBK, 0, &full[stage]);
+        ++issued;
+        if (++stage == stages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (!ok) {  // drain the copies in flight (the last min(issued, stages) loads)
+        for (int i = 0; i < min(issued, stages); ++i) {
+          const int q = issued - 1 - i;
+          (void)mbar_wait_bounded(&full[q % stages], static_cast<uint32_t>((q / stages) & 1), kWaitTimeoutNs);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_i8(kBM, NT);
+      bool ok = true;
+      if (kFused) {
+        ok = !*abort_flag && mbar_wait_bounded(b_ready, 0, kWaitTimeoutNs);
+        if (!ok && !*abort_flag) flag_timeout(abort_flag);
+      }
+      SQ_TRACE_MARK(1);
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int j = 0; ok && j < my_nkb; ++j) {
+        if (*abort_flag || !mbar_wait_bounded(&full[stage], phase, kWaitTimeoutNs)) {
+          if (!*abort_flag) flag_timeout(abort_flag);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (j == 0) SQ_TRACE_MARK(2);
+        const uint32_t st = smem_u32(smem + stage * p.stage_bytes);
+        const uint64_t bdesc = kFused ? smem_desc_k_sw128(smem_u32(bsm + j * (NT * kBK)))
+                                      : smem_desc_k_sw128(st + kSmallABytes);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const uint64_t adesc = smem_desc_k_sw128(st + h * (kBM * kBK));
+#pragma unroll
+          for (int kk = 0; kk < kBK / kUmmaK; ++kk)
+            mma_i8(tmem_base + static_cast<uint32_t>(h * kHalfCols + kk * NT), adesc + static_cast<uint64_t>(kk * 2),
+                   bdesc + static_cast<uint64_t>(kk * 2), idesc, j != 0 ? 1u : 0u);
+        }
+        mma_commit(&empty[stage]);
+        if (++stage == stages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      SQ_TRACE_MARK(3);
+      if (ok) mma_commit(acc_full);
+      mma_commit(drain);
+      (void)mbar_wait_bounded(drain, 0, kWaitTimeoutNs);
+    }
+  } else {
+    // ------------------------------------------------- quantisation (warps 2..9)
+    const int qt = threadIdx.x - 64;
+    const int qw = qt >> 5;
+    const int M = p.M;
+    if (kFused) {
+      const int K = p.K;
+      const int nvec = K >> 3;
+      const int v_lo = kb0 * (kBK / 8);
+      const int v_hi = min(nvec, kb1 * (kBK / 8));
+      const uint4* X4 = reinterpret_cast<const uint4*>(p.X);
+      const float4* s4 = reinterpret_cast<const float4*>(p.s);
+      // pass 1: max of |fl(X / s)| over this CTA's K-slice, eight rows at a time
+      // with all of a group's loads issued before any arithmetic
+      float rmax[NT];
+#pragma unroll
+      for (int m = 0; m < NT; ++m) rmax[m] = 0.0f;
+      for (int v = v_lo + qt; v < v_hi; v += kSmallQuantThreads) {
+        f2x ns[4], rs[4];
+        load_s8(s4, v, ns, rs);
+#pragma unroll
+        for (int g = 0; g < NT; g += 8) {
+          if (g < M) {
+            uint4 w[8];
+#pragma unroll
+            for (int r = 0; r < 8; ++r)
+              w[r] = (g + r < M) ? __ldg(X4 + static_cast<int64_t>(g + r) * nvec + v) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+            for (int r = 0; r < 8; ++r) {
+              f2x t[4];
+              smooth8(w[r], ns, rs, t);
+#pragma unroll
+              for (int e = 0; e < 4; ++e) rmax[g + r] = f2_absmax(rmax[g + r], t[e]);
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int m = 0; m < NT; ++m) {
+        const float r = warp_max(rmax[m]);
+        if (lane == 0) red[qw * NT + m] = r;
+      }
+      named_bar_sync(1, kSmallQuantThreads);
+      if (qt < NT) {
+        float mx = 0.0f;
+#pragma unroll
+        for (int w = 0; w < kSmallQuantThreads / 32; ++w) mx = fmaxf(mx, red[w * NT + qt]);
+        cmax[qt] = mx;
+      }
+      // exchange of the slice maxima across the cluster (warps 0, 1 arrived early)
+      asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+      if (qt < NT) {
+        const uint32_t a = smem_u32(cmax + qt);
+        float mx = 0.0f;
+        for (int r = 0; r < S; ++r) mx = fmaxf(mx, ld_cluster_f32(map_cluster_rank(a, static_cast<uint32_t>(r))));
+        xs_s[qt] = __fdiv_rn(fmaxf(mx, kClampFloor), kQmax);
+      }
+      named_bar_sync(1, kSmallQuantThreads);
+      // pass 2: the codes of this CTA's K-slice, into the swizzled B operand
+      for (int v = v_lo + qt; v < v_hi; v += kSmallQuantThreads) {
+        f2x ns[4], rs[4];
+        load_s8(s4, v, ns, rs);
+        const int c = v * 8 - kb0 * kBK;
+#pragma unroll
+        for (int g = 0; g < NT; g += 8) {
+          if (g < M) {
+            uint4 w[8];
+#pragma unroll
+            for (int r = 0; r < 8; ++r)
+              w[r] = (g + r < M) ? __ldg(X4 + static_cast<int64_t>(g + r) * nvec + v) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+            for (int r = 0; r < 8; ++r) {
+              if (g + r < M) {
+                const float sc = xs_s[g + r];
+                const float rsc = __frcp_rn(sc);
+                const f2x nsc2 = f2_pack(-sc, -sc), rsc2 = f2_pack(rsc, rsc);
+                f2x t[4];
+                smooth8(w[r], ns, rs, t);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) t[e] = f2_round_codes(f2_div_rn(t[e], nsc2, rsc2));
+                *reinterpret_cast<uint2*>(bsm + b_code_offset<NT>(g + r, c)) = pack8_codes(t[0], t[1], t[2], t[3]);
+              }
+            }
+          }
+        }
+      }
+      // make the generic-proxy smem writes visible to the tensor core, then release the MMA warp
+      fence_proxy_async_smem();
+      named_bar_sync(1, kSmallQuantThreads);
+      if (qt == 0) mbar_arrive(b_ready);
+    } else {
+      if (qt < NT) xs_s[qt] = (qt < M) ? __ldg(p.x_scale + qt) : 0.0f;
+    }
+
+    // ------------------------------------------------- accumulators to shared memory (warps 2..5)
+    if (warp < 6) {
+      const int quarter = warp & 3;
+      bool have = my_nkb > 0;
+      if (have) {
+        const bool mine = !*abort_flag && mbar_wait_bounded(acc_full, 0, kWaitTimeoutNs);
+        have = __all_sync(0xFFFFFFFFu, mine);
+        if (!have && lane == 0 && !*abort_flag) flag_timeout(abort_flag);
+      }
+      if (have) tc_fence_after();
+      if (warp == 2 && lane == 0) SQ_TRACE_MARK(4);
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int n_local = h * kBM + quarter * 32 + lane;
+        uint32_t acc[NT];
+#pragma unroll
+        for (int i = 0; i < NT; ++i) acc[i] = 0u;
+        if (have) {
+          const uint32_t taddr =
+              tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(h * kHalfCols);
+#pragma unroll
+          for (int c = 0; c < kHalfCols; c += 32) {
+            uint32_t r32[32];
+            tmem_ld_32cols(taddr + static_cast<uint32_t>(c), r32);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) acc[(c + i) % NT] += r32[i];
+          }
+        }
+        uint4* dst = reinterpret_cast<uint4*>(part + n_local * NT);
+#pragma unroll
+        for (int i = 0; i < NT / 4; ++i)
+          dst[i] = make_uint4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]);
+      }
+    }
+  }
+
+  // ------------------------------------------- split-K reduction over the cluster
+  // Every rank reduces its share of the 256 rows: for each (row, 4 tokens) it
+  // reads the S partial sums (one per rank, through distributed shared memory),
+  // adds them, dequantises and stores.  The S loads are issued before any add.
+  tc_fence_before();
+  __syncthreads();
+  if (kFused && warp < 2) cluster_wait();  // completes the phase these warps arrived at early
+  cluster_sync_all();  // every CTA's partial accumulators are in its shared memory
+  if (threadIdx.x == 0) SQ_TRACE_MARK(5);
+  if (warp >= 2) {
+    const int rows_per_rank = (kSmallRows + S - 1) / S;
+    const int r_lo = static_cast<int>(rank) * rows_per_rank;
+    const int r_hi = min(kSmallRows, r_lo + rows_per_rank);
+    const int items = (r_hi - r_lo) * (NT / 4);
+    for (int it = threadIdx.x - 64; it < items; it += kSmallQuantThreads) {
+      const int n_local = r_lo + it / (NT / 4);
+      const int q4 = it % (NT / 4);
+      const uint32_t addr = smem_u32(part + n_local * NT + q4 * 4);
+      uint4 v[8];
+#pragma unroll
+      for (int r = 0; r < 8; ++r)
+        if (r < S) v[r] = ld_cluster_v4(map_cluster_rank(addr, static_cast<uint32_t>(r)));
+      int32_t acc[4] = {0, 0, 0, 0};
+#pragma unroll
+      for (int r = 0; r < 8; ++r)
+        if (r < S) {
+          acc[0] += static_cast<int32_t>(v[r].x), acc[1] += static_cast<int32_t>(v[r].y);
+          acc[2] += static_cast<int32_t>(v[r].z), acc[3] += static_cast<int32_t>(v[r].w);
+        }
+      const int n = rb * kSmallRows + n_local;
+      if (n < p.N) {
+        const float ws = __ldg(p.w_scale + n);
+        const float b = p.bias != nullptr ? __uint_as_float(static_cast<uint32_t>(__ldg(p.bias + n)) << 16) : 0.0f;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int m = q4 * 4 + j;
+          if (m < p.M) {
+            const float y = __fmaf_rn(__int2float_rn(acc[j]), __fmul_rn(xs_s[m], ws), b);
+            p.Y[static_cast<int64_t>(m) * p.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(y));
+          }
+        }
+      }
+    }
+  }
+  cluster_sync_all();  // no CTA leaves while another may still read its shared memory
+  if (threadIdx.x == 0) SQ_TRACE_MARK(6);
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+}  // namespace
+}  // namespace sq

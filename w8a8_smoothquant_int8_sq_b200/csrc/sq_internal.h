@@ -12,6 +12,10 @@ namespace sq {
 // one row per thread block held in registers).
 constexpr int64_t kMaxQuantK = 16384;
 
+// cudaSharedmemCarveoutMaxShared: every libsq kernel asks for the same L1 /
+// shared-memory split, so back-to-back kernels need no reconfiguration.
+constexpr int kCarveoutMaxShared = 100;
+
 struct DeviceInfo {
   int device = -1;
   int sm_count = 0;
@@ -23,6 +27,8 @@ struct DeviceInfo {
 cudaError_t current_device_info(DeviceInfo* out);
 
 // ---- calibration (sq_quant.cu)
+// 32-bit words of calibration scratch: mx[K], mw[K], one counter per 256 columns.
+size_t calibrate_workspace_words(int64_t K);
 cudaError_t launch_calibrate(const uint16_t* C, int64_t R, int64_t K, const uint16_t* W, int64_t N, float alpha,
                              float* s, float* mx_inout, void* ws, cudaStream_t st, const DeviceInfo& dev);
 
@@ -54,6 +60,25 @@ struct GemmArgs {
   Epilogue epi;
 };
 cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t st, const DeviceInfo& dev, const char** why);
+
+// Few tokens (M <= kSmallMaxM): weight-streaming kernel, split-K over a thread
+// block cluster.  With X != null the per-token quantisation of X / s is fused
+// (codes and scales identical to launch_row_quant); otherwise Xq and x_scale
+// come from the caller.  Returns cudaErrorNotSupported when the shape does not
+// fit the kernel (the caller then uses the general path).
+constexpr int64_t kSmallMaxM = 32;
+struct SmallArgs {
+  const uint16_t* X;      // fused: bf16 [M][K]
+  const float* s;         // fused: [K]
+  const int8_t* Xq;       // prequantised: [M][K]
+  const float* x_scale;   // prequantised: [M]
+  const int8_t* Wq;       // [N][K]
+  const float* w_scale;   // [N]
+  const uint16_t* bias;   // [N] or null
+  int64_t M, N, K;
+  uint16_t* Y;            // [M][N]
+};
+cudaError_t launch_small_m(const SmallArgs& a, cudaStream_t st, const DeviceInfo& dev, const char** why);
 
 // Device status word (bit 0: pipeline wait timeout).
 cudaError_t read_device_status(uint32_t* flags, bool clear);
