@@ -14,9 +14,11 @@ batch of 512 rows.
 Timing: every step is preceded by an L2 flush (the inputs are smaller than
 L2): a 256 MiB write, then a 512 MiB read, so that L2 holds neither the
 step's inputs nor dirty lines whose write-back would land inside the timed
-step.  CUDA events on the launching stream bracket the step and
-each library call inside it; each call is replayed from its own CUDA graph so
-that host launch latency does not leak into the device timeline.  With N > 1
+step.  The step (the four library calls) is captured as a CUDA graph with timing-event
+nodes before and after it; the kernels overlap each other's launch through
+programmatic dependent launch.  A second capture with event nodes between the
+calls, replayed the same number of times after the same flush, gives the
+per-call device times used for the roofline and the breakdown.  With N > 1
 (one process per GPU under torchrun) every rank runs an independent replica
 (the layer shards by tokens with no exchange): the value is the tokens all
 ranks processed divided by the slowest rank's time.
@@ -271,64 +273,75 @@ def run_ours(args, wl, rank, world, local_rank):
         "sq_quantize_act": lambda: sq.sq_quantize_act(X, s, Xq=Xq, x_scale=x_scale),
         "sq_linear": lambda: sq.sq_linear(Xq, x_scale, Wq, w_scale, b, Y=Y),
     }
-    launches_per_call = {"sq_calibrate": 2, "sq_prepare_weight": 1, "sq_quantize_act": 1, "sq_linear": 1}
+    launches_per_call = {"sq_calibrate": 1, "sq_prepare_weight": 1, "sq_quantize_act": 1, "sq_linear": 1}
     names = list(calls)
-    # initialise library caches outside capture, then one graph per call
+    # initialise library caches outside capture, then capture the step twice:
+    # as one graph with no nodes between the calls (the kernels overlap each
+    # other's launch through programmatic dependent launch) for the step time,
+    # and with timing-event nodes between the calls for the per-call times.
     for f in calls.values():
         f()
     torch.cuda.synchronize()
-    graphs = {}
-    for n in names:
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
+    step_evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)]
+    g_step = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_step):
+        step_evs[0].record()
+        for n in names:
             calls[n]()
-        graphs[n] = g
+        step_evs[1].record()
+    call_evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(names) + 1)]
+    g_calls = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_calls):
+        call_evs[0].record()
+        for i, n in enumerate(names):
+            calls[n]()
+            call_evs[i + 1].record()
     torch.cuda.synchronize()
 
-    stream = torch.cuda.current_stream()
-
-    def step(evs=None):
+    def flush_l2():
         flush.fill_(1)
         flush_read.max()
-        if evs is not None:
-            evs[0].record(stream)
-        for i, n in enumerate(names):
-            graphs[n].replay()
-            if evs is not None:
-                evs[i + 1].record(stream)
 
     sampler = ClockSampler(local_rank) if rank == 0 else None
     if sampler:
         sampler.start()
     t_settle = time.perf_counter()
     for _ in range(args.warmup):
-        step()
+        flush_l2()
+        g_step.replay()
+        flush_l2()
+        g_calls.replay()
     torch.cuda.synchronize()
     # keep the GPU under load briefly so the clock sampler sees steady clocks
     while time.perf_counter() - t_settle < args.settle_s:
         for _ in range(50):
-            step()
+            flush_l2()
+            g_step.replay()
         torch.cuda.synchronize()
 
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)] for _ in range(args.steps)]
+    total_ms = 0.0
     t_wall = time.perf_counter()
     for k in range(args.steps):
-        step(evs[k])
-    torch.cuda.synchronize()
+        flush_l2()
+        g_step.replay()
+        torch.cuda.synchronize()  # the events are read before the next replay re-records them
+        total_ms += step_evs[0].elapsed_time(step_evs[1])
     wall = time.perf_counter() - t_wall
     if world > 1:
         dist.barrier()
+    # per-call device times (same flush, same buffers), for the roofline and the breakdown
+    per_call = {n: 0.0 for n in names}
+    for k in range(args.steps):
+        flush_l2()
+        g_calls.replay()
+        torch.cuda.synchronize()
+        for i, n in enumerate(names):
+            per_call[n] += call_evs[i].elapsed_time(call_evs[i + 1])
     clocks = sampler.stop() if sampler else None
 
-    per_call = {n: 0.0 for n in names}
-    total_ms = 0.0
-    for e in evs:
-        total_ms += e[0].elapsed_time(e[-1])
-        for i, n in enumerate(names):
-            per_call[n] += e[i].elapsed_time(e[i + 1])
     step_ms = total_ms / args.steps
     per_call = {n: v / args.steps for n, v in per_call.items()}
     if world > 1:
@@ -340,6 +353,7 @@ def run_ours(args, wl, rank, world, local_rank):
     assert sq.sq_device_status() == 0, "device-side timeout flagged"
 
     # ------------------------------------------------------------- e2e leg
+    stream = torch.cuda.current_stream()
     e2e = None
     if not args.no_e2e:
         hC = torch.from_numpy(inp["C"].view(np.int16)).view(torch.bfloat16).pin_memory()
@@ -426,7 +440,7 @@ def run_ours(args, wl, rank, world, local_rank):
         "tops_per_step": 2.0 * wl.M * wl.N * wl.K * world / (step_ms * 1e-3) / 1e12,
         "gemm_tops": kernels["sq_linear"]["achieved_tops"],
         "roofline": roof, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
-        "gpu_launches": args.steps * sum(launches_per_call.values()),
+        "gpu_launches": 2 * args.steps * sum(launches_per_call.values()),
         "clocks": clocks, "wall_s_timed": wall,
     }
     print(json.dumps(line), flush=True)

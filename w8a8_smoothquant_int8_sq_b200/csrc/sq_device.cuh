@@ -129,6 +129,17 @@ __device__ __forceinline__ float warp_max(float v) {
   return v;
 }
 
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialization may start while the previous kernel in the stream finishes.
+// griddep_wait() blocks until that kernel has completed and its memory
+// operations are visible; every libsq kernel calls it before its first global
+// memory access.  griddep_launch_dependents() lets the next kernel begin its
+// own launch and set-up early.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // named barrier `id` (1..15) over `nthreads` threads (a multiple of 32)
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");

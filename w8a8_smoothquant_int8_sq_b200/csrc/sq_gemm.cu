@@ -58,6 +58,9 @@ constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // 2 s per wait
 #ifndef SQ_GEMM_BN
 #define SQ_GEMM_BN 0
 #endif
+#ifndef SQ_GEMM_SPLITK  // 1: split K over a cluster when 128 x 256 tiles do not fill the GPU
+#define SQ_GEMM_SPLITK 0
+#endif
 #ifndef SQ_GEMM_CHAINS128  // accumulator chains for 128-wide tiles (1 or 2)
 #define SQ_GEMM_CHAINS128 2
 #endif
@@ -95,10 +98,28 @@ struct SmemLayout {
   // barriers after the ring
   static constexpr int kBarOffset = kRingBytes;
   static constexpr int kNumBars = 2 * STAGES + 4 + 1;  // full, empty, tfull[2], tempty[2], drain
-  static constexpr int kMiscOffset = kBarOffset + kNumBars * 8;
+  // per epilogue warp: the tile's w_scale[BN] and bias[BN] (fp32)
+  static constexpr int kEpiOffset = (kBarOffset + kNumBars * 8 + 15) / 16 * 16;
+  static constexpr int kEpiBytes = 4 * 2 * BN * 4;
+  static constexpr int kMiscOffset = kEpiOffset + kEpiBytes;
   static constexpr int kBytes = kMiscOffset + 16;
   static constexpr int kAlloc = kBytes + 1024;  // manual 1024-byte alignment
 };
+
+#ifdef SQ_TRACE
+// Optional phase timestamps (build with -DSQ_TRACE): per CTA of the general
+// GEMM, globaltimer at 0 start, 1 first stage consumed, 2 last MMA issued,
+// 3 last epilogue store issued.
+__device__ unsigned long long g_big_trace[1024][4];
+#define SQ_BIG_MARK(i)                                               \
+  do {                                                               \
+    if (blockIdx.x < 1024) g_big_trace[blockIdx.x][i] = globaltimer_ns(); \
+  } while (0)
+#else
+#define SQ_BIG_MARK(i) \
+  do {                 \
+  } while (0)
+#endif
 
 __device__ __forceinline__ void flag_timeout(volatile int* abort_flag) {
   *abort_flag = 1;
@@ -157,6 +178,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  griddep_wait();
+  griddep_launch_dependents();
+  if (threadIdx.x == 0) SQ_BIG_MARK(0);
 
   const int num_tiles = p.num_m_blocks * p.num_n_blocks;
   const int nk = p.num_k_blocks;
@@ -247,6 +271,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           tc_fence_after();
+          if (it == 0 && kb == 0) SQ_BIG_MARK(1);
           const uint32_t sa = smem_u32(smem + stage * L::kStageBytes);
           const uint32_t sb = sa + L::kABytes;
           const uint64_t adesc = smem_desc_k_sw128(sa);
@@ -264,6 +289,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         if (!ok) break;
+        SQ_BIG_MARK(2);
         mma_commit(&tfull[acc]);
       }
       // drain: wait until every MMA this thread issued has completed
@@ -273,10 +299,41 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ------------------------------------------------------------ epilogue
     const int quarter = warp & 3;  // TMEM lanes [32*quarter, 32*quarter + 32) for this warp
+    // this warp's copy of the tile's w_scale and bias, staged before the
+    // accumulator is ready so that no global load sits between TMEM and the stores
+    float* ep_ws = reinterpret_cast<float*>(smem + L::kEpiOffset) + (warp - 2) * (2 * BN);
+    float* ep_b = ep_ws + BN;
     int it = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
       const int acc = it & 1;
       const uint32_t acc_phase = (it >> 1) & 1;
+      const int m_blk = tile % p.num_m_blocks;
+      const int n_blk = tile / p.num_m_blocks;
+      const int row = m_blk * kBM + quarter * 32 + lane;
+      const bool row_ok = row < p.M;
+      float xs = 0.0f;
+      if (EPI == 0) {
+        const int nb = n_blk * BN;
+        __syncwarp();  // the previous tile's reads of the staging area are done
+        for (int i = lane * 4; i < BN; i += 128) {
+          float4 w4 = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (nb + i + 4 <= p.N && p.vec_ok) {
+            w4 = __ldg(reinterpret_cast<const float4*>(p.w_scale + nb + i));
+          } else {
+            if (nb + i < p.N) w4.x = __ldg(p.w_scale + nb + i);
+            if (nb + i + 1 < p.N) w4.y = __ldg(p.w_scale + nb + i + 1);
+            if (nb + i + 2 < p.N) w4.z = __ldg(p.w_scale + nb + i + 2);
+            if (nb + i + 3 < p.N) w4.w = __ldg(p.w_scale + nb + i + 3);
+          }
+          *reinterpret_cast<float4*>(ep_ws + i) = w4;
+        }
+        for (int i = lane; i < BN; i += 32)
+          ep_b[i] = (p.bias != nullptr && nb + i < p.N)
+                        ? __uint_as_float(static_cast<uint32_t>(__ldg(p.bias + nb + i)) << 16)
+                        : 0.0f;
+        xs = row_ok ? __ldg(p.x_scale + row) : 0.0f;
+        __syncwarp();
+      }
       // every lane observes the phase itself; the vote keeps the warp uniform
       // for the warp-collective tcgen05.ld even if lanes disagree on a timeout
       const bool mine = !*abort_flag && mbar_wait_bounded(&tfull[acc], acc_phase, kWaitTimeoutNs);
@@ -285,11 +342,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      const int m_blk = tile % p.num_m_blocks;
-      const int n_blk = tile / p.num_m_blocks;
-      const int row = m_blk * kBM + quarter * 32 + lane;
-      const bool row_ok = row < p.M;
-      const float xs = (EPI == 0 && row_ok) ? __ldg(p.x_scale + row) : 0.0f;
       const uint32_t t_base =
           tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * CHAINS * BN);
 #pragma unroll 1
@@ -310,38 +362,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool full_chunk = (n0 + 32 <= p.N);
         const bool vec = full_chunk && p.vec_ok;
         if (EPI == 0) {
-          float ws[32], bs[32];
-          if (vec) {
-#pragma unroll
-            for (int j = 0; j < 32; j += 4) {
-              const float4 w4 = __ldg(reinterpret_cast<const float4*>(p.w_scale + n0 + j));
-              ws[j] = w4.x, ws[j + 1] = w4.y, ws[j + 2] = w4.z, ws[j + 3] = w4.w;
-            }
-            if (p.bias != nullptr) {
-#pragma unroll
-              for (int j = 0; j < 32; j += 8) {
-                const uint4 b8 = __ldg(reinterpret_cast<const uint4*>(p.bias + n0 + j));
-                bs[j] = bf16_lo(b8.x), bs[j + 1] = bf16_hi(b8.x), bs[j + 2] = bf16_lo(b8.y), bs[j + 3] = bf16_hi(b8.y);
-                bs[j + 4] = bf16_lo(b8.z), bs[j + 5] = bf16_hi(b8.z), bs[j + 6] = bf16_lo(b8.w), bs[j + 7] = bf16_hi(b8.w);
-              }
-            } else {
-#pragma unroll
-              for (int j = 0; j < 32; ++j) bs[j] = 0.0f;
-            }
-          } else {
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const bool in = n0 + j < p.N;
-              ws[j] = in ? __ldg(p.w_scale + n0 + j) : 0.0f;
-              bs[j] = (in && p.bias != nullptr) ? __uint_as_float(static_cast<uint32_t>(__ldg(p.bias + n0 + j)) << 16)
-                                                : 0.0f;
-            }
-          }
           uint32_t packed[16];
 #pragma unroll
           for (int j = 0; j < 32; j += 2) {
-            const float y0 = __fmaf_rn(__int2float_rn(static_cast<int>(r[j])), __fmul_rn(xs, ws[j]), bs[j]);
-            const float y1 = __fmaf_rn(__int2float_rn(static_cast<int>(r[j + 1])), __fmul_rn(xs, ws[j + 1]), bs[j + 1]);
+            const float y0 =
+                __fmaf_rn(__int2float_rn(static_cast<int>(r[j])), __fmul_rn(xs, ep_ws[c0 + j]), ep_b[c0 + j]);
+            const float y1 = __fmaf_rn(__int2float_rn(static_cast<int>(r[j + 1])), __fmul_rn(xs, ep_ws[c0 + j + 1]),
+                                       ep_b[c0 + j + 1]);
             packed[j / 2] = pack_bf16x2(y0, y1);
           }
           if (row_ok) {
@@ -375,6 +402,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);
+      if (warp == 2 && lane == 0) SQ_BIG_MARK(3);
     }
   }
 
@@ -389,6 +417,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 }  // namespace sq
 
 #include "sq_gemm_small.cuh"
+#include "sq_gemm_splitk.cuh"
 
 namespace sq {
 namespace {
@@ -459,8 +488,7 @@ cudaError_t run_gemm(const GemmArgs& a, cudaStream_t st, const DeviceInfo& dev, 
   }
   const int tiles = p.num_m_blocks * p.num_n_blocks;
   const int grid = std::min(tiles, dev.sm_count);
-  kern<<<grid, kThreads, L::kAlloc, st>>>(tmA, tmB, p);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(grid), dim3(kThreads), L::kAlloc, st, tmA, tmB, p);
 }
 
 template <int NT, bool kFused>
@@ -470,7 +498,7 @@ cudaError_t run_small(const SmallArgs& a, cudaStream_t st, const DeviceInfo& dev
   const int smem_cap = static_cast<int>(dev.max_smem_optin) - 1024;
   const int part_bytes = kSmallRows * NT * 4;
   const int stage_bytes = kSmallABytes + (kFused ? 0 : NT * kBK);
-  const int fixed = part_bytes + 128 + 9 * NT * 4 + 256 + 16;
+  const int fixed = part_bytes + 128 + 9 * NT * 4 + 2 * kSmallRows * 4 + 256 + 16;
   // split K over a cluster of S CTAs: as many splits as keep one wave of CTAs
   // (S <= 8, at least two k-blocks each), more if the fused codes would not fit
   int S = 1;
@@ -502,7 +530,8 @@ cudaError_t run_small(const SmallArgs& a, cudaStream_t st, const DeviceInfo& dev
   p.part_off = p.b_off + b_bytes;
   p.xs_off = p.part_off + part_bytes;
   p.red_off = p.xs_off + 128;
-  p.bar_off = p.red_off + 9 * NT * 4;
+  p.wsb_off = p.red_off + 9 * NT * 4;
+  p.bar_off = p.wsb_off + 2 * kSmallRows * 4;
   p.misc_off = p.bar_off + 256;
   const int alloc = p.misc_off + 16 + 1024;
   CUtensorMap tmW, tmX;
@@ -520,20 +549,45 @@ cudaError_t run_small(const SmallArgs& a, cudaStream_t st, const DeviceInfo& dev
     *why = "cudaFuncSetAttribute failed";
     return e;
   }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(S), static_cast<unsigned>(nrb), 1);
-  cfg.blockDim = dim3(kSmallThreads, 1, 1);
-  cfg.dynamicSmemBytes = static_cast<size_t>(alloc);
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = static_cast<unsigned>(S);
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, kern, tmW, tmX, p);
+  e = launch_pdl_cluster(kern, dim3(static_cast<unsigned>(S), static_cast<unsigned>(nrb), 1), dim3(kSmallThreads),
+                         static_cast<size_t>(alloc), st, static_cast<unsigned>(S), tmW, tmX, p);
   if (e != cudaSuccess) *why = "cluster launch of the small-M kernel failed";
+  return e;
+}
+
+template <int EPI>
+cudaError_t run_splitk(const GemmArgs& a, int S, cudaStream_t st, const DeviceInfo& dev, const char** why) {
+  (void)dev;
+  CUtensorMap tmA, tmB;
+  if (!make_tmap_i8(&tmA, a.A, a.M, a.K, kBM) || !make_tmap_i8(&tmB, a.B, a.N, a.K, kSkBN)) {
+    *why = "cuTensorMapEncodeTiled failed or unavailable";
+    return cudaErrorInvalidValue;
+  }
+  SkParams p{};
+  p.M = static_cast<int>(a.M);
+  p.N = static_cast<int>(a.N);
+  p.K = static_cast<int>(a.K);
+  p.num_m_blocks = static_cast<int>((a.M + kBM - 1) / kBM);
+  p.nk = static_cast<int>((a.K + kBK - 1) / kBK);
+  p.kb_per_split = (p.nk + S - 1) / S;
+  p.x_scale = a.x_scale;
+  p.w_scale = a.w_scale;
+  p.bias = a.bias;
+  p.out = a.out;
+  const int elem = (EPI == 0) ? 2 : 4;
+  p.vec_ok = ((a.N * elem) % 16 == 0) && (reinterpret_cast<uintptr_t>(a.out) % 16 == 0);
+  const int tiles = p.num_m_blocks * static_cast<int>((a.N + kSkBN - 1) / kSkBN);
+  auto kern = gemm_i8_splitk_kernel<EPI>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSkAlloc);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, kCarveoutMaxShared);
+  if (e != cudaSuccess) {
+    *why = "cudaFuncSetAttribute failed";
+    return e;
+  }
+  e = launch_pdl_cluster(kern, dim3(static_cast<unsigned>(S), static_cast<unsigned>(tiles), 1), dim3(kSkThreads),
+                         static_cast<size_t>(kSkAlloc), st, static_cast<unsigned>(S), tmA, tmB, p);
+  if (e != cudaSuccess) *why = "cluster launch of the split-K GEMM failed";
   return e;
 }
 
@@ -547,9 +601,19 @@ cudaError_t launch_small_m(const SmallArgs& a, cudaStream_t st, const DeviceInfo
 }
 
 cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t st, const DeviceInfo& dev, const char** why) {
-  // Tile width: 256-column tiles when they still fill the machine, else 128.
+  // 128 x 256 output tiles when there are at least as many as SMs.  With
+  // fewer, 128 x 128 tiles put about twice as many SMs to work: an M=128 int8
+  // MMA costs about the same for N=128 as for N=256, so each SM's main loop
+  // takes as long either way.  (Splitting K over a cluster instead, build knob
+  // SQ_GEMM_SPLITK, measured slower on B200: its reduction through distributed
+  // shared memory costs more than the main loop it shortens.)
   const int64_t mb = (a.M + kBM - 1) / kBM;
   const int64_t tiles256 = mb * ((a.N + 255) / 256);
+  const int64_t nk = (a.K + kBK - 1) / kBK;
+  int S = 1;
+  if (SQ_GEMM_SPLITK && SQ_GEMM_BN == 0 && tiles256 < dev.sm_count)
+    while (S < 8 && tiles256 * S * 2 <= dev.sm_count && nk >= 4 * S) S *= 2;
+  if (S > 1) return a.epi == Epilogue::kBf16Dequant ? run_splitk<0>(a, S, st, dev, why) : run_splitk<1>(a, S, st, dev, why);
   const bool wide = SQ_GEMM_BN == 256 || (SQ_GEMM_BN == 0 && tiles256 >= dev.sm_count);
   if (a.epi == Epilogue::kBf16Dequant) {
     return wide ? run_gemm<256, 4, 0, 1>(a, st, dev, why) : run_gemm<128, 6, 0, SQ_GEMM_CHAINS128>(a, st, dev, why);
@@ -558,6 +622,18 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t st, const DeviceInfo& de
 }
 
 #ifdef SQ_TRACE
+extern "C" __attribute__((visibility("default"))) int sq_trace_read_sk(unsigned long long* host, int n) {
+  return cudaMemcpyFromSymbol(host, g_sk_trace, sizeof(unsigned long long) * 8 * static_cast<size_t>(n)) ==
+                 cudaSuccess
+             ? 0
+             : 1;
+}
+extern "C" __attribute__((visibility("default"))) int sq_trace_read_big(unsigned long long* host, int n) {
+  return cudaMemcpyFromSymbol(host, g_big_trace, sizeof(unsigned long long) * 4 * static_cast<size_t>(n)) ==
+                 cudaSuccess
+             ? 0
+             : 1;
+}
 extern "C" __attribute__((visibility("default"))) int sq_trace_read(unsigned long long* host, int n) {
   return cudaMemcpyFromSymbol(host, g_small_trace, sizeof(unsigned long long) * 8 * static_cast<size_t>(n)) ==
                  cudaSuccess

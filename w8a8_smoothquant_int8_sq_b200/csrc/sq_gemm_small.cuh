@@ -55,7 +55,7 @@ struct SmallParams {
   const uint16_t* bias;  // [N] or null
   uint16_t* Y;           // [M][N]
   // shared-memory layout (bytes from the 1024-aligned base)
-  int b_off, part_off, xs_off, red_off, bar_off, misc_off;
+  int b_off, part_off, xs_off, red_off, wsb_off, bar_off, misc_off;
 };
 
 __device__ __forceinline__ uint32_t cluster_rank() {
@@ -142,6 +142,7 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
   float* xs_s = reinterpret_cast<float*>(smem + p.xs_off);
   float* red = reinterpret_cast<float*>(smem + p.red_off);  // [8 warps][NT], then the slice maxima [NT]
   float* cmax = red + 8 * NT;
+  float* wsb = reinterpret_cast<float*>(smem + p.wsb_off);  // w_scale[256], bias[256] of this row block
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + p.bar_off);
   uint64_t* full = bars;
   uint64_t* empty = bars + kSmallMaxStages;
@@ -190,6 +191,8 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  griddep_wait();
+  griddep_launch_dependents();
   if (threadIdx.x == 0) SQ_TRACE_MARK(0);
   // fused: warps 0 and 1 take no part in the mid-kernel exchange of row maxima;
   // they arrive now and complete that phase at the end
@@ -360,6 +363,13 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
     } else {
       if (qt < NT) xs_s[qt] = (qt < M) ? __ldg(p.x_scale + qt) : 0.0f;
     }
+    // stage this row block's w_scale and bias for the reduction (off the critical path)
+    {
+      const int n = rb * kSmallRows + qt;  // one row per quantisation thread
+      wsb[qt] = (n < p.N) ? __ldg(p.w_scale + n) : 0.0f;
+      wsb[kSmallRows + qt] =
+          (p.bias != nullptr && n < p.N) ? __uint_as_float(static_cast<uint32_t>(__ldg(p.bias + n)) << 16) : 0.0f;
+    }
 
     // ------------------------------------------------- accumulators to shared memory (warps 2..5)
     if (warp < 6) {
@@ -429,8 +439,8 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
         }
       const int n = rb * kSmallRows + n_local;
       if (n < p.N) {
-        const float ws = __ldg(p.w_scale + n);
-        const float b = p.bias != nullptr ? __uint_as_float(static_cast<uint32_t>(__ldg(p.bias + n)) << 16) : 0.0f;
+        const float ws = wsb[n_local];
+        const float b = wsb[kSmallRows + n_local];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const int m = q4 * 4 + j;

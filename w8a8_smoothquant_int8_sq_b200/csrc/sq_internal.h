@@ -5,6 +5,7 @@
 #include <cstddef>
 #include <cstdint>
 #include <cuda_runtime.h>
+#include <utility>
 
 namespace sq {
 
@@ -15,6 +16,38 @@ constexpr int64_t kMaxQuantK = 16384;
 // cudaSharedmemCarveoutMaxShared: every libsq kernel asks for the same L1 /
 // shared-memory split, so back-to-back kernels need no reconfiguration.
 constexpr int kCarveoutMaxShared = 100;
+
+// Launch a kernel with programmatic stream serialization (it may begin while
+// the previous kernel in the stream drains; the kernel itself waits for that
+// kernel's results before touching global memory) and, when cluster_x >= 1,
+// as clusters of cluster_x CTAs along x (cluster_x == 0: no cluster launch).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl_cluster(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                               unsigned cluster_x, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  unsigned n = 1;
+  if (cluster_x >= 1) {
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = cluster_x;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    n = 2;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args&&... args) {
+  return launch_pdl_cluster(kern, grid, block, smem, st, 0u, std::forward<Args>(args)...);
+}
 
 struct DeviceInfo {
   int device = -1;

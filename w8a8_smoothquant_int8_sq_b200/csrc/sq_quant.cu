@@ -60,6 +60,8 @@ __global__ void __launch_bounds__(kColThreads) colmax_kernel(const uint16_t* __r
                                                              uint32_t* ws, int chunks_c, int chunks_w,
                                                              int64_t rows_c, int64_t rows_w, double alpha,
                                                              float* __restrict__ mx_inout, float* __restrict__ s) {
+  griddep_wait();
+  griddep_launch_dependents();
   const bool is_w = blockIdx.z == 1;
   const int chunks = is_w ? chunks_w : chunks_c;
   if (static_cast<int>(blockIdx.y) >= chunks) return;  // not counted: only chunks_c + chunks_w blocks arrive
@@ -160,9 +162,9 @@ cudaError_t launch_calibrate(const uint16_t* C, int64_t R, int64_t K, const uint
   const int chunks_w = static_cast<int>((N + rows_w - 1) / rows_w);
   const int chunks_c = R > 0 ? static_cast<int>((R + rows_c - 1) / rows_c) : 0;
   dim3 grid(static_cast<unsigned>(stripes), static_cast<unsigned>(std::max(chunks_c, chunks_w)), 2);
-  colmax_kernel<<<grid, kColThreads, 0, st>>>(C, R, W, N, static_cast<int>(K), static_cast<uint32_t*>(ws), chunks_c,
-                                             chunks_w, rows_c, rows_w, static_cast<double>(alpha), mx_inout, s);
-  return cudaGetLastError();
+  return launch_pdl(colmax_kernel, grid, dim3(kColThreads), 0, st, C, R, W, N, static_cast<int>(K),
+                    static_cast<uint32_t*>(ws), chunks_c, chunks_w, rows_c, rows_w, static_cast<double>(alpha),
+                    mx_inout, s);
 }
 
 // ============================================ calibration without allocation
@@ -249,6 +251,8 @@ __global__ void __launch_bounds__(kRowThreads) row_quant_kernel(const uint16_t* 
   int64_t row = static_cast<int64_t>(blockIdx.x) * RPC + slot;
   const int64_t row_step = static_cast<int64_t>(gridDim.x) * RPC;
 
+  griddep_wait();
+  griddep_launch_dependents();
   uint4 xv[VPL];
   load_row_vectors<VPL, WPR>(xv, src, row, rows, K, nvec, wsub, lane);  // in flight during the table build
 
@@ -342,8 +346,7 @@ static cudaError_t launch_rq(const uint16_t* src, int64_t rows, int K, const flo
   constexpr int RPC = 8 / WPR;
   const int64_t groups = (rows + RPC - 1) / RPC;
   const int64_t grid = std::min<int64_t>(groups, static_cast<int64_t>(dev.sm_count) * per_sm);
-  kern<<<static_cast<unsigned>(grid), kRowThreads, smem, st>>>(src, rows, K, s, q, scale);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(static_cast<unsigned>(grid)), dim3(kRowThreads), smem, st, src, rows, K, s, q, scale);
 }
 
 template <bool kMul>
