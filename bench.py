@@ -126,6 +126,25 @@ def ncu_traffic(kernel_call, wl_name):
     return e.get("dram_bytes_per_launch")
 
 
+# ------------------------------------------------------------- multi-rank
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The largest value of x over all ranks (for times: the slowest rank).
+    With one process per GPU the replicas run independently; this is the only
+    collective, and it carries a single number."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank: float, world: int, ms: float) -> float:
+    """Units processed by all ranks per second, over the slowest rank's time."""
+    return units_per_rank * world / (ms * 1e-3)
+
+
 # ------------------------------------------------------------------- clocks
 class ClockSampler:
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,utilization.gpu,clocks_event_reasons.active,"
@@ -342,12 +361,8 @@ def run_ours(args, wl, rank, world, local_rank):
             per_call[n] += call_evs[i].elapsed_time(call_evs[i + 1])
     clocks = sampler.stop() if sampler else None
 
-    step_ms = total_ms / args.steps
+    step_ms = max_over_ranks(total_ms / args.steps, world, dev)
     per_call = {n: v / args.steps for n, v in per_call.items()}
-    if world > 1:
-        t = torch.tensor([step_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        step_ms = float(t.item())
 
     # correctness guard on the timed buffers (cheap; sq_forward path equals these calls)
     assert sq.sq_device_status() == 0, "device-side timeout flagged"
@@ -386,13 +401,9 @@ def run_ours(args, wl, rank, world, local_rank):
             e2e_step()
         e1.record(stream)
         torch.cuda.synchronize()
-        e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
-        if world > 1:
-            t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, world, dev)
         h2d = sum(t.numel() * t.element_size() for t in (hC, hW, hX) + ((hb,) if hb is not None else ()))
-        e2e = {"value": wl.M * world / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+        e2e = {"value": whole_job_rate(wl.M, world, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": hY.numel() * hY.element_size(), "ms_per_step": e2e_ms,
                "call": "sq_calibrate + sq_prepare_weight + sq_forward"}
 
@@ -432,7 +443,7 @@ def run_ours(args, wl, rank, world, local_rank):
         cpu = {"value": v, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
                "sample": f"{n} whole {wl.name} steps in {el:.1f} s (calibrate, fold+quantise W, forward)"}
 
-    value = wl.M * world / (step_ms * 1e-3)
+    value = whole_job_rate(wl.M, world, step_ms)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",

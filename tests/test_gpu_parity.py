@@ -195,3 +195,30 @@ def test_fault_injection(sq):
 
 def test_device_status_clean(sq):
     assert sq.sq_device_status() == 0
+
+
+def test_prefill_full_size_sampled(sq):
+    """The largest layer (X[8192x8192], W[28672x8192]) on the GPU at full size;
+    the oracle checks s over all channels and sampled rows of Wq / Xq and a
+    sampled block of Y (each output depends only on its row of Xq and of Wq)."""
+    wl = workloads.get("prefill")
+    inp = workloads.make_inputs(wl)
+    Cd, Wd, Xd = dev_bf16(inp["C"]), dev_bf16(inp["W"]), dev_bf16(inp["X"])
+    s_g = sq.sq_calibrate(Cd, Wd, wl.alpha_f32)
+    Wq_g, ws_g = sq.sq_prepare_weight(Wd, s_g)
+    Y_g = sq.sq_forward(Xd, s_g, Wq_g, ws_g)
+    torch.cuda.synchronize()
+    s_o, _ = O.calibrate(inp["C"], inp["W"], wl.alpha_f32)
+    assert_scales_close(host(s_g), s_o, "prefill: s")
+    rng = np.random.default_rng(4242)
+    rows_w = np.sort(rng.choice(wl.N, 96, replace=False))
+    rows_x = np.sort(np.concatenate([[0, wl.M - 1], rng.choice(wl.M, 62, replace=False)]))
+    s_h = host(s_g)
+    Wq_o, ws_o = O.fold_and_quantize_weight(inp["W"][rows_w], s_h)
+    assert np.array_equal(host(Wq_g[torch.as_tensor(rows_w, device="cuda")]), Wq_o)
+    assert np.array_equal(host(ws_g)[rows_w], ws_o)
+    Xq_o, xs_o = O.quantize_activation(inp["X"][rows_x], s_h)
+    acc_o = O.int8_gemm(Xq_o, Wq_o)
+    y_g = host_bf16_bits(Y_g)[np.ix_(rows_x, rows_w)]
+    ratio = assert_y_close(y_g, acc_o, xs_o, ws_o, None, "prefill: sampled Y")
+    print(f"\n[parity] prefill sampled {len(rows_x)}x{len(rows_w)}: y_tol_ratio {ratio}")

@@ -1,0 +1,45 @@
+"""Device-side failure detection without a GPU fault: every pipeline wait of
+the GEMM is bounded.  With the test hook on, the producer never fills the first
+stage, the waits give up after 50 ms, the kernel reports bit 0 of the status
+word and returns; the context stays usable and the next call is exact."""
+import time
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import smoothquant as O
+from tests.helpers import dev, host
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def sq():
+    assert torch.cuda.is_available(), "GPU test"
+    import w8a8_smoothquant_int8_sq_b200 as m
+    return m
+
+
+def test_pipeline_wait_timeout_is_reported_and_the_context_survives(sq):
+    rng = np.random.default_rng(99)
+    M, N, K = 256, 512, 4096  # general GEMM (M > 32), 32 k-blocks: more than the ring holds
+    Xq = rng.integers(-127, 128, (M, K), dtype=np.int64).astype(np.int8)
+    Wq = rng.integers(-127, 128, (N, K), dtype=np.int64).astype(np.int8)
+    Xq_d, Wq_d = dev(Xq), dev(Wq)
+    assert sq.sq_device_status(clear=True) == 0
+    try:
+        sq.sq_debug_pipeline_stall(True, 50_000_000)
+        t0 = time.perf_counter()
+        sq.sq_gemm_s32(Xq_d, Wq_d)
+        torch.cuda.synchronize()
+        elapsed = time.perf_counter() - t0
+    finally:
+        sq.sq_debug_pipeline_stall(False)
+    flags = sq.sq_device_status(clear=True)
+    assert flags & 1, "the stalled pipeline was not reported"
+    assert elapsed < 5.0
+    # the context is intact: the same call now returns the exact product
+    acc = host(sq.sq_gemm_s32(Xq_d, Wq_d))
+    assert np.array_equal(acc.astype(np.int64), O.int8_gemm(Xq, Wq))
+    assert sq.sq_device_status() == 0

@@ -24,6 +24,7 @@ __all__ = [
     "sq_version", "sq_calibrate", "sq_calibrate_workspace_bytes", "sq_calibrate_noalloc", "sq_prepare_weight",
     "sq_quantize_act", "sq_linear", "sq_workspace_bytes", "sq_forward",
     "sq_forward_workspace_bytes", "sq_gemm_s32", "sq_device_status", "sq_debug_fail_after",
+    "sq_debug_pipeline_stall",
     "STATUS",
 ]
 
@@ -56,6 +57,7 @@ _SIGNATURES = [
     ("sq_gemm_s32", ctypes.c_int, (_P, _P, _I64, _I64, _I64, _P, _P)),
     ("sq_device_status", ctypes.c_int, (ctypes.POINTER(ctypes.c_uint32), ctypes.c_int)),
     ("sq_debug_fail_after", None, (ctypes.c_int,)),
+    ("sq_debug_pipeline_stall", None, (ctypes.c_int, _I64)),
 ]
 
 _LIB = None
@@ -304,3 +306,9 @@ def sq_device_status(clear: bool = False) -> int:
 def sq_debug_fail_after(n: int) -> None:
     """Host-side fault injection: after n more launches, entry points fail with SQ_ERR_CUDA."""
     _load().sq_debug_fail_after(int(n))
+
+
+def sq_debug_pipeline_stall(enable: bool, timeout_ns: int = 0) -> None:
+    """Test hook: the general GEMM skips its first stage and its waits give up
+    after timeout_ns, reporting bit 0 of the device status word (no GPU fault)."""
+    _load().sq_debug_pipeline_stall(1 if enable else 0, int(timeout_ns))

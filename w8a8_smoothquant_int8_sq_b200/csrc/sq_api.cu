@@ -130,6 +130,10 @@ const char* sq_status_string(sq_status st) {
 
 void sq_debug_fail_after(int n) { g_fail_after.store(n < 0 ? -1 : n); }
 
+void sq_debug_pipeline_stall(int enable, int64_t timeout_ns) {
+  sq::debug_pipeline_stall(enable != 0, timeout_ns > 0 ? static_cast<unsigned long long>(timeout_ns) : 0ull);
+}
+
 // ------------------------------------------------------------ calibration
 size_t sq_calibrate_workspace_bytes(int64_t K) {
   if (K <= 0) return 0;

@@ -23,6 +23,7 @@
 // returns.
 #include <algorithm>
 #include <cstdint>
+#include <atomic>
 #include <mutex>
 
 #include "sq_device.cuh"
@@ -80,6 +81,8 @@ __device__ __forceinline__ int k_start(int m_blk, int n_blk, int nk) {
 }
 
 struct KParams {
+  unsigned long long timeout_ns;  // limit of every mbarrier wait
+  int skip_first_load;            // test hook: the producer never loads the first stage
   int M, N, K;
   int num_m_blocks, num_n_blocks, num_k_blocks;
   const float* x_scale;
@@ -220,9 +223,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int k0 = k_start(m_blk, n_blk, nk);
         for (int kb = 0; kb < nk; ++kb, ++seq) {
           if (kPrefetchAhead > 0) prefetch_upto(seq + 1 + kPrefetchAhead);
+          if (p.skip_first_load && seq == 0) {  // test hook: this stage never fills
+            if (++stage == STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
+            continue;
+          }
           int kk = kb + k0;
           if (kk >= nk) kk -= nk;
-          if (*abort_flag || !mbar_wait_bounded(&empty[stage], phase ^ 1u, kWaitTimeoutNs)) {
+          if (*abort_flag || !mbar_wait_bounded(&empty[stage], phase ^ 1u, p.timeout_ns)) {
             if (!*abort_flag) flag_timeout(abort_flag);
             ok = false;
             break;
@@ -244,7 +254,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // drain: every copy this thread issued must land before the CTA exits
 #pragma unroll
         for (int i = 0; i < STAGES; ++i)
-          if (issued[i]) (void)mbar_wait_bounded(&full[i], issued_phase[i], kWaitTimeoutNs);
+          if (issued[i]) (void)mbar_wait_bounded(&full[i], issued_phase[i], p.timeout_ns);
       }
     }
   } else if (warp == 1) {
@@ -258,14 +268,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x, ++it) {
         const int acc = it & 1;
         const uint32_t acc_phase = (it >> 1) & 1;
-        if (*abort_flag || !mbar_wait_bounded(&tempty[acc], acc_phase ^ 1u, kWaitTimeoutNs)) {
+        if (*abort_flag || !mbar_wait_bounded(&tempty[acc], acc_phase ^ 1u, p.timeout_ns)) {
           if (!*abort_flag) flag_timeout(abort_flag);
           break;
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * CHAINS * BN);
         for (int kb = 0; kb < nk; ++kb) {
-          if (*abort_flag || !mbar_wait_bounded(&full[stage], phase, kWaitTimeoutNs)) {
+          if (*abort_flag || !mbar_wait_bounded(&full[stage], phase, p.timeout_ns)) {
             if (!*abort_flag) flag_timeout(abort_flag);
             ok = false;
             break;
@@ -294,7 +304,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // drain: wait until every MMA this thread issued has completed
       mma_commit(drain);
-      (void)mbar_wait_bounded(drain, 0, kWaitTimeoutNs);
+      (void)mbar_wait_bounded(drain, 0, p.timeout_ns);
     }
   } else {
     // ------------------------------------------------------------ epilogue
@@ -336,7 +346,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // every lane observes the phase itself; the vote keeps the warp uniform
       // for the warp-collective tcgen05.ld even if lanes disagree on a timeout
-      const bool mine = !*abort_flag && mbar_wait_bounded(&tfull[acc], acc_phase, kWaitTimeoutNs);
+      const bool mine = !*abort_flag && mbar_wait_bounded(&tfull[acc], acc_phase, p.timeout_ns);
       if (!__all_sync(0xFFFFFFFFu, mine)) {
         if (lane == 0 && !*abort_flag) flag_timeout(abort_flag);
         break;
@@ -423,6 +433,10 @@ namespace sq {
 namespace {
 
 // ----------------------------------------------------------- host helpers
+// test hook state (sq_debug_pipeline_stall)
+std::atomic<int> g_debug_stall{0};
+std::atomic<unsigned long long> g_debug_timeout_ns{kWaitTimeoutNs};
+
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                    CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
@@ -464,6 +478,8 @@ cudaError_t run_gemm(const GemmArgs& a, cudaStream_t st, const DeviceInfo& dev, 
     return cudaErrorInvalidValue;
   }
   KParams p;
+  p.timeout_ns = g_debug_stall.load() ? g_debug_timeout_ns.load() : kWaitTimeoutNs;
+  p.skip_first_load = g_debug_stall.load() ? 1 : 0;
   p.M = static_cast<int>(a.M);
   p.N = static_cast<int>(a.N);
   p.K = static_cast<int>(a.K);
@@ -641,6 +657,11 @@ extern "C" __attribute__((visibility("default"))) int sq_trace_read(unsigned lon
              : 1;
 }
 #endif
+
+void debug_pipeline_stall(bool enable, unsigned long long timeout_ns) {
+  g_debug_timeout_ns.store(timeout_ns > 0 ? timeout_ns : kWaitTimeoutNs);
+  g_debug_stall.store(enable ? 1 : 0);
+}
 
 cudaError_t read_device_status(uint32_t* flags, bool clear) {
   cudaError_t e = cudaDeviceSynchronize();

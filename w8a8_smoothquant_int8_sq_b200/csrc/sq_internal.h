@@ -113,6 +113,10 @@ struct SmallArgs {
 };
 cudaError_t launch_small_m(const SmallArgs& a, cudaStream_t st, const DeviceInfo& dev, const char** why);
 
+// Test hook: while enabled, the general GEMM's producer skips its first stage
+// and every wait gives up after timeout_ns (the kernel then reports bit 0).
+void debug_pipeline_stall(bool enable, unsigned long long timeout_ns);
+
 // Device status word (bit 0: pipeline wait timeout).
 cudaError_t read_device_status(uint32_t* flags, bool clear);
 
