@@ -90,7 +90,9 @@ SQ_API const char* sq_status_string(sq_status st);
  *   workspace  device scratch of at least sq_calibrate_workspace_bytes(K)
  *              bytes, 16-byte aligned; contents on entry are ignored.
  * Launches: one memset of the workspace and one kernel (column max-abs over
- * C and W; the last block to finish each 256-column stripe computes s there).
+ * C and W, streamed through shared memory by TMA; the last block to finish
+ * each 256-column stripe computes s there and zeroes the stripe's workspace
+ * words again).
  */
 SQ_API size_t sq_calibrate_workspace_bytes(int64_t K);
 SQ_API sq_status sq_calibrate(const sq_bf16* C, int64_t R, int64_t K,
@@ -113,8 +115,11 @@ SQ_API sq_status sq_calibrate(const sq_bf16* C, int64_t R, int64_t K,
  *   before any stream capture on the device.
  *   All calls on a device share the array: calls that may run at the same time
  *   on the GPU (different streams without ordering) race and give wrong s.
- *   Each call clears the part it uses before reducing into it, so one call's
- *   leftovers never reach the next.
+ *   Launches: one kernel and no memset.  The array is zero when the library
+ *   loads and each call zeroes the words it used once it has read them, so
+ *   one call's values never reach the next.  A call that timed out on the
+ *   device (sq_device_status) may leave the array dirty; clearing the status
+ *   with sq_device_status(&flags, 1) zeroes it again.
  */
 SQ_API sq_status sq_calibrate_noalloc(const sq_bf16* C, int64_t R, int64_t K,
                                       const sq_bf16* W, int64_t N, float alpha,
@@ -188,8 +193,11 @@ SQ_API sq_status sq_gemm_s32(const int8_t* Xq, const int8_t* Wq, int64_t M, int6
 
 /* ------------------------------------------------------ device status word
  * sq_device_status -- read (and with clear != 0, reset) the device-side status
- * flags of the current device: bit 0 = a pipeline wait in a GEMM kernel timed
- * out.  Synchronises the device.  Returns SQ_ERR_TIMEOUT if any bit is set.
+ * flags of the current device: bit 0 = a bounded wait in a library kernel (a
+ * GEMM pipeline wait, or a wait for streamed rows in the calibration and
+ * quantisation kernels) timed out; the results of that call are undefined.
+ * Synchronises the device.  Returns SQ_ERR_TIMEOUT if any bit is set.
+ * Clearing a set status also re-zeroes the scratch of sq_calibrate_noalloc.
  */
 SQ_API sq_status sq_device_status(uint32_t* flags, int clear);
 

@@ -93,6 +93,8 @@ def test_workload_stage_parity(sq, name):
     (32, 4104, 1024, False),    # largest few-token case, ragged last weight block
     (8, 4096, 4096, True),      # few tokens, four-way split-K cluster
     (33, 256, 512, True),       # just above the few-token path
+    (40, 96, 16384, False),     # largest K: eight warps per row in the row quantisers
+    (3, 64, 16384, True),       # largest K on the few-token path
 ])
 def test_ragged_shapes(sq, M, N, K, with_bias):
     rng = np.random.default_rng(M * 7919 + N * 31 + K)
@@ -145,6 +147,22 @@ def test_running_max_two_batches(sq):
     # R == 0: s from the running max alone
     s3 = sq.sq_calibrate(None, dev_bf16(W), wl.alpha_f32, mx_inout=mx)
     assert torch.equal(s3, s_one)
+
+
+def test_calibrate_leaves_workspace_zero(sq):
+    """Whatever the workspace holds on entry, a call ends with the words it
+    reduced into -- mx[K], mw[K] and one counter per 256 columns -- zeroed (the
+    last block of each column stripe clears them)."""
+    wl = workloads.get("tiny")
+    inp = workloads.make_inputs(wl, ("C", "W"))
+    K = wl.K
+    ws = torch.full((sq.sq_calibrate_workspace_bytes(K),), 0xA5, dtype=torch.uint8, device="cuda")
+    s1 = sq.sq_calibrate(dev_bf16(inp["C"]), dev_bf16(inp["W"]), wl.alpha_f32, workspace=ws)
+    torch.cuda.synchronize()
+    used = 4 * (2 * K + (K + 255) // 256)
+    assert int(ws[:used].count_nonzero()) == 0
+    s_o, _ = O.calibrate(inp["C"], inp["W"], wl.alpha_f32)
+    assert_scales_close(host(s1), s_o, "tiny: s with a dirty workspace on entry")
 
 
 def test_alpha_special_cases(sq):

@@ -157,7 +157,7 @@ sq_status sq_calibrate(const sq_bf16* C, int64_t R, int64_t K, const sq_bf16* W,
   if (!aligned16(workspace)) return fail(SQ_ERR_ALIGN, "workspace is not 16-byte aligned");
   sq::DeviceInfo dev;
   SQ_TRY(prologue(&dev));
-  return cuda_status(sq::launch_calibrate(C, R, K, W, N, alpha, s, mx_inout, workspace,
+  return cuda_status(sq::launch_calibrate(C, R, K, W, N, alpha, s, mx_inout, workspace, /*ws_is_zero=*/false,
                                           static_cast<cudaStream_t>(stream), dev),
                      "calibrate launch");
 }

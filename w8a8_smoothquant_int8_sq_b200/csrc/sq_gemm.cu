@@ -111,9 +111,9 @@ struct SmemLayout {
 
 #ifdef SQ_TRACE
 // Optional phase timestamps (build with -DSQ_TRACE): per CTA of the general
-// GEMM, globaltimer at 0 start, 1 first stage consumed, 2 last MMA issued,
-// 3 last epilogue store issued.
-__device__ unsigned long long g_big_trace[1024][4];
+// GEMM, globaltimer at 0 past the wait for the previous kernel, 1 first stage
+// consumed, 2 last MMA issued, 3 last epilogue store issued, 4 block start.
+__device__ unsigned long long g_big_trace[1024][5];
 #define SQ_BIG_MARK(i)                                               \
   do {                                                               \
     if (blockIdx.x < 1024) g_big_trace[blockIdx.x][i] = globaltimer_ns(); \
@@ -181,6 +181,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  if (threadIdx.x == 0) SQ_BIG_MARK(4);
   griddep_wait();
   griddep_launch_dependents();
   if (threadIdx.x == 0) SQ_BIG_MARK(0);
@@ -645,7 +646,7 @@ extern "C" __attribute__((visibility("default"))) int sq_trace_read_sk(unsigned 
              : 1;
 }
 extern "C" __attribute__((visibility("default"))) int sq_trace_read_big(unsigned long long* host, int n) {
-  return cudaMemcpyFromSymbol(host, g_big_trace, sizeof(unsigned long long) * 4 * static_cast<size_t>(n)) ==
+  return cudaMemcpyFromSymbol(host, g_big_trace, sizeof(unsigned long long) * 5 * static_cast<size_t>(n)) ==
                  cudaSuccess
              ? 0
              : 1;
@@ -674,8 +675,31 @@ cudaError_t read_device_status(uint32_t* flags, bool clear) {
     e = cudaMemcpyToSymbol(g_sq_device_status, &z, sizeof(z));
     if (e != cudaSuccess) return e;
   }
-  *flags = v;
+  uint32_t q = 0;
+  e = read_quant_status(&q, clear);
+  if (e != cudaSuccess) return e;
+  *flags = v | q;
   return cudaSuccess;
+}
+
+bool make_tmap_2d(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int elem_bytes, int box_cols,
+                  int box_rows) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (enc == nullptr) return false;
+  CUtensorMapDataType dt;
+  switch (elem_bytes) {
+    case 1: dt = CU_TENSOR_MAP_DATA_TYPE_UINT8; break;
+    case 2: dt = CU_TENSOR_MAP_DATA_TYPE_UINT16; break;
+    case 4: dt = CU_TENSOR_MAP_DATA_TYPE_UINT32; break;
+    default: return false;
+  }
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * static_cast<cuuint64_t>(elem_bytes)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
 }
 
 }  // namespace sq

@@ -4,13 +4,14 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <utility>
 
 namespace sq {
 
-// Largest K the row quantisers keep on chip (s and 1/s staged in shared memory,
-// one row per thread block held in registers).
+// Largest K the row quantisers handle: a row is held in registers by at most
+// eight warps of eight 16-byte vectors per lane.
 constexpr int64_t kMaxQuantK = 16384;
 
 // cudaSharedmemCarveoutMaxShared: every libsq kernel asks for the same L1 /
@@ -59,11 +60,25 @@ struct DeviceInfo {
 // Cached properties of the current device.
 cudaError_t current_device_info(DeviceInfo* out);
 
+// 2-D tensor map over a row-major [rows][cols] matrix of elem_bytes-wide
+// elements (row pitch cols * elem_bytes), box box_cols x box_rows, no swizzle,
+// zero fill outside the matrix.  False when the driver's encoder is
+// unavailable or rejects the arguments.
+bool make_tmap_2d(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int elem_bytes, int box_cols,
+                  int box_rows);
+
+// Status word of the HBM-bound kernels (bit 0: a wait timed out).  Clearing a
+// set word also re-zeroes the no-allocation calibration scratch.
+cudaError_t read_quant_status(uint32_t* flags, bool clear);
+
 // ---- calibration (sq_quant.cu)
 // 32-bit words of calibration scratch: mx[K], mw[K], one counter per 256 columns.
 size_t calibrate_workspace_words(int64_t K);
+// ws_is_zero: the caller guarantees the workspace words are zero (no memset).
+// Every call leaves them zero.
 cudaError_t launch_calibrate(const uint16_t* C, int64_t R, int64_t K, const uint16_t* W, int64_t N, float alpha,
-                             float* s, float* mx_inout, void* ws, cudaStream_t st, const DeviceInfo& dev);
+                             float* s, float* mx_inout, void* ws, bool ws_is_zero, cudaStream_t st,
+                             const DeviceInfo& dev);
 
 // Largest K accepted by sq_calibrate_noalloc (its fixed scratch holds 2*K words).
 constexpr int64_t kNoAllocMaxK = 16384;

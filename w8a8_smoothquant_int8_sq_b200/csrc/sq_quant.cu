@@ -19,26 +19,95 @@
 
 namespace sq {
 
+// Latched by a wait in these kernels that ran out of time (bit 0), like the
+// GEMM's status word; read and cleared through read_device_status.
+__device__ unsigned int g_sq_quant_status = 0u;
+constexpr unsigned long long kQuantWaitTimeoutNs = 2000000000ull;  // 2 s per wait
+
+
+
+#ifdef SQ_TRACE
+// Optional block timestamps (build with -DSQ_TRACE): per kernel kind (0 colmax,
+// 1 row quant of weights, 2 row quant of activations) and block, globaltimer at
+// 0 block start, 1 past the wait for the previous kernel, 2 block end.
+__device__ unsigned long long g_blk_trace[3][2048][3];
+struct BlockTrace {
+  int kind, id;
+  __device__ BlockTrace(int k) : kind(k), id(blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z)) {
+    mark(0);
+  }
+  __device__ void mark(int i) const {
+    if (threadIdx.x == 0 && id < 2048) g_blk_trace[kind][id][i] = globaltimer_ns();
+  }
+  __device__ ~BlockTrace() { mark(2); }
+};
+#define SQ_BLOCK_TRACE(kind) BlockTrace blk_trace_(kind)
+#define SQ_BLOCK_MARK(i) blk_trace_.mark(i)
+extern "C" __attribute__((visibility("default"))) int sq_trace_read_blocks(unsigned long long* host) {
+  return cudaMemcpyFromSymbol(host, g_blk_trace, sizeof(g_blk_trace)) == cudaSuccess ? 0 : 1;
+}
+extern "C" __attribute__((visibility("default"))) int sq_trace_clear_blocks() {
+  static unsigned long long zero[3][2048][3];
+  return cudaMemcpyToSymbol(g_blk_trace, zero, sizeof(zero)) == cudaSuccess ? 0 : 1;
+}
+#else
+#define SQ_BLOCK_TRACE(kind) \
+  do {                       \
+  } while (0)
+#define SQ_BLOCK_MARK(i) \
+  do {                   \
+  } while (0)
+#endif
+
 // ====================================================== column max-abs (K1)
-// Blocks are laid out as (256-column stripe) x (chunk of rows) x {C, W}; about
-// two blocks per SM in total, each walking its chunk in batches of 8 rows per
-// warp with the next batch's loads issued before the current one is reduced
-// (16 loads of 16 bytes in flight per lane).  |x| is taken on the bf16 bit
-// patterns with the sign bit cleared: for non-negative bf16 values the integer
-// order of the patterns is the numeric order, so the max is exact and needs no
-// conversion until the end.  Block results are merged with an unsigned
-// atomicMax on the fp32 bit patterns (valid for values >= 0) into the
+// Work unit: one 256-column stripe of a contiguous range of rows of C or of W;
+// one thread block per unit.  A producer warp streams the unit as 32-row x
+// 256-column boxes (16 KB of bf16) by TMA into a ring of shared-memory stages;
+// eight consumer warps take four rows of every box each, lane l reading the
+// 16 bytes of columns 8l..8l+7 of a row (one contiguous 512-byte row per warp
+// instruction, free of bank conflicts).  Bytes in flight are set by the ring
+// (six stages per block, two blocks per SM), not by registers.
+// |x| is taken on the bf16 bit patterns with the sign bit cleared: for
+// non-negative bf16 values the integer order of the patterns is the numeric
+// order, so the max is exact and needs no conversion until the end.  Rows past
+// the matrix end are zero-filled by TMA and rows past the unit's end belong to
+// the same matrix, so neither changes a max.  Block results are merged with an
+// unsigned atomicMax on the fp32 bit patterns (valid for values >= 0) into the
 // workspace.  The last block of each stripe to finish (a per-stripe arrival
 // counter) turns the stripe's maxima into s:
 //     s_j = max( max(mx_j, 1e-8)^a / max(mw_j, 1e-8)^(1-a), 1e-8 )
 // evaluated in double and rounded once to fp32 (calibrate_smoothquant), after
 // merging the caller's running maximum (SmoothQuantW8A8.calibrate).
-// Workspace layout (cleared by a memset before the launch): mx[K], mw[K]
-// (fp32 bit patterns), count[stripes].
-constexpr int kColThreads = 256;
-constexpr int kColStripe = 256;
-constexpr int kColBatch = 8;                              // rows per warp per batch
-constexpr int kColBatchRows = kColBatch * (kColThreads / 32);  // rows per block per batch
+// Workspace layout: mx[K], mw[K] (fp32 bit patterns), count[stripes].  It must
+// be zero when the kernel starts, and the last block of each stripe zeroes the
+// stripe's words again once it has read them, so a call leaves the workspace
+// zero (a caller workspace is cleared by a memset first, the library's own
+// scratch is not).
+constexpr int kColConsumers = 8;                                 // consumer warps
+constexpr int kColThreads = 32 * (kColConsumers + 1);            // + one producer warp
+constexpr int kColStripe = 256;                                  // columns per box (TMA box limit)
+constexpr int kColBoxRows = 4 * kColConsumers;                   // rows per box
+constexpr int kColStageBytes = kColStripe * kColBoxRows * 2;     // 16 KB
+#ifndef SQ_COLMAX_STAGES  // build-time tuning knob: ring depth per block
+#define SQ_COLMAX_STAGES 6
+#endif
+constexpr int kColStages = SQ_COLMAX_STAGES;
+constexpr int kColRedOffset = kColStages * kColStageBytes;       // [8][256] u32 block reduction
+constexpr int kColBarOffset = kColRedOffset + kColConsumers * kColStripe * 4;
+constexpr int kColFlagOffset = kColBarOffset + 2 * kColStages * 8;
+constexpr int kColSmemBytes = kColFlagOffset + 16 + 1024;        // + alignment slack
+
+struct ColmaxParams {
+  int K, box_cols, stripes;
+  int chunks_c, chunks_w;  // row ranges per stripe of C and of W
+  int rows_c, rows_w;      // rows per range (multiples of kColBoxRows)
+  int R, N;
+  uint32_t* ws;
+  double alpha;
+  float* mx_inout;
+  float* s;
+  unsigned long long timeout_ns;
+};
 
 __device__ __forceinline__ float smoothing_factor(float mx, float mw, double alpha) {
   const double floor = static_cast<double>(kClampFloor);
@@ -48,123 +117,190 @@ __device__ __forceinline__ float smoothing_factor(float mx, float mw, double alp
   return __double2float_rn(v);
 }
 
-__device__ __forceinline__ void colmax_load_batch(uint4 (&v)[kColBatch], const uint16_t* base, int64_t r, int64_t r1,
-                                                  int K) {
-#pragma unroll
-  for (int i = 0; i < kColBatch; ++i)
-    v[i] = (r + i < r1) ? __ldcg(reinterpret_cast<const uint4*>(base + (r + i) * K)) : make_uint4(0u, 0u, 0u, 0u);
-}
-
-__global__ void __launch_bounds__(kColThreads) colmax_kernel(const uint16_t* __restrict__ C, int64_t R,
-                                                             const uint16_t* __restrict__ W, int64_t N, int K,
-                                                             uint32_t* ws, int chunks_c, int chunks_w,
-                                                             int64_t rows_c, int64_t rows_w, double alpha,
-                                                             float* __restrict__ mx_inout, float* __restrict__ s) {
-  griddep_wait();
-  griddep_launch_dependents();
-  const bool is_w = blockIdx.z == 1;
-  const int chunks = is_w ? chunks_w : chunks_c;
-  if (static_cast<int>(blockIdx.y) >= chunks) return;  // not counted: only chunks_c + chunks_w blocks arrive
-  const uint16_t* A = is_w ? W : C;
-  const int64_t rows = is_w ? N : R;
-  const int64_t chunk_rows = is_w ? rows_w : rows_c;
-  uint32_t* ws_mx = ws;
-  uint32_t* ws_mw = ws + K;
-  unsigned int* count = reinterpret_cast<unsigned int*>(ws + 2 * K);
-  uint32_t* out = is_w ? ws_mw : ws_mx;
+__global__ void __launch_bounds__(kColThreads) colmax_kernel(const __grid_constant__ CUtensorMap tmC,
+                                                             const __grid_constant__ CUtensorMap tmW,
+                                                             const ColmaxParams p) {
+  SQ_BLOCK_TRACE(0);
+  extern __shared__ uint8_t col_smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(col_smem_raw) + 1023) & ~uintptr_t(1023));
+  uint32_t* red = reinterpret_cast<uint32_t*>(smem + kColRedOffset);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kColBarOffset);
+  uint64_t* empty = full + kColStages;
+  volatile int* flags = reinterpret_cast<volatile int*>(smem + kColFlagOffset);  // [0] abort, [1] last block
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int col = blockIdx.x * kColStripe + lane * 8;
-  const int64_t r0 = static_cast<int64_t>(blockIdx.y) * chunk_rows;
-  const int64_t r1 = min(rows, r0 + chunk_rows);
+  int b = static_cast<int>(blockIdx.x);
+  const bool is_w = b >= p.stripes * p.chunks_c;
+  if (is_w) b -= p.stripes * p.chunks_c;
+  const int stripe = b % p.stripes, chunk = b / p.stripes;
+  const int rows = is_w ? p.N : p.R;
+  const int chunk_rows = is_w ? p.rows_w : p.rows_c;
+  const int r0 = chunk * chunk_rows;
+  const int r1 = min(rows, r0 + chunk_rows);
+  const int nbox = (r1 - r0 + kColBoxRows - 1) / kColBoxRows;
+  const CUtensorMap* map = is_w ? &tmW : &tmC;
+  const int row_bytes = p.box_cols * 2;  // a box row in shared memory
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kColStages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], kColConsumers);
+    }
+    flags[0] = 0;
+    fence_mbar_init();
+  }
+  if (warp == kColConsumers && lane == 0) tma_prefetch_desc(map);
+  __syncthreads();
+  griddep_wait();
+  SQ_BLOCK_MARK(1);
+  griddep_launch_dependents();
 
   uint32_t m0 = 0, m1 = 0, m2 = 0, m3 = 0;  // packed pairs of |bf16| patterns
-  if (col < K) {
-    const uint16_t* base = A + col;
-    uint4 cur[kColBatch], nxt[kColBatch];
-    int64_t r = r0 + warp * kColBatch;
-    colmax_load_batch(cur, base, r, r1, K);
-    for (int64_t b0 = r0; b0 < r1; b0 += kColBatchRows, r += kColBatchRows) {
-      const bool more = b0 + kColBatchRows < r1;
-      if (more) colmax_load_batch(nxt, base, r + kColBatchRows, r1, K);
-#pragma unroll
-      for (int i = 0; i < kColBatch; ++i) {
-        m0 = __vmaxu2(m0, cur[i].x & 0x7FFF7FFFu);
-        m1 = __vmaxu2(m1, cur[i].y & 0x7FFF7FFFu);
-        m2 = __vmaxu2(m2, cur[i].z & 0x7FFF7FFFu);
-        m3 = __vmaxu2(m3, cur[i].w & 0x7FFF7FFFu);
+  if (warp == kColConsumers) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      const uint32_t box_bytes = static_cast<uint32_t>(row_bytes * kColBoxRows);
+      int j = 0;
+      for (; j < nbox; ++j) {
+        const int st = j % kColStages;
+        if (j >= kColStages &&
+            (flags[0] || !mbar_wait_bounded(&empty[st], static_cast<uint32_t>((j / kColStages - 1) & 1), p.timeout_ns))) {
+          flags[0] = 1;
+          atomicOr(&g_sq_quant_status, 1u);
+          break;
+        }
+        mbar_arrive_expect_tx(&full[st], box_bytes);
+        tma_load_2d(smem + st * kColStageBytes, map, stripe * p.box_cols, r0 + j * kColBoxRows, &full[st]);
       }
-      if (!more) break;
+      if (j < nbox) {
+        // gave up: let the copies already issued land before the block exits
+        for (int q = max(0, j - kColStages); q < j; ++q)
+          (void)mbar_wait_bounded(&full[q % kColStages], static_cast<uint32_t>((q / kColStages) & 1), p.timeout_ns);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ consumers
+    const bool active = lane * 8 < p.box_cols;
+    const uint8_t* my_rows = smem + warp * 4 * row_bytes + lane * 16;
+    for (int j = 0; j < nbox; ++j) {
+      const int st = j % kColStages;
+      if (flags[0] || !mbar_wait_bounded(&full[st], static_cast<uint32_t>((j / kColStages) & 1), p.timeout_ns)) {
+        flags[0] = 1;
+        atomicOr(&g_sq_quant_status, 1u);
+        break;
+      }
+      if (active) {
+        const uint8_t* src = my_rows + st * kColStageBytes;
 #pragma unroll
-      for (int i = 0; i < kColBatch; ++i) cur[i] = nxt[i];
+        for (int i = 0; i < 4; ++i) {
+          const uint4 v = *reinterpret_cast<const uint4*>(src + i * row_bytes);
+          m0 = __vmaxu2(m0, v.x & 0x7FFF7FFFu);
+          m1 = __vmaxu2(m1, v.y & 0x7FFF7FFFu);
+          m2 = __vmaxu2(m2, v.z & 0x7FFF7FFFu);
+          m3 = __vmaxu2(m3, v.w & 0x7FFF7FFFu);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[st]);
+    }
+    const uint32_t m[4] = {m0, m1, m2, m3};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      red[warp * kColStripe + lane * 8 + 2 * i] = (m[i] & 0xFFFFu) << 16;  // fp32 pattern of the bf16 value
+      red[warp * kColStripe + lane * 8 + 2 * i + 1] = m[i] & 0xFFFF0000u;
     }
   }
-  __shared__ uint32_t red[kColThreads / 32][kColStripe];
-  __shared__ bool last;
-  const uint32_t m[4] = {m0, m1, m2, m3};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    red[warp][lane * 8 + 2 * i] = (m[i] & 0xFFFFu) << 16;  // fp32 pattern of the bf16 value
-    red[warp][lane * 8 + 2 * i + 1] = m[i] & 0xFFFF0000u;
-  }
   __syncthreads();
-  uint32_t vmax = 0;
+  uint32_t* ws_mx = p.ws;
+  uint32_t* ws_mw = p.ws + p.K;
+  unsigned int* count = reinterpret_cast<unsigned int*>(p.ws + 2 * p.K);
+  const int c = stripe * kColStripe + static_cast<int>(threadIdx.x);
+  if (threadIdx.x < kColStripe) {
+    uint32_t vmax = 0;
 #pragma unroll
-  for (int w = 0; w < kColThreads / 32; ++w) vmax = max(vmax, red[w][threadIdx.x]);
-  const int c = blockIdx.x * kColStripe + threadIdx.x;
-  if (c < K && vmax != 0u) atomicMax(out + c, vmax);
+    for (int w = 0; w < kColConsumers; ++w) vmax = max(vmax, red[w * kColStripe + threadIdx.x]);
+    if (c < p.K && vmax != 0u) atomicMax((is_w ? ws_mw : ws_mx) + c, vmax);
+  }
 
   // arrival: the last block of this stripe computes s for the stripe
   __threadfence();
   __syncthreads();
   if (threadIdx.x == 0) {
-    const unsigned int total = static_cast<unsigned int>(chunks_c + chunks_w);
-    last = (atomicAdd(count + blockIdx.x, 1u) == total - 1u);
+    const unsigned int total = static_cast<unsigned int>(p.chunks_c + p.chunks_w);
+    flags[1] = (atomicAdd(count + stripe, 1u) == total - 1u) ? 1 : 0;
   }
   __syncthreads();
-  if (!last || c >= K) return;
+  if (!flags[1] || threadIdx.x >= kColStripe) return;
   __threadfence();
+  if (threadIdx.x == 0) count[stripe] = 0u;  // every block of the stripe has arrived
+  if (c >= p.K) return;
   float mx = __uint_as_float(__ldcg(ws_mx + c));
-  if (mx_inout != nullptr) {  // running max over calibration batches
-    mx = fmaxf(mx, mx_inout[c]);
-    mx_inout[c] = mx;
+  const float mw = __uint_as_float(__ldcg(ws_mw + c));
+  ws_mx[c] = 0u;  // leave the workspace as it was found: zero
+  ws_mw[c] = 0u;
+  if (p.mx_inout != nullptr) {  // running max over calibration batches
+    mx = fmaxf(mx, p.mx_inout[c]);
+    p.mx_inout[c] = mx;
   }
-  s[c] = smoothing_factor(mx, __uint_as_float(__ldcg(ws_mw + c)), alpha);
+  p.s[c] = smoothing_factor(mx, mw, p.alpha);
 }
 
 static int col_stripes(int64_t K) { return static_cast<int>((K + kColStripe - 1) / kColStripe); }
 
 size_t calibrate_workspace_words(int64_t K) { return static_cast<size_t>(2 * K + col_stripes(K)); }
 
-// rows per block for `rows` rows split into about `g` chunks (multiple of a batch)
+// rows per range for `rows` rows split into about `g` ranges (multiple of a box)
 static int64_t chunk_rows_for(int64_t rows, int64_t g) {
   const int64_t per = (rows + g - 1) / g;
-  return std::max<int64_t>(kColBatchRows, (per + kColBatchRows - 1) / kColBatchRows * kColBatchRows);
+  return std::max<int64_t>(kColBoxRows, (per + kColBoxRows - 1) / kColBoxRows * kColBoxRows);
 }
 
 cudaError_t launch_calibrate(const uint16_t* C, int64_t R, int64_t K, const uint16_t* W, int64_t N, float alpha,
-                             float* s, float* mx_inout, void* ws, cudaStream_t st, const DeviceInfo& dev) {
-  cudaError_t e = cudaMemsetAsync(ws, 0, calibrate_workspace_words(K) * sizeof(uint32_t), st);
-  if (e != cudaSuccess) return e;
-  static bool attr_set = false;  // idempotent attribute; a race only repeats the call
-  if (!attr_set) {
-    e = cudaFuncSetAttribute(colmax_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, kCarveoutMaxShared);
+                             float* s, float* mx_inout, void* ws, bool ws_is_zero, cudaStream_t st,
+                             const DeviceInfo& dev) {
+  cudaError_t e = cudaSuccess;
+  if (!ws_is_zero) {
+    e = cudaMemsetAsync(ws, 0, calibrate_workspace_words(K) * sizeof(uint32_t), st);
     if (e != cudaSuccess) return e;
-    attr_set = true;
   }
-  // about two blocks per SM over all stripes, split between C and W by rows
+  static int per_sm = 0;  // idempotent set-up; a race only repeats it
+  if (per_sm == 0) {
+    e = cudaFuncSetAttribute(colmax_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kColSmemBytes);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(colmax_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, kCarveoutMaxShared);
+    int n = 0;
+    if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, colmax_kernel, kColThreads, kColSmemBytes);
+    if (e != cudaSuccess) return e;
+    per_sm = std::max(n, 1);
+  }
+  const int box_cols = static_cast<int>(std::min<int64_t>(K, kColStripe));
+  CUtensorMap tmC, tmW;
+  if (!make_tmap_2d(&tmW, W, N, K, 2, box_cols, kColBoxRows) ||
+      !make_tmap_2d(&tmC, R > 0 ? C : W, R > 0 ? R : N, K, 2, box_cols, kColBoxRows))
+    return cudaErrorInvalidValue;
+  // about one wave of resident blocks over all stripes, split between C and W by rows
   const int stripes = col_stripes(K);
-  const int64_t g_total = std::max<int64_t>(1, (2 * static_cast<int64_t>(dev.sm_count) + stripes - 1) / stripes);
-  int64_t g_w = std::max<int64_t>(1, (g_total * N + (N + R) - 1) / (N + R));
-  int64_t g_c = R > 0 ? std::max<int64_t>(1, g_total - g_w) : 0;
-  const int64_t rows_w = chunk_rows_for(N, g_w);
-  const int64_t rows_c = R > 0 ? chunk_rows_for(R, g_c) : kColBatchRows;
-  const int chunks_w = static_cast<int>((N + rows_w - 1) / rows_w);
-  const int chunks_c = R > 0 ? static_cast<int>((R + rows_c - 1) / rows_c) : 0;
-  dim3 grid(static_cast<unsigned>(stripes), static_cast<unsigned>(std::max(chunks_c, chunks_w)), 2);
-  return launch_pdl(colmax_kernel, grid, dim3(kColThreads), 0, st, C, R, W, N, static_cast<int>(K),
-                    static_cast<uint32_t*>(ws), chunks_c, chunks_w, rows_c, rows_w, static_cast<double>(alpha),
-                    mx_inout, s);
+  const int64_t g_total = std::max<int64_t>(1, static_cast<int64_t>(per_sm) * dev.sm_count / stripes);
+  const int64_t g_w = std::max<int64_t>(1, (g_total * N + (N + R) / 2) / (N + R));
+  const int64_t g_c = R > 0 ? std::max<int64_t>(1, g_total - g_w) : 0;
+  ColmaxParams p;
+  p.K = static_cast<int>(K);
+  p.box_cols = box_cols;
+  p.stripes = stripes;
+  p.rows_w = static_cast<int>(chunk_rows_for(N, g_w));
+  p.rows_c = R > 0 ? static_cast<int>(chunk_rows_for(R, g_c)) : kColBoxRows;
+  p.chunks_w = static_cast<int>((N + p.rows_w - 1) / p.rows_w);
+  p.chunks_c = R > 0 ? static_cast<int>((R + p.rows_c - 1) / p.rows_c) : 0;
+  p.R = static_cast<int>(R);
+  p.N = static_cast<int>(N);
+  p.ws = static_cast<uint32_t*>(ws);
+  p.alpha = static_cast<double>(alpha);
+  p.mx_inout = mx_inout;
+  p.s = s;
+  p.timeout_ns = kQuantWaitTimeoutNs;
+  const int64_t grid = static_cast<int64_t>(stripes) * (p.chunks_c + p.chunks_w);
+  return launch_pdl(colmax_kernel, dim3(static_cast<unsigned>(grid)), dim3(kColThreads),
+                    static_cast<size_t>(kColSmemBytes), st, tmC, tmW, p);
 }
 
 // ============================================ calibration without allocation
@@ -176,6 +312,27 @@ cudaError_t launch_calibrate(const uint16_t* C, int64_t R, int64_t K, const uint
 // Host code must not pass the symbol itself to a kernel (on the host it only
 // names a stand-in object); the device address comes from cudaGetSymbolAddress.
 static __device__ __align__(256) uint32_t g_calib_noalloc_scratch[2 * kNoAllocMaxK + kNoAllocMaxK / 256];
+
+// Reads the status word; clearing it also re-zeroes the no-allocation scratch,
+// which a timed-out calibration may have left dirty.
+cudaError_t read_quant_status(uint32_t* flags, bool clear) {
+  unsigned int v = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(&v, g_sq_quant_status, sizeof(v));
+  if (e != cudaSuccess) return e;
+  if (clear) {
+    const unsigned int z = 0;
+    e = cudaMemcpyToSymbol(g_sq_quant_status, &z, sizeof(z));
+    if (e != cudaSuccess) return e;
+    if (v != 0u) {
+      void* p = nullptr;
+      e = cudaGetSymbolAddress(&p, g_calib_noalloc_scratch);
+      if (e == cudaSuccess) e = cudaMemset(p, 0, sizeof(g_calib_noalloc_scratch));
+      if (e != cudaSuccess) return e;
+    }
+  }
+  *flags = v;
+  return cudaSuccess;
+}
 
 cudaError_t launch_calibrate_noalloc(const uint16_t* C, int64_t R, int64_t K, const uint16_t* W, int64_t N,
                                      float alpha, float* s, float* mx_inout, cudaStream_t st, const DeviceInfo& dev) {
@@ -195,9 +352,9 @@ cudaError_t launch_calibrate_noalloc(const uint16_t* C, int64_t R, int64_t K, co
     }
     ws = addr[dev.device];
   }
-  // launch_calibrate clears the words it uses before the reduction, so the
-  // previous call's contents never leak into this one.
-  return launch_calibrate(C, R, K, W, N, alpha, s, mx_inout, ws, st, dev);
+  // The array is zero at load time and every call leaves it zero, so no memset
+  // is needed (read_quant_status(clear) re-zeroes it after a timed-out call).
+  return launch_calibrate(C, R, K, W, N, alpha, s, mx_inout, ws, /*ws_is_zero=*/true, st, dev);
 }
 
 // ===================================================== row quantisers (K2/K3)
@@ -251,7 +408,9 @@ __global__ void __launch_bounds__(kRowThreads) row_quant_kernel(const uint16_t* 
   int64_t row = static_cast<int64_t>(blockIdx.x) * RPC + slot;
   const int64_t row_step = static_cast<int64_t>(gridDim.x) * RPC;
 
+  SQ_BLOCK_TRACE(kMul ? 1 : 2);
   griddep_wait();
+  SQ_BLOCK_MARK(1);
   griddep_launch_dependents();
   uint4 xv[VPL];
   load_row_vectors<VPL, WPR>(xv, src, row, rows, K, nvec, wsub, lane);  // in flight during the table build
@@ -349,18 +508,25 @@ static cudaError_t launch_rq(const uint16_t* src, int64_t rows, int K, const flo
   return launch_pdl(kern, dim3(static_cast<unsigned>(grid)), dim3(kRowThreads), smem, st, src, rows, K, s, q, scale);
 }
 
+#ifndef SQ_RQ_VPL  // build-time tuning knob: most 16-byte vectors a lane holds (4 or 8)
+#define SQ_RQ_VPL 4
+#endif
+
 template <bool kMul>
 static cudaError_t dispatch_rq(const uint16_t* src, int64_t rows, int K, const float* s, int8_t* q, float* scale,
                                cudaStream_t st, const DeviceInfo& dev) {
-  // vectors per lane (up to 8), then warps per row (up to 8) to cover K
+  // vectors per lane (up to SQ_RQ_VPL), then warps per row (up to 8) to cover K
+  constexpr int V = SQ_RQ_VPL;
+  static_assert(V == 4 || V == 8, "SQ_RQ_VPL must be 4 or 8");
   const int nvec = K / 8;
   if (nvec <= 32) return launch_rq<kMul, 1, 1>(src, rows, K, s, q, scale, st, dev);
   if (nvec <= 64) return launch_rq<kMul, 1, 2>(src, rows, K, s, q, scale, st, dev);
   if (nvec <= 128) return launch_rq<kMul, 1, 4>(src, rows, K, s, q, scale, st, dev);
-  if (nvec <= 256) return launch_rq<kMul, 1, 8>(src, rows, K, s, q, scale, st, dev);
-  if (nvec <= 512) return launch_rq<kMul, 2, 8>(src, rows, K, s, q, scale, st, dev);
-  if (nvec <= 1024) return launch_rq<kMul, 4, 8>(src, rows, K, s, q, scale, st, dev);
-  return launch_rq<kMul, 8, 8>(src, rows, K, s, q, scale, st, dev);
+  if (nvec <= 32 * V) return launch_rq<kMul, 1, V>(src, rows, K, s, q, scale, st, dev);
+  if (nvec <= 64 * V) return launch_rq<kMul, 2, V>(src, rows, K, s, q, scale, st, dev);
+  if (nvec <= 128 * V) return launch_rq<kMul, 4, V>(src, rows, K, s, q, scale, st, dev);
+  if (nvec <= 256 * V) return launch_rq<kMul, 8, V>(src, rows, K, s, q, scale, st, dev);
+  return launch_rq<kMul, 8, 8>(src, rows, K, s, q, scale, st, dev);  // K up to 16384
 }
 
 cudaError_t launch_row_quant(bool multiply, const uint16_t* src, int64_t rows, int64_t K, const float* s, int8_t* q,
