@@ -283,6 +283,7 @@ def run_ours(args, wl, rank, world, local_rank):
     Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
     ws_cal = torch.empty(sq.sq_calibrate_workspace_bytes(K), dtype=torch.uint8, device=dev)
     ws_fwd = torch.empty(max(sq.sq_forward_workspace_bytes(M, N, K), 16), dtype=torch.uint8, device=dev)
+    ws_lin = torch.empty(max(sq.sq_workspace_bytes(M, N, K), 16), dtype=torch.uint8, device=dev)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     flush_read = torch.ones(FLUSH_READ_BYTES // 4, dtype=torch.int32, device=dev)
 
@@ -290,7 +291,7 @@ def run_ours(args, wl, rank, world, local_rank):
         "sq_calibrate": lambda: sq.sq_calibrate(C, W, wl.alpha_f32, s=s, workspace=ws_cal),
         "sq_prepare_weight": lambda: sq.sq_prepare_weight(W, s, Wq=Wq, w_scale=w_scale),
         "sq_quantize_act": lambda: sq.sq_quantize_act(X, s, Xq=Xq, x_scale=x_scale),
-        "sq_linear": lambda: sq.sq_linear(Xq, x_scale, Wq, w_scale, b, Y=Y),
+        "sq_linear": lambda: sq.sq_linear(Xq, x_scale, Wq, w_scale, b, Y=Y, workspace=ws_lin),
     }
     launches_per_call = {"sq_calibrate": 1, "sq_prepare_weight": 1, "sq_quantize_act": 1, "sq_linear": 1}
     names = list(calls)

@@ -159,9 +159,16 @@ SQ_API sq_status sq_quantize_act(const sq_bf16* X, int64_t M, int64_t K, const f
  *   Y[M][N]   OUT bf16.  The int32 accumulation is exact (|acc| <= 127^2 K,
  *             K <= 133143); the epilogue runs in fp32 and rounds to bf16
  *             (nearest even), i.e. within one bf16 ulp of the exact value.
- *   workspace may be NULL when sq_workspace_bytes(M, N, K) == 0.
+ *   workspace  optional device scratch (16-byte aligned; contents on entry
+ *              ignored).  sq_workspace_bytes(M, N, K) gives the size that lets
+ *              the GEMM split K over pairs of CTAs when the output has few
+ *              128 x 256 tiles (at most half as many as SMs), exchanging
+ *              partial sums through it (64 KB per CTA); 0 when no such split
+ *              applies.  NULL or less than that size selects a path that needs
+ *              none (same results, slower for such shapes).
  * Runs the tcgen05 (kind::i8) GEMM: TMA-fed shared-memory tiles, int32
- * accumulators in tensor memory, fused dequant + bias epilogue.
+ * accumulators in tensor memory, fused dequant + bias epilogue.  M <= 32 uses
+ * a weight-streaming kernel instead (split-K over a thread-block cluster).
  */
 SQ_API size_t sq_workspace_bytes(int64_t M, int64_t N, int64_t K);
 SQ_API sq_status sq_linear(const int8_t* Xq, const float* x_scale, const int8_t* Wq,
@@ -175,7 +182,8 @@ SQ_API sq_status sq_linear(const int8_t* Xq, const float* x_scale, const int8_t*
  *
  *   X[M][K] bf16, s[K], Wq[N][K], w_scale[N], bias[N] or NULL -> Y[M][N] bf16
  *   workspace  at least sq_forward_workspace_bytes(M, N, K) bytes (holds the
- *              intermediate Xq and x_scale); contents on entry are ignored.
+ *              intermediate Xq and x_scale, then sq_linear's workspace);
+ *              contents on entry are ignored.
  * The codes and scales are identical to those of sq_quantize_act.
  */
 SQ_API size_t sq_forward_workspace_bytes(int64_t M, int64_t N, int64_t K);
@@ -209,8 +217,8 @@ SQ_API sq_status sq_device_status(uint32_t* flags, int clear);
 SQ_API void sq_debug_fail_after(int n);
 
 /* sq_debug_pipeline_stall -- device-side failure test: while enabled
- * (enable != 0), the general GEMM used by sq_linear / sq_forward / sq_gemm_s32
- * for M > 32 never loads its first pipeline stage and every pipeline wait gives
+ * (enable != 0), the GEMM kernels used by sq_linear / sq_forward / sq_gemm_s32
+ * for M > 32 never load their first pipeline stage and every pipeline wait gives
  * up after timeout_ns (<= 0: the normal 2 s).  The kernel then sets bit 0 of
  * the device status word, drains its copies in flight, frees its tensor memory
  * and returns: the call's output is invalid, the CUDA context stays usable and

@@ -9,7 +9,7 @@ import pytest
 import torch
 
 from oracle import smoothquant as O
-from tests.helpers import dev, host
+from tests.helpers import assert_y_close, dev, host, host_bf16_bits
 
 pytestmark = pytest.mark.gpu
 
@@ -42,4 +42,34 @@ def test_pipeline_wait_timeout_is_reported_and_the_context_survives(sq):
     # the context is intact: the same call now returns the exact product
     acc = host(sq.sq_gemm_s32(Xq_d, Wq_d))
     assert np.array_equal(acc.astype(np.int64), O.int8_gemm(Xq, Wq))
+    assert sq.sq_device_status() == 0
+
+
+def test_split_k_wait_timeout_is_reported_and_the_context_survives(sq):
+    """The same failure in the split-K GEMM (few 128 x 256 tiles, K split over a
+    CTA pair, partial sums exchanged through the workspace): the stalled CTA
+    still stores its (zero) partial, so its partner never waits for it."""
+    rng = np.random.default_rng(98)
+    M, N, K = 256, 512, 4096  # 4 tiles of 128 x 256: split-K when a workspace is given
+    Xq = rng.integers(-127, 128, (M, K), dtype=np.int64).astype(np.int8)
+    Wq = rng.integers(-127, 128, (N, K), dtype=np.int64).astype(np.int8)
+    xs = (rng.random(M, dtype=np.float32) * 1e-3 + 1e-4).astype(np.float32)
+    ws = (rng.random(N, dtype=np.float32) * 1e-3 + 1e-4).astype(np.float32)
+    assert sq.sq_workspace_bytes(M, N, K) > 0
+    args = (dev(Xq), dev(xs), dev(Wq), dev(ws))
+    assert sq.sq_device_status(clear=True) == 0
+    try:
+        sq.sq_debug_pipeline_stall(True, 50_000_000)
+        t0 = time.perf_counter()
+        sq.sq_linear(*args)
+        torch.cuda.synchronize()
+        elapsed = time.perf_counter() - t0
+    finally:
+        sq.sq_debug_pipeline_stall(False)
+    flags = sq.sq_device_status(clear=True)
+    assert flags & 1, "the stalled split-K pipeline was not reported"
+    assert elapsed < 5.0
+    Y = sq.sq_linear(*args)
+    torch.cuda.synchronize()
+    assert_y_close(host_bf16_bits(Y), O.int8_gemm(Xq, Wq), xs, ws, None, "split-K after a timeout")
     assert sq.sq_device_status() == 0

@@ -217,17 +217,23 @@ sq_status sq_quantize_act(const sq_bf16* X, int64_t M, int64_t K, const float* s
 }
 
 // ------------------------------------------------------------- int8 linear
+// SMs assumed when no device can be queried (a B200), so that sizes asked
+// before a device is current are the ones a B200 will want.
+constexpr int kDefaultSmCount = 148;
+
 size_t sq_workspace_bytes(int64_t M, int64_t N, int64_t K) {
-  (void)M;
-  (void)N;
-  (void)K;
-  return 0;
+  if (M <= sq::kSmallMaxM || M <= 0 || N <= 0 || K <= 0) return 0;  // the few-token kernel needs none
+  sq::DeviceInfo dev;
+  const int sms = sq::current_device_info(&dev) == cudaSuccess ? dev.sm_count : kDefaultSmCount;
+  return sq::gemm_workspace_bytes(M, N, K, sms);
 }
 
 static sq_status gemm_common(const int8_t* Xq, const float* x_scale, const int8_t* Wq, const float* w_scale,
                              const sq_bf16* bias, int64_t M, int64_t N, int64_t K, void* out, sq::Epilogue epi,
-                             void* stream, const sq::DeviceInfo& dev) {
+                             void* stream, const sq::DeviceInfo& dev, void* ws = nullptr, size_t ws_bytes = 0) {
   sq::GemmArgs a;
+  a.ws = ws;
+  a.ws_bytes = ws_bytes;
   a.A = Xq;
   a.B = Wq;
   a.M = M;
@@ -255,9 +261,7 @@ sq_status sq_linear(const int8_t* Xq, const float* x_scale, const int8_t* Wq, co
   SQ_NONNULL(w_scale);
   SQ_NONNULL(Y);
   if (bias != nullptr && !aligned16(bias)) return fail(SQ_ERR_ALIGN, "bias is not 16-byte aligned");
-  if (workspace_bytes < sq_workspace_bytes(M, N, K))
-    return fail(SQ_ERR_WORKSPACE, "workspace smaller than sq_workspace_bytes(M, N, K)");
-  (void)workspace;
+  if (workspace != nullptr && !aligned16(workspace)) return fail(SQ_ERR_ALIGN, "workspace is not 16-byte aligned");
   sq::DeviceInfo dev;
   SQ_TRY(prologue(&dev));
   if (M <= sq::kSmallMaxM) {  // few tokens: weight-streaming split-K kernel
@@ -266,7 +270,8 @@ sq_status sq_linear(const int8_t* Xq, const float* x_scale, const int8_t* Wq, co
     cudaError_t e = sq::launch_small_m(a, static_cast<cudaStream_t>(stream), dev, &why);
     if (e != cudaErrorNotSupported) return cuda_status(e, why);
   }
-  return gemm_common(Xq, x_scale, Wq, w_scale, bias, M, N, K, Y, sq::Epilogue::kBf16Dequant, stream, dev);
+  return gemm_common(Xq, x_scale, Wq, w_scale, bias, M, N, K, Y, sq::Epilogue::kBf16Dequant, stream, dev,
+                     workspace, workspace == nullptr ? 0 : workspace_bytes);
 }
 
 // ----------------------------------------------------------- fused forward
@@ -302,11 +307,14 @@ sq_status sq_forward(const sq_bf16* X, const float* s, const int8_t* Wq, const f
     if (e != cudaErrorNotSupported) return cuda_status(e, why);
   }
   int8_t* Xq = static_cast<int8_t*>(workspace);
-  float* xs = reinterpret_cast<float*>(static_cast<char*>(workspace) + forward_xq_bytes(M, K));
+  const size_t xs_off = forward_xq_bytes(M, K);
+  float* xs = reinterpret_cast<float*>(static_cast<char*>(workspace) + xs_off);
+  const size_t gemm_off = xs_off + round_up(static_cast<size_t>(M) * sizeof(float), 256);
   sq_status st = cuda_status(
       sq::launch_row_quant(false, X, M, K, s, Xq, xs, static_cast<cudaStream_t>(stream), dev), "quantize_act launch");
   if (st != SQ_OK) return st;
-  return gemm_common(Xq, xs, Wq, w_scale, bias, M, N, K, Y, sq::Epilogue::kBf16Dequant, stream, dev);
+  return gemm_common(Xq, xs, Wq, w_scale, bias, M, N, K, Y, sq::Epilogue::kBf16Dequant, stream, dev,
+                     static_cast<char*>(workspace) + gemm_off, workspace_bytes - gemm_off);
 }
 
 // ---------------------------------------------------------------- test hook

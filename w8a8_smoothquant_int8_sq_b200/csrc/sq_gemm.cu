@@ -59,8 +59,8 @@ constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // 2 s per wait
 #ifndef SQ_GEMM_BN
 #define SQ_GEMM_BN 0
 #endif
-#ifndef SQ_GEMM_SPLITK  // 1: split K over a cluster when 128 x 256 tiles do not fill the GPU
-#define SQ_GEMM_SPLITK 0
+#ifndef SQ_GEMM_SPLITK  // 1: split K over a CTA pair when 128 x 256 tiles fill at most half the SMs
+#define SQ_GEMM_SPLITK 1
 #endif
 #ifndef SQ_GEMM_CHAINS128  // accumulator chains for 128-wide tiles (1 or 2)
 #define SQ_GEMM_CHAINS128 2
@@ -572,9 +572,9 @@ cudaError_t run_small(const SmallArgs& a, cudaStream_t st, const DeviceInfo& dev
   return e;
 }
 
-template <int EPI>
-cudaError_t run_splitk(const GemmArgs& a, int S, cudaStream_t st, const DeviceInfo& dev, const char** why) {
-  (void)dev;
+// K split over a CTA pair (cluster of 2); the pair exchanges partial sums
+// through `a.ws` (at least splitk_workspace_bytes).
+cudaError_t run_splitk(const GemmArgs& a, cudaStream_t st, const char** why) {
   CUtensorMap tmA, tmB;
   if (!make_tmap_i8(&tmA, a.A, a.M, a.K, kBM) || !make_tmap_i8(&tmB, a.B, a.N, a.K, kSkBN)) {
     *why = "cuTensorMapEncodeTiled failed or unavailable";
@@ -586,15 +586,17 @@ cudaError_t run_splitk(const GemmArgs& a, int S, cudaStream_t st, const DeviceIn
   p.K = static_cast<int>(a.K);
   p.num_m_blocks = static_cast<int>((a.M + kBM - 1) / kBM);
   p.nk = static_cast<int>((a.K + kBK - 1) / kBK);
-  p.kb_per_split = (p.nk + S - 1) / S;
+  p.kb_per_split = (p.nk + 1) / 2;
   p.x_scale = a.x_scale;
   p.w_scale = a.w_scale;
   p.bias = a.bias;
-  p.out = a.out;
-  const int elem = (EPI == 0) ? 2 : 4;
-  p.vec_ok = ((a.N * elem) % 16 == 0) && (reinterpret_cast<uintptr_t>(a.out) % 16 == 0);
+  p.out = static_cast<uint16_t*>(a.out);
+  p.part = static_cast<uint4*>(a.ws);
+  p.vec_ok = ((a.N * 2) % 16 == 0) && (reinterpret_cast<uintptr_t>(a.out) % 16 == 0);
+  p.skip_first_load = g_debug_stall.load() ? 1 : 0;
+  p.timeout_ns = g_debug_stall.load() ? g_debug_timeout_ns.load() : kWaitTimeoutNs;
   const int tiles = p.num_m_blocks * static_cast<int>((a.N + kSkBN - 1) / kSkBN);
-  auto kern = gemm_i8_splitk_kernel<EPI>;
+  auto kern = gemm_i8_splitk_kernel;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSkAlloc);
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, kCarveoutMaxShared);
@@ -602,8 +604,8 @@ cudaError_t run_splitk(const GemmArgs& a, int S, cudaStream_t st, const DeviceIn
     *why = "cudaFuncSetAttribute failed";
     return e;
   }
-  e = launch_pdl_cluster(kern, dim3(static_cast<unsigned>(S), static_cast<unsigned>(tiles), 1), dim3(kSkThreads),
-                         static_cast<size_t>(kSkAlloc), st, static_cast<unsigned>(S), tmA, tmB, p);
+  e = launch_pdl_cluster(kern, dim3(2u, static_cast<unsigned>(tiles), 1), dim3(kSkThreads),
+                         static_cast<size_t>(kSkAlloc), st, 2u, tmA, tmB, p);
   if (e != cudaSuccess) *why = "cluster launch of the split-K GEMM failed";
   return e;
 }
@@ -617,21 +619,35 @@ cudaError_t launch_small_m(const SmallArgs& a, cudaStream_t st, const DeviceInfo
   return fused ? run_small<32, true>(a, st, dev, why) : run_small<32, false>(a, st, dev, why);
 }
 
+// Split K over a CTA pair when 128 x 256 tiles fill at most half the SMs and
+// K has at least four 128-byte k-blocks (bf16 epilogue only).
+static bool use_splitk(int64_t M, int64_t N, int64_t K, int sm_count) {
+  const int64_t tiles256 = ((M + kBM - 1) / kBM) * ((N + 255) / 256);
+  const int64_t nk = (K + kBK - 1) / kBK;
+  return SQ_GEMM_SPLITK && SQ_GEMM_BN == 0 && 2 * tiles256 <= sm_count && nk >= 4;
+}
+
+size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int sm_count) {
+  if (!use_splitk(M, N, K, sm_count)) return 0;
+  const int64_t tiles256 = ((M + kBM - 1) / kBM) * ((N + 255) / 256);
+  return static_cast<size_t>(tiles256) * 2 * kSkSlotBytes;
+}
+
 cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t st, const DeviceInfo& dev, const char** why) {
-  // 128 x 256 output tiles when there are at least as many as SMs.  With
-  // fewer, 128 x 128 tiles put about twice as many SMs to work: an M=128 int8
-  // MMA costs about the same for N=128 as for N=256, so each SM's main loop
-  // takes as long either way.  (Splitting K over a cluster instead, build knob
-  // SQ_GEMM_SPLITK, measured slower on B200: its reduction through distributed
-  // shared memory costs more than the main loop it shortens.)
-  const int64_t mb = (a.M + kBM - 1) / kBM;
-  const int64_t tiles256 = mb * ((a.N + 255) / 256);
-  const int64_t nk = (a.K + kBK - 1) / kBK;
-  int S = 1;
-  if (SQ_GEMM_SPLITK && SQ_GEMM_BN == 0 && tiles256 < dev.sm_count)
-    while (S < 8 && tiles256 * S * 2 <= dev.sm_count && nk >= 4 * S) S *= 2;
-  if (S > 1) return a.epi == Epilogue::kBf16Dequant ? run_splitk<0>(a, S, st, dev, why) : run_splitk<1>(a, S, st, dev, why);
-  const bool wide = SQ_GEMM_BN == 256 || (SQ_GEMM_BN == 0 && tiles256 >= dev.sm_count);
+  // An M=128 int8 MMA costs about the same for N=128 as for N=256, so the main
+  // loop of an SM takes as long for a 128 x 128 tile as for a 128 x 256 one.
+  // With t tiles of 128 x 256:
+  //   2t <= SMs: split each tile's K over a CTA pair (twice the SMs, half the
+  //              main loop each, plus one exchange of partial sums), given a
+  //              workspace for that exchange; without one, 128 x 128 tiles;
+  //   else:      128 x 256 tiles, persistent (128-wide tiles would give an SM
+  //              two tiles' worth of MMAs where a 256-wide one gives it one).
+  const int64_t tiles256 = ((a.M + kBM - 1) / kBM) * ((a.N + 255) / 256);
+  if (a.epi == Epilogue::kBf16Dequant && a.ws != nullptr) {
+    const size_t need = gemm_workspace_bytes(a.M, a.N, a.K, dev.sm_count);
+    if (need > 0 && a.ws_bytes >= need) return run_splitk(a, st, why);
+  }
+  const bool wide = SQ_GEMM_BN == 256 || (SQ_GEMM_BN == 0 && 2 * tiles256 > dev.sm_count);
   if (a.epi == Epilogue::kBf16Dequant) {
     return wide ? run_gemm<256, 4, 0, 1>(a, st, dev, why) : run_gemm<128, 6, 0, SQ_GEMM_CHAINS128>(a, st, dev, why);
   }

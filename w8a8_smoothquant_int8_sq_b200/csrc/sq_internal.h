@@ -106,8 +106,14 @@ struct GemmArgs {
   const uint16_t* bias;     // [N] or null
   void* out;                // Y bf16 [M][N] or acc int32 [M][N]
   Epilogue epi;
+  void* ws = nullptr;       // optional scratch (16-byte aligned) for the split-K exchange
+  size_t ws_bytes = 0;
 };
 cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t st, const DeviceInfo& dev, const char** why);
+
+// Scratch the GEMM can use for an M x N x K problem on a device with sm_count
+// SMs (0: none; the split-K path is taken only when at least this much is given).
+size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int sm_count);
 
 // Few tokens (M <= kSmallMaxM): weight-streaming kernel, split-K over a thread
 // block cluster.  With X != null the per-token quantisation of X / s is fused

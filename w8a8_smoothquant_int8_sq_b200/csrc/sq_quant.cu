@@ -29,8 +29,9 @@ constexpr unsigned long long kQuantWaitTimeoutNs = 2000000000ull;  // 2 s per wa
 #ifdef SQ_TRACE
 // Optional block timestamps (build with -DSQ_TRACE): per kernel kind (0 colmax,
 // 1 row quant of weights, 2 row quant of activations) and block, globaltimer at
-// 0 block start, 1 past the wait for the previous kernel, 2 block end.
-__device__ unsigned long long g_blk_trace[3][2048][3];
+// 0 block start, 1 past the wait for the previous kernel, 2 block end, 3 a
+// kernel-specific point (colmax: the block's maxima merged, before arrival).
+__device__ unsigned long long g_blk_trace[3][2048][4];
 struct BlockTrace {
   int kind, id;
   __device__ BlockTrace(int k) : kind(k), id(blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z)) {
@@ -47,7 +48,7 @@ extern "C" __attribute__((visibility("default"))) int sq_trace_read_blocks(unsig
   return cudaMemcpyFromSymbol(host, g_blk_trace, sizeof(g_blk_trace)) == cudaSuccess ? 0 : 1;
 }
 extern "C" __attribute__((visibility("default"))) int sq_trace_clear_blocks() {
-  static unsigned long long zero[3][2048][3];
+  static unsigned long long zero[3][2048][4];
   return cudaMemcpyToSymbol(g_blk_trace, zero, sizeof(zero)) == cudaSuccess ? 0 : 1;
 }
 #else
@@ -223,6 +224,7 @@ __global__ void __launch_bounds__(kColThreads) colmax_kernel(const __grid_consta
   }
 
   // arrival: the last block of this stripe computes s for the stripe
+  SQ_BLOCK_MARK(3);
   __threadfence();
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -374,6 +376,9 @@ cudaError_t launch_calibrate_noalloc(const uint16_t* C, int64_t R, int64_t K, co
 // s (and 1/s) sit in shared memory as four float4 arrays indexed by vector, so
 // the table reads of a warp are contiguous and free of bank conflicts.
 constexpr int kRowThreads = 256;
+#ifndef SQ_RQ_L2_AHEAD  // build-time tuning knob: 1 prefetches the row after next into L2
+#define SQ_RQ_L2_AHEAD 1
+#endif
 
 template <int VPL, int WPR>
 __device__ __forceinline__ void load_row_vectors(uint4 (&xv)[VPL], const uint16_t* __restrict__ src, int64_t row,
@@ -461,6 +466,15 @@ __global__ void __launch_bounds__(kRowThreads) row_quant_kernel(const uint16_t* 
     }
     const int64_t next = row + row_step;
     load_row_vectors<VPL, WPR>(xv, src, next, rows, K, nvec, wsub, lane);  // prefetch
+#if SQ_RQ_L2_AHEAD
+    {
+      // and the row after that into L2, so the register prefetch above finds
+      // its row in L2 instead of paying a DRAM latency per row
+      const int64_t ahead = next + row_step;
+      if (wsub == 0 && lane == 0 && ahead < rows)
+        bulk_prefetch_l2(src + ahead * static_cast<int64_t>(K), static_cast<uint32_t>(K) * 2u);
+    }
+#endif
     m = warp_max(m);
     if (WPR > 1) {
       if (lane == 0) red[it & 1][warp] = m;
