@@ -184,7 +184,9 @@ SQ_API sq_status sq_linear(const int8_t* Xq, const float* x_scale, const int8_t*
  *   workspace  at least sq_forward_workspace_bytes(M, N, K) bytes (holds the
  *              intermediate Xq and x_scale, then sq_linear's workspace);
  *              contents on entry are ignored.
- * The codes and scales are identical to those of sq_quantize_act.
+ * The codes and scales are identical to those of sq_quantize_act.  Up to 8
+ * tokens the quantisation runs inside the weight-streaming kernel; otherwise
+ * the row quantiser runs first and sq_linear's kernels follow.
  */
 SQ_API size_t sq_forward_workspace_bytes(int64_t M, int64_t N, int64_t K);
 SQ_API sq_status sq_forward(const sq_bf16* X, const float* s, const int8_t* Wq,

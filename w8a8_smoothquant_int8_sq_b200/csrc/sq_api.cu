@@ -300,7 +300,7 @@ sq_status sq_forward(const sq_bf16* X, const float* s, const int8_t* Wq, const f
   if (!aligned16(workspace)) return fail(SQ_ERR_ALIGN, "workspace is not 16-byte aligned");
   sq::DeviceInfo dev;
   SQ_TRY(prologue(&dev));
-  if (M <= sq::kSmallMaxM) {  // few tokens: quantisation fused into the weight-streaming kernel
+  if (M <= sq::kSmallFusedMaxM) {  // few tokens: quantisation fused into the weight-streaming kernel
     sq::SmallArgs a{X, s, nullptr, nullptr, Wq, w_scale, bias, M, N, K, Y};
     const char* why = "fused small-M kernel";
     cudaError_t e = sq::launch_small_m(a, static_cast<cudaStream_t>(stream), dev, &why);
@@ -313,6 +313,12 @@ sq_status sq_forward(const sq_bf16* X, const float* s, const int8_t* Wq, const f
   sq_status st = cuda_status(
       sq::launch_row_quant(false, X, M, K, s, Xq, xs, static_cast<cudaStream_t>(stream), dev), "quantize_act launch");
   if (st != SQ_OK) return st;
+  if (M <= sq::kSmallMaxM) {  // few tokens, quantised first: the weight-streaming kernel on the codes
+    sq::SmallArgs a{nullptr, nullptr, Xq, xs, Wq, w_scale, bias, M, N, K, Y};
+    const char* why = "small-M kernel";
+    cudaError_t e = sq::launch_small_m(a, static_cast<cudaStream_t>(stream), dev, &why);
+    if (e != cudaErrorNotSupported) return cuda_status(e, why);
+  }
   return gemm_common(Xq, xs, Wq, w_scale, bias, M, N, K, Y, sq::Epilogue::kBf16Dequant, stream, dev,
                      static_cast<char*>(workspace) + gemm_off, workspace_bytes - gemm_off);
 }

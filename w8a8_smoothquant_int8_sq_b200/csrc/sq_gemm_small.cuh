@@ -16,18 +16,24 @@
 //     about 4 KB of Wq per MMA; spreading the rows over ~128 CTAs keeps that
 //     above the HBM rate.
 //   * split-K over a thread-block cluster of S CTAs: each CTA streams its
-//     share of the row block's K; the S partial int32 accumulators are summed
-//     through distributed shared memory at the end, every rank reducing a
-//     share of the rows (exact, no global scratch).
+//     share of the row block's K; at the end every CTA pushes its partial
+//     int32 sums of each row (real tokens only) into the shared memory of the
+//     rank that reduces that row, and after one cluster barrier each rank adds
+//     the S partials of its rows from its own shared memory (exact, no global
+//     scratch, no remote load on the critical path).
 //   * prequantised codes (sq_linear): the codes travel by TMA in the same
 //     stage as the weight box (NT-row box, rows past M zero-filled), so the
 //     first MMA waits only for the first stage.
-//   * fused quantisation (sq_forward): eight warps quantise this CTA's K-slice
-//     of X / s (correctly rounded fp32 division, as sq_quantize_act).  The
-//     per-token maxima over the whole row are assembled from the S ranks'
-//     slice maxima through distributed shared memory at a mid-kernel cluster
-//     barrier; the codes then go straight into the shared-memory B operand in
-//     the 128-byte-swizzled K-major layout the tensor core reads.
+//   * fused quantisation (sq_forward, up to 8 tokens): eight warps quantise
+//     this CTA's K-slice of X / s (correctly rounded fp32 division, as
+//     sq_quantize_act), holding their X vectors in registers between the two
+//     passes.  The per-token maxima over the whole row are assembled from the
+//     S ranks' slice maxima through distributed shared memory at a mid-kernel
+//     cluster barrier; the codes then go straight into the shared-memory B
+//     operand in the 128-byte-swizzled K-major layout the tensor core reads.
+//     The MMAs cannot start before the codes exist, and past that point the
+//     kernel runs at the weight-stream rate, so the fused path is only about
+//     as fast as quantising first; beyond 8 tokens sq_forward quantises first.
 //
 // Warps: 0 TMA producer, 1 TMEM owner + MMA issuer, 2..9 quantisation and
 // reduction (2..5 also drain TMEM: lane quarters 2, 3, 0, 1).  Every mbarrier
@@ -35,6 +41,13 @@
 
 namespace sq {
 namespace {
+
+// Build-time knob: when the fused kernel's producer starts streaming the
+// weight (0 at once, 1 once the activation loads have returned, 2 once the row
+// scales are known, 3 once the codes are written).
+#ifndef SQ_SMALL_GATE
+#define SQ_SMALL_GATE 0
+#endif
 
 constexpr int kSmallThreads = 320;
 constexpr int kSmallQuantThreads = 256;  // warps 2..9
@@ -83,6 +96,11 @@ __device__ __forceinline__ uint4 ld_cluster_v4(uint32_t addr) {
                : "memory");
   return v;
 }
+__device__ __forceinline__ void st_cluster_v4(uint32_t addr, uint4 v) {
+  asm volatile("st.shared::cluster.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z),
+               "r"(v.w)
+               : "memory");
+}
 __device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
   float v;
   asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
@@ -103,8 +121,10 @@ __device__ __forceinline__ uint32_t b_code_offset(int m, int c) {
 #ifdef SQ_TRACE
 // Optional phase timestamps (build with -DSQ_TRACE): per CTA, globaltimer at
 // 0 start, 1 codes ready, 2 first stage consumed, 3 last MMA issued,
-// 4 accumulators read, 5 after the reduction barrier, 6 end.
-__device__ unsigned long long g_small_trace[1024][8];
+// 4 accumulators read, 5 after the reduction barrier, 6 end; fused: 7 pass-1
+// loads returned, 8 slice maxima reduced, 9 after the exchange barrier,
+// 10 scales formed, 11 codes written (warp 2, lane 0).
+__device__ unsigned long long g_small_trace[1024][12];
 #define SQ_TRACE_MARK(i)                                        \
   do {                                                          \
     const int cta_ = blockIdx.y * gridDim.x + blockIdx.x;       \
@@ -131,6 +151,84 @@ __device__ __forceinline__ void load_s8(const float4* s4, int v, f2x (&ns)[4], f
   rs[2] = f2_pack(__frcp_rn(b.x), __frcp_rn(b.y)), rs[3] = f2_pack(__frcp_rn(b.z), __frcp_rn(b.w));
 }
 
+// Warp max of 16 per-lane values rm[0..15] by reduce-scatter: 16 shuffles
+// instead of 16 x 5.  Afterwards lane l holds the max of value l >> 1.
+__device__ __forceinline__ float warp_max16_scatter(const float (&rm)[16], int lane) {
+  float a[8];
+  const bool hi4 = lane & 16;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const float give = hi4 ? rm[j] : rm[8 + j];
+    const float keep = hi4 ? rm[8 + j] : rm[j];
+    a[j] = fmaxf(keep, __shfl_xor_sync(0xFFFFFFFFu, give, 16));
+  }
+  float b[4];
+  const bool hi3 = lane & 8;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float give = hi3 ? a[j] : a[4 + j];
+    const float keep = hi3 ? a[4 + j] : a[j];
+    b[j] = fmaxf(keep, __shfl_xor_sync(0xFFFFFFFFu, give, 8));
+  }
+  float c[2];
+  const bool hi2 = lane & 4;
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    const float give = hi2 ? b[j] : b[2 + j];
+    const float keep = hi2 ? b[2 + j] : b[j];
+    c[j] = fmaxf(keep, __shfl_xor_sync(0xFFFFFFFFu, give, 4));
+  }
+  const bool hi1 = lane & 2;
+  float d = fmaxf(hi1 ? c[1] : c[0], __shfl_xor_sync(0xFFFFFFFFu, hi1 ? c[0] : c[1], 2));
+  return fmaxf(d, __shfl_xor_sync(0xFFFFFFFFu, d, 1));
+}
+
+// Fused quantisation, pass 1, for one 16-byte vector v of the K-slice and the
+// first R token rows held in registers: loads (s, then the R rows of X, all
+// issued before any arithmetic), -s and RN(1/s), and the rows' max |fl(x/s)|.
+template <int R>
+__device__ __forceinline__ void fused_pass1(const uint4* X4, const float4* s4, int nvec, int v, bool has, int M,
+                                            uint4 (&xr)[16], f2x (&ns)[4], f2x (&rs)[4], float (&rmax)[16]) {
+  float4 sa = make_float4(1.f, 1.f, 1.f, 1.f), sb = sa;
+  if (has) {
+    sa = __ldg(s4 + 2 * v);
+    sb = __ldg(s4 + 2 * v + 1);
+  }
+#pragma unroll
+  for (int r = 0; r < R; ++r)
+    xr[r] = (has && r < M) ? __ldg(X4 + static_cast<int64_t>(r) * nvec + v) : make_uint4(0u, 0u, 0u, 0u);
+  ns[0] = f2_pack(-sa.x, -sa.y), ns[1] = f2_pack(-sa.z, -sa.w), ns[2] = f2_pack(-sb.x, -sb.y), ns[3] = f2_pack(-sb.z, -sb.w);
+  rs[0] = f2_pack(__frcp_rn(sa.x), __frcp_rn(sa.y)), rs[1] = f2_pack(__frcp_rn(sa.z), __frcp_rn(sa.w));
+  rs[2] = f2_pack(__frcp_rn(sb.x), __frcp_rn(sb.y)), rs[3] = f2_pack(__frcp_rn(sb.z), __frcp_rn(sb.w));
+  // every one of the R rows, real or padding (zeros), with no branch, so the
+  // rows' dependency chains interleave
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    f2x t[4];
+    smooth8(xr[r], ns, rs, t);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) rmax[r] = f2_absmax(rmax[r], t[e]);
+  }
+}
+
+// Fused quantisation, pass 2: the codes of the first R rows of vector v into
+// the swizzled B operand (padding rows get code 0; their accumulator columns
+// are never read).
+template <int NT, int R>
+__device__ __forceinline__ void fused_pass2(const uint4 (&xr)[16], const f2x (&ns)[4], const f2x (&rs)[4],
+                                            const float* xs_s, const float* rxs_s, uint8_t* bsm, int c) {
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const float sc = xs_s[r], rsc = rxs_s[r];
+    const f2x nsc2 = f2_pack(-sc, -sc), rsc2 = f2_pack(rsc, rsc);
+    f2x t[4];
+    smooth8(xr[r], ns, rs, t);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) t[e] = f2_round_codes(f2_div_rn(t[e], nsc2, rsc2));
+    *reinterpret_cast<uint2*>(bsm + b_code_offset<NT>(r, c)) = pack8_codes(t[0], t[1], t[2], t[3]);
+  }
+}
+
 template <int NT, bool kFused>
 __global__ void __launch_bounds__(kSmallThreads, 1)
     gemm_small_m_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
@@ -142,6 +240,7 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
   float* xs_s = reinterpret_cast<float*>(smem + p.xs_off);
   float* red = reinterpret_cast<float*>(smem + p.red_off);  // [8 warps][NT], then the slice maxima [NT]
   float* cmax = red + 8 * NT;
+  float* rxs_s = red + 9 * NT;  // fused: RN(1 / x_scale) per token
   float* wsb = reinterpret_cast<float*>(smem + p.wsb_off);  // w_scale[256], bias[256] of this row block
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + p.bar_off);
   uint64_t* full = bars;
@@ -149,6 +248,7 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
   uint64_t* b_ready = bars + 2 * kSmallMaxStages;
   uint64_t* acc_full = b_ready + 1;
   uint64_t* drain = b_ready + 2;
+  uint64_t* x_in = b_ready + 3;  // fused: every quantisation warp holds its slice of X
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + p.misc_off);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + p.misc_off + 4);
 
@@ -174,6 +274,7 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
     mbar_init(b_ready, 1);
     mbar_init(acc_full, 1);
     mbar_init(drain, 1);
+    mbar_init(x_in, kSmallQuantThreads / 32);
     *abort_flag = 0;
     fence_mbar_init();
     fence_proxy_async_smem();
@@ -205,7 +306,15 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
       uint32_t phase = 0;
       int issued = 0;
       bool ok = true;
-      for (int kb = kb0; kb < kb1; ++kb) {
+      // fused: start the weight stream only once the activation loads have
+      // returned; issued behind a full ring of weight boxes they would wait for
+      // the whole ring to drain from HBM, and the MMAs wait for their codes
+      if (kFused && SQ_SMALL_GATE > 0 &&
+          (*abort_flag || !mbar_wait_bounded(SQ_SMALL_GATE == 3 ? b_ready : x_in, 0, kWaitTimeoutNs))) {
+        if (!*abort_flag) flag_timeout(abort_flag);
+        ok = false;
+      }
+      for (int kb = kb0; ok && kb < kb1; ++kb) {
         if (*abort_flag || !mbar_wait_bounded(&empty[stage], phase ^ 1u, kWaitTimeoutNs)) {
           if (!*abort_flag) flag_timeout(abort_flag);
           ok = false;
@@ -282,12 +391,36 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
       const int v_hi = min(nvec, kb1 * (kBK / 8));
       const uint4* X4 = reinterpret_cast<const uint4*>(p.X);
       const float4* s4 = reinterpret_cast<const float4*>(p.s);
-      // pass 1: max of |fl(X / s)| over this CTA's K-slice, eight rows at a time
-      // with all of a group's loads issued before any arithmetic
+      // With at most one 16-byte vector of the K-slice per thread and at most
+      // 16 tokens, each thread keeps its X vectors in registers from pass 1 to
+      // pass 2: all of its global loads are issued at once, before any
+      // arithmetic, and nothing is read twice.
+      constexpr int kRegRows = 16;
+      const bool in_regs = NT == kRegRows && v_hi - v_lo <= kSmallQuantThreads;
+      uint4 xr[kRegRows];
+      f2x rns[4], rrs[4];
       float rmax[NT];
 #pragma unroll
       for (int m = 0; m < NT; ++m) rmax[m] = 0.0f;
-      for (int v = v_lo + qt; v < v_hi; v += kSmallQuantThreads) {
+      if (in_regs) {
+        float rm16[16];
+#pragma unroll
+        for (int m = 0; m < 16; ++m) rm16[m] = 0.0f;
+        const int v = v_lo + qt;
+        const bool has = v < v_hi;
+        if (M <= 8)
+          fused_pass1<8>(X4, s4, nvec, v, has, M, xr, rns, rrs, rm16);
+        else
+          fused_pass1<16>(X4, s4, nvec, v, has, M, xr, rns, rrs, rm16);
+        __syncwarp();
+        if (SQ_SMALL_GATE == 1 && lane == 0) mbar_arrive(x_in);  // this warp's pass-1 loads have all returned
+        if (warp == 2 && lane == 0) SQ_TRACE_MARK(7);
+        const float wm = warp_max16_scatter(rm16, lane);
+        if ((lane & 1) == 0) red[qw * NT + (lane >> 1)] = wm;
+      }
+      // pass 1: max of |fl(X / s)| over this CTA's K-slice, eight rows at a time
+      // with all of a group's loads issued before any arithmetic
+      for (int v = v_lo + qt; !in_regs && v < v_hi; v += kSmallQuantThreads) {
         f2x ns[4], rs[4];
         load_s8(s4, v, ns, rs);
 #pragma unroll
@@ -307,10 +440,14 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
           }
         }
       }
+      if (!in_regs) {
+        __syncwarp();
+        if (SQ_SMALL_GATE == 1 && lane == 0) mbar_arrive(x_in);  // this warp's pass-1 loads have all returned
 #pragma unroll
-      for (int m = 0; m < NT; ++m) {
-        const float r = warp_max(rmax[m]);
-        if (lane == 0) red[qw * NT + m] = r;
+        for (int m = 0; m < NT; ++m) {
+          const float r = warp_max(rmax[m]);
+          if (lane == 0) red[qw * NT + m] = r;
+        }
       }
       named_bar_sync(1, kSmallQuantThreads);
       if (qt < NT) {
@@ -319,17 +456,37 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
         for (int w = 0; w < kSmallQuantThreads / 32; ++w) mx = fmaxf(mx, red[w * NT + qt]);
         cmax[qt] = mx;
       }
+      if (warp == 2 && lane == 0) SQ_TRACE_MARK(8);
       // exchange of the slice maxima across the cluster (warps 0, 1 arrived early)
       asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+      if (warp == 2 && lane == 0) SQ_TRACE_MARK(9);
       if (qt < NT) {
+        // all S remote loads are issued before the first use of any of them
         const uint32_t a = smem_u32(cmax + qt);
+        float part_max[8];
+#pragma unroll
+        for (int r = 0; r < 8; ++r)
+          if (r < S) part_max[r] = ld_cluster_f32(map_cluster_rank(a, static_cast<uint32_t>(r)));
         float mx = 0.0f;
-        for (int r = 0; r < S; ++r) mx = fmaxf(mx, ld_cluster_f32(map_cluster_rank(a, static_cast<uint32_t>(r))));
-        xs_s[qt] = __fdiv_rn(fmaxf(mx, kClampFloor), kQmax);
+#pragma unroll
+        for (int r = 0; r < 8; ++r)
+          if (r < S) mx = fmaxf(mx, part_max[r]);
+        const float sc = __fdiv_rn(fmaxf(mx, kClampFloor), kQmax);
+        xs_s[qt] = sc;
+        rxs_s[qt] = __frcp_rn(sc);
       }
       named_bar_sync(1, kSmallQuantThreads);
+      if (SQ_SMALL_GATE == 2 && lane == 0) mbar_arrive(x_in);  // the row scales are known
+      if (warp == 2 && lane == 0) SQ_TRACE_MARK(10);
       // pass 2: the codes of this CTA's K-slice, into the swizzled B operand
-      for (int v = v_lo + qt; v < v_hi; v += kSmallQuantThreads) {
+      if (in_regs && v_lo + qt < v_hi) {
+        const int c = (v_lo + qt) * 8 - kb0 * kBK;
+        if (M <= 8)
+          fused_pass2<NT, 8>(xr, rns, rrs, xs_s, rxs_s, bsm, c);
+        else
+          fused_pass2<NT, 16>(xr, rns, rrs, xs_s, rxs_s, bsm, c);
+      }
+      for (int v = v_lo + qt; !in_regs && v < v_hi; v += kSmallQuantThreads) {
         f2x ns[4], rs[4];
         load_s8(s4, v, ns, rs);
         const int c = v * 8 - kb0 * kBK;
@@ -344,7 +501,7 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
             for (int r = 0; r < 8; ++r) {
               if (g + r < M) {
                 const float sc = xs_s[g + r];
-                const float rsc = __frcp_rn(sc);
+                const float rsc = rxs_s[g + r];
                 const f2x nsc2 = f2_pack(-sc, -sc), rsc2 = f2_pack(rsc, rsc);
                 f2x t[4];
                 smooth8(w[r], ns, rs, t);
@@ -356,6 +513,7 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
           }
         }
       }
+      if (warp == 2 && lane == 0) SQ_TRACE_MARK(11);
       // make the generic-proxy smem writes visible to the tensor core, then release the MMA warp
       fence_proxy_async_smem();
       named_bar_sync(1, kSmallQuantThreads);
@@ -400,36 +558,46 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
             for (int i = 0; i < 32; ++i) acc[(c + i) % NT] += r32[i];
           }
         }
-        uint4* dst = reinterpret_cast<uint4*>(part + n_local * NT);
+        // push the row's partial sums to the rank that reduces this row, into
+        // that rank's slot for this sender (fire-and-forget stores; the
+        // cluster barrier below waits for them)
+        const int rpr = kSmallRows / S;
+        const int owner = n_local / rpr;
+        const uint32_t dst = map_cluster_rank(
+            smem_u32(part + (static_cast<int>(rank) * rpr + (n_local - owner * rpr)) * NT), static_cast<uint32_t>(owner));
+        const int nq = (p.M + 3) / 4;  // token quads that hold real tokens
 #pragma unroll
         for (int i = 0; i < NT / 4; ++i)
-          dst[i] = make_uint4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]);
+          if (i < nq) st_cluster_v4(dst + 16u * i, make_uint4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]));
       }
     }
   }
 
   // ------------------------------------------- split-K reduction over the cluster
-  // Every rank reduces its share of the 256 rows: for each (row, 4 tokens) it
-  // reads the S partial sums (one per rank, through distributed shared memory),
-  // adds them, dequantises and stores.  The S loads are issued before any add.
+  // Rank q reduces rows [q*256/S, (q+1)*256/S): every rank has pushed its
+  // partial sums of those rows into rank q's shared memory (one slot per
+  // sender), so after the cluster barrier the S partials of a row are local
+  // loads; the sum is dequantised and stored.  Token quads past M are skipped.
+  // No CTA reads another's shared memory after the barrier, so none has to
+  // wait for the others before leaving.
   tc_fence_before();
   __syncthreads();
   if (kFused && warp < 2) cluster_wait();  // completes the phase these warps arrived at early
-  cluster_sync_all();  // every CTA's partial accumulators are in its shared memory
+  cluster_sync_all();  // every rank's pushes have landed
   if (threadIdx.x == 0) SQ_TRACE_MARK(5);
   if (warp >= 2) {
-    const int rows_per_rank = (kSmallRows + S - 1) / S;
-    const int r_lo = static_cast<int>(rank) * rows_per_rank;
-    const int r_hi = min(kSmallRows, r_lo + rows_per_rank);
-    const int items = (r_hi - r_lo) * (NT / 4);
+    const int rpr = kSmallRows / S;
+    const int r_lo = static_cast<int>(rank) * rpr;
+    const int items = rpr * ((p.M + 3) / 4);
     for (int it = threadIdx.x - 64; it < items; it += kSmallQuantThreads) {
-      const int n_local = r_lo + it / (NT / 4);
-      const int q4 = it % (NT / 4);
-      const uint32_t addr = smem_u32(part + n_local * NT + q4 * 4);
+      // consecutive threads take consecutive rows (outputs n) of one token
+      // quad, so a warp's Y stores for a token cover one contiguous run
+      const int lr = it % rpr;
+      const int q4 = it / rpr;
       uint4 v[8];
 #pragma unroll
       for (int r = 0; r < 8; ++r)
-        if (r < S) v[r] = ld_cluster_v4(map_cluster_rank(addr, static_cast<uint32_t>(r)));
+        if (r < S) v[r] = *reinterpret_cast<const uint4*>(part + (r * rpr + lr) * NT + q4 * 4);
       int32_t acc[4] = {0, 0, 0, 0};
 #pragma unroll
       for (int r = 0; r < 8; ++r)
@@ -437,6 +605,7 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
           acc[0] += static_cast<int32_t>(v[r].x), acc[1] += static_cast<int32_t>(v[r].y);
           acc[2] += static_cast<int32_t>(v[r].z), acc[3] += static_cast<int32_t>(v[r].w);
         }
+      const int n_local = r_lo + lr;
       const int n = rb * kSmallRows + n_local;
       if (n < p.N) {
         const float ws = wsb[n_local];
@@ -452,7 +621,8 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
       }
     }
   }
-  cluster_sync_all();  // no CTA leaves while another may still read its shared memory
+  tc_fence_before();
+  __syncthreads();
   if (threadIdx.x == 0) SQ_TRACE_MARK(6);
   if (warp == 1) {
     tc_fence_after();

@@ -121,6 +121,12 @@ size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int sm_count);
 // come from the caller.  Returns cudaErrorNotSupported when the shape does not
 // fit the kernel (the caller then uses the general path).
 constexpr int64_t kSmallMaxM = 32;
+// sq_forward fuses the activation quantisation into that kernel up to this
+// many tokens; above it (to kSmallMaxM) the row quantiser runs first.
+#ifndef SQ_SMALL_FUSED_MAX  // build-time knob
+#define SQ_SMALL_FUSED_MAX 8
+#endif
+constexpr int64_t kSmallFusedMaxM = SQ_SMALL_FUSED_MAX;
 struct SmallArgs {
   const uint16_t* X;      // fused: bf16 [M][K]
   const float* s;         // fused: [K]
