@@ -86,7 +86,9 @@ SQ_API const char* sq_status_string(sq_status st);
  *              in float64 and the quotient is rounded once to fp32.
  *   mx_inout   NULL, or [K] fp32 running max-abs of activations: read, merged
  *              with this batch's column max, written back (start from zeros).
- *              With R == 0 it must be non-NULL and s comes from it alone.
+ *              With R == 0 it must be non-NULL and s comes from it alone:
+ *              that call followed by sq_prepare_weight is the page's
+ *              recompute_smooth_scale (new alpha after freezing).
  *   workspace  device scratch of at least sq_calibrate_workspace_bytes(K)
  *              bytes, 16-byte aligned; contents on entry are ignored.
  * Launches: one memset of the workspace and one kernel (column max-abs over

@@ -149,6 +149,33 @@ def test_running_max_two_batches(sq):
     assert torch.equal(s3, s_one)
 
 
+def test_recompute_after_alpha_change(sq):
+    """SmoothQuantW8A8.recompute_smooth_scale: after freezing, a new alpha
+    gives a new s from the stored running activation max and the weight's
+    column max alone (no calibration rows: R == 0), and W is folded and
+    quantised again with it -- the calibration and weight-prep kernels reused."""
+    wl = workloads.get("proj")
+    inp = workloads.make_inputs(wl, ("C", "W"))
+    C, W = inp["C"], inp["W"]
+    Cd, Wd = dev_bf16(C), dev_bf16(W)
+    mx = torch.zeros(wl.K, dtype=torch.float32, device="cuda")
+    sq.sq_calibrate(Cd[:200], Wd, 0.5, mx_inout=mx)   # two calibration batches,
+    sq.sq_calibrate(Cd[200:], Wd, 0.5, mx_inout=mx)   # then frozen at alpha 0.5
+    for alpha in (np.float32(0.35).item(), np.float32(0.8).item()):
+        s_g = sq.sq_calibrate(None, Wd, alpha, mx_inout=mx)
+        Wq_g, ws_g = sq.sq_prepare_weight(Wd, s_g)
+        torch.cuda.synchronize()
+        s_o, mx_o = O.calibrate(C[:0], W, alpha, mx_prev=host(mx))
+        assert np.array_equal(host(mx), mx_o)
+        assert_scales_close(host(s_g), s_o, f"recomputed s at alpha {alpha}")
+        Wq_o, ws_o = O.fold_and_quantize_weight(W, host(s_g))
+        _, _, vw = O.fold_and_quantize_weight_f64(W, host(s_g))
+        assert_scales_close(host(ws_g), ws_o, f"re-quantised w_scale at alpha {alpha}")
+        assert_codes(host(Wq_g), Wq_o, vw, f"re-quantised Wq at alpha {alpha}")
+        # the same s as calibrating on all rows at once with the new alpha
+        assert torch.equal(s_g, sq.sq_calibrate(Cd, Wd, alpha))
+
+
 def test_calibrate_leaves_workspace_zero(sq):
     """Whatever the workspace holds on entry, a call ends with the words it
     reduced into -- mx[K], mw[K] and one counter per 256 columns -- zeroed (the
