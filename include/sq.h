@@ -91,10 +91,10 @@ SQ_API const char* sq_status_string(sq_status st);
  *              recompute_smooth_scale (new alpha after freezing).
  *   workspace  device scratch of at least sq_calibrate_workspace_bytes(K)
  *              bytes, 16-byte aligned; contents on entry are ignored.
- * Launches: one memset of the workspace and one kernel (column max-abs over
- * C and W, streamed through shared memory by TMA; the last block to finish
- * each 256-column stripe computes s there and zeroes the stripe's workspace
- * words again).
+ * Launches: a small kernel that clears the workspace, then one kernel
+ * (column max-abs over C and W, streamed through shared memory by TMA; the
+ * last block to finish each 256-column stripe computes s there and zeroes
+ * the stripe's workspace words again).
  */
 SQ_API size_t sq_calibrate_workspace_bytes(int64_t K);
 SQ_API sq_status sq_calibrate(const sq_bf16* C, int64_t R, int64_t K,

@@ -593,6 +593,10 @@ cudaError_t run_splitk(const GemmArgs& a, cudaStream_t st, const char** why) {
   p.out = static_cast<uint16_t*>(a.out);
   p.part = static_cast<uint4*>(a.ws);
   p.vec_ok = ((a.N * 2) % 16 == 0) && (reinterpret_cast<uintptr_t>(a.out) % 16 == 0);
+  // Y by TMA stores of 32 x 32 boxes (64-byte rows, 64-byte swizzle) when its
+  // row pitch allows a tensor map; otherwise per-thread stores
+  CUtensorMap tmY = tmA;  // unused unless tma_store
+  p.tma_store = p.vec_ok && make_tmap_2d(&tmY, a.out, a.M, a.N, 2, kSkChunkCols, 32, 64) ? 1 : 0;
   p.skip_first_load = g_debug_stall.load() ? 1 : 0;
   p.timeout_ns = g_debug_stall.load() ? g_debug_timeout_ns.load() : kWaitTimeoutNs;
   const int tiles = p.num_m_blocks * static_cast<int>((a.N + kSkBN - 1) / kSkBN);
@@ -605,7 +609,7 @@ cudaError_t run_splitk(const GemmArgs& a, cudaStream_t st, const char** why) {
     return e;
   }
   e = launch_pdl_cluster(kern, dim3(2u, static_cast<unsigned>(tiles), 1), dim3(kSkThreads),
-                         static_cast<size_t>(kSkAlloc), st, 2u, tmA, tmB, p);
+                         static_cast<size_t>(kSkAlloc), st, 2u, tmA, tmB, tmY, p);
   if (e != cudaSuccess) *why = "cluster launch of the split-K GEMM failed";
   return e;
 }
@@ -699,7 +703,7 @@ cudaError_t read_device_status(uint32_t* flags, bool clear) {
 }
 
 bool make_tmap_2d(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int elem_bytes, int box_cols,
-                  int box_rows) {
+                  int box_rows, int swizzle_bytes) {
   EncodeTiledFn enc = get_encode_fn();
   if (enc == nullptr) return false;
   CUtensorMapDataType dt;
@@ -713,8 +717,16 @@ bool make_tmap_2d(CUtensorMap* map, const void* base, int64_t rows, int64_t cols
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * static_cast<cuuint64_t>(elem_bytes)};
   cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows)};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                   CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUtensorMapSwizzle sw;
+  switch (swizzle_bytes) {
+    case 0: sw = CU_TENSOR_MAP_SWIZZLE_NONE; break;
+    case 32: sw = CU_TENSOR_MAP_SWIZZLE_32B; break;
+    case 64: sw = CU_TENSOR_MAP_SWIZZLE_64B; break;
+    case 128: sw = CU_TENSOR_MAP_SWIZZLE_128B; break;
+    default: return false;
+  }
+  CUresult r = enc(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 

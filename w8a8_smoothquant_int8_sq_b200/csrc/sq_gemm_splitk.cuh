@@ -40,6 +40,10 @@ constexpr int kSkRingBytes = kSkStages * kSkStageBytes;
 constexpr int kSkChunkCols = 32;                          // columns per tcgen05.ld
 constexpr int kSkChunks = kSkHalf / kSkChunkCols;         // 4
 constexpr size_t kSkSlotBytes = static_cast<size_t>(kBM) * kSkHalf * 4;  // 64 KB per (tile, sender)
+// ring reuse after the main loop: [0, 64 KB) the peer's partial, then the
+// output boxes (4 warps x 4 chunks x 32 rows x 64 bytes = 32 KB)
+constexpr int kSkYOffset = static_cast<int>(kSkSlotBytes);
+static_assert(kSkYOffset + 4 * 4 * 32 * 64 <= kSkRingBytes, "the output boxes reuse the ring");
 // shared memory after the ring: w_scale[128], bias[128], x_scale[128] of the owned half, barriers, misc
 constexpr int kSkWsOffset = kSkRingBytes;
 constexpr int kSkBiasOffset = kSkWsOffset + kSkHalf * 4;
@@ -59,6 +63,7 @@ struct SkParams {
   uint16_t* out;  // bf16 Y [M][N]
   uint4* part;    // workspace: 2 slots of kSkSlotBytes per tile
   int vec_ok;
+  int tma_store;        // Y written by TMA stores (tmY valid)
   int skip_first_load;  // test hook: never load the first stage
   unsigned long long timeout_ns;
 };
@@ -85,7 +90,7 @@ __device__ unsigned long long g_sk_trace[1024][8];
 
 __global__ void __launch_bounds__(kSkThreads, 1)
     gemm_i8_splitk_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                          const SkParams p) {
+                          const __grid_constant__ CUtensorMap tmY, const SkParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   float* ws_s = reinterpret_cast<float*>(smem + kSkWsOffset);
@@ -284,7 +289,7 @@ __global__ void __launch_bounds__(kSkThreads, 1)
       for (int u = 0; u < 8; ++u) v[4 * u] += q[u].x, v[4 * u + 1] += q[u].y, v[4 * u + 2] += q[u].z, v[4 * u + 3] += q[u].w;
       const int cc = c * kSkChunkCols;  // column within the owned half
       const int n0 = n_blk * kSkBN + static_cast<int>(rank) * kSkHalf + cc;
-      if (!row_ok || n0 >= p.N) continue;
+      if (n0 >= p.N) continue;  // warp-uniform
       uint32_t packed[16];
 #pragma unroll
       for (int j = 0; j < 32; j += 2) {
@@ -293,6 +298,25 @@ __global__ void __launch_bounds__(kSkThreads, 1)
                                    b_s[cc + j + 1]);
         packed[j / 2] = pack_bf16x2(y0, y1);
       }
+      if (p.tma_store) {
+        // this warp's 32 rows x 32 columns into its own 2 KB box (row = lane,
+        // 64 bytes; 16-byte unit u of row r at u ^ ((r >> 1) & 3), the 64-byte
+        // swizzle, so the 32 lanes' writes spread over all banks), then one
+        // TMA store; rows past M and columns past N are not written
+        uint8_t* box = smem + kSkYOffset + ((quarter * kSkChunks + c) * 32) * (kSkChunkCols * 2);
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          *reinterpret_cast<uint4*>(box + lane * 64 + ((u ^ ((lane >> 1) & 3)) << 4)) =
+              make_uint4(packed[4 * u], packed[4 * u + 1], packed[4 * u + 2], packed[4 * u + 3]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&tmY, n0, m_blk * kBM + quarter * 32, box);
+          bulk_commit_group();
+        }
+        continue;
+      }
+      if (!row_ok) continue;
       uint16_t* yrow = p.out + static_cast<int64_t>(m) * p.N + n0;
       if (n0 + kSkChunkCols <= p.N && p.vec_ok) {
         uint4* dst = reinterpret_cast<uint4*>(yrow);
@@ -305,6 +329,7 @@ __global__ void __launch_bounds__(kSkThreads, 1)
           if (n0 + j < p.N) yrow[j] = static_cast<uint16_t>(packed[j / 2] >> ((j & 1) * 16));
       }
     }
+    if (p.tma_store && lane == 0) bulk_wait_group_read0();  // the boxes are read before the block exits
     if (warp == 2 && lane == 0) SQ_SK_MARK(6);
   }
   tc_fence_before();

@@ -61,11 +61,12 @@ struct DeviceInfo {
 cudaError_t current_device_info(DeviceInfo* out);
 
 // 2-D tensor map over a row-major [rows][cols] matrix of elem_bytes-wide
-// elements (row pitch cols * elem_bytes), box box_cols x box_rows, no swizzle,
-// zero fill outside the matrix.  False when the driver's encoder is
-// unavailable or rejects the arguments.
+// elements (row pitch cols * elem_bytes), box box_cols x box_rows, zero fill
+// outside the matrix; swizzle_bytes 0 (none), 32, 64 or 128 (the shared-memory
+// box's 16-byte units permuted as the hardware swizzle mode of that span).
+// False when the driver's encoder is unavailable or rejects the arguments.
 bool make_tmap_2d(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int elem_bytes, int box_cols,
-                  int box_rows);
+                  int box_rows, int swizzle_bytes = 0);
 
 // Status word of the HBM-bound kernels (bit 0: a wait timed out).  Clearing a
 // set word also re-zeroes the no-allocation calibration scratch.

@@ -82,7 +82,7 @@ extern "C" __attribute__((visibility("default"))) int sq_trace_clear_blocks() {
 // Workspace layout: mx[K], mw[K] (fp32 bit patterns), count[stripes].  It must
 // be zero when the kernel starts, and the last block of each stripe zeroes the
 // stripe's words again once it has read them, so a call leaves the workspace
-// zero (a caller workspace is cleared by a memset first, the library's own
+// zero (a caller workspace is cleared by a small kernel first, the library's own
 // scratch is not).
 constexpr int kColConsumers = 8;                                 // consumer warps
 constexpr int kColThreads = 32 * (kColConsumers + 1);            // + one producer warp
@@ -247,6 +247,20 @@ __global__ void __launch_bounds__(kColThreads) colmax_kernel(const __grid_consta
   p.s[c] = smoothing_factor(mx, mw, p.alpha);
 }
 
+#ifndef SQ_CALIB_MEMSET  // build-time knob: 1 clears the workspace with cudaMemsetAsync
+#define SQ_CALIB_MEMSET 0
+#endif
+
+// Clears n words.  Nothing the previous kernel in the stream writes is touched
+// before its results are visible (griddepcontrol.wait first).
+__global__ void __launch_bounds__(256) zero_words_kernel(uint32_t* __restrict__ w, size_t n) {
+  griddep_wait();
+  griddep_launch_dependents();
+  for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x)
+    w[i] = 0u;
+}
+
 static int col_stripes(int64_t K) { return static_cast<int>((K + kColStripe - 1) / kColStripe); }
 
 size_t calibrate_workspace_words(int64_t K) { return static_cast<size_t>(2 * K + col_stripes(K)); }
@@ -262,7 +276,15 @@ cudaError_t launch_calibrate(const uint16_t* C, int64_t R, int64_t K, const uint
                              const DeviceInfo& dev) {
   cudaError_t e = cudaSuccess;
   if (!ws_is_zero) {
+#if SQ_CALIB_MEMSET
     e = cudaMemsetAsync(ws, 0, calibrate_workspace_words(K) * sizeof(uint32_t), st);
+#else
+    // a small kernel rather than a memset node, so that it chains with its
+    // neighbours through programmatic dependent launch
+    const size_t words = calibrate_workspace_words(K);
+    const unsigned blocks = static_cast<unsigned>(std::min<size_t>((words + 1023) / 1024, 4 * dev.sm_count));
+    e = launch_pdl(zero_words_kernel, dim3(blocks), dim3(256), 0, st, static_cast<uint32_t*>(ws), words);
+#endif
     if (e != cudaSuccess) return e;
   }
   static int per_sm = 0;  // idempotent set-up; a race only repeats it
@@ -379,6 +401,9 @@ constexpr int kRowThreads = 256;
 #ifndef SQ_RQ_L2_AHEAD  // build-time tuning knob: 1 prefetches the row after next into L2
 #define SQ_RQ_L2_AHEAD 1
 #endif
+#ifndef SQ_RQ_EARLY_L2  // build-time tuning knob: rows per row group prefetched into L2 before the wait
+#define SQ_RQ_EARLY_L2 4
+#endif
 
 template <int VPL, int WPR>
 __device__ __forceinline__ void load_row_vectors(uint4 (&xv)[VPL], const uint16_t* __restrict__ src, int64_t row,
@@ -414,6 +439,18 @@ __global__ void __launch_bounds__(kRowThreads) row_quant_kernel(const uint16_t* 
   const int64_t row_step = static_cast<int64_t>(gridDim.x) * RPC;
 
   SQ_BLOCK_TRACE(kMul ? 1 : 2);
+#if SQ_RQ_EARLY_L2
+  // While the previous kernel is still running, pull this block's first rows
+  // into L2.  A prefetch is only a hint and L2 is where every SM's writes
+  // land, so even rows the previous kernel is still writing are read
+  // correctly after the wait below.
+  if (wsub == 0 && lane == 0) {
+    for (int i = 0; i < SQ_RQ_EARLY_L2; ++i) {
+      const int64_t r = row + i * row_step;
+      if (r < rows) bulk_prefetch_l2(src + r * static_cast<int64_t>(K), static_cast<uint32_t>(K) * 2u);
+    }
+  }
+#endif
   griddep_wait();
   SQ_BLOCK_MARK(1);
   griddep_launch_dependents();
@@ -434,6 +471,7 @@ __global__ void __launch_bounds__(kRowThreads) row_quant_kernel(const uint16_t* 
     }
   }
   __syncthreads();
+  SQ_BLOCK_MARK(3);
   const f2x* sA2 = reinterpret_cast<const f2x*>(sA);
   const f2x* sB2 = reinterpret_cast<const f2x*>(sB);
   const f2x* rA2 = reinterpret_cast<const f2x*>(rA);
