@@ -1,0 +1,50 @@
+"""bench.py's roofline report on CPU, from made-up call times: every workload
+gets a bound per call from the two rooflines (decode's GEMM is HBM-bound, the
+larger GEMMs tensor-bound), fractions are achieved / peak, the longest call is
+the one reported, and long kernels are held to the sustained tensor peak."""
+import bench
+import workloads
+
+NAMES = ["sq_calibrate", "sq_prepare_weight", "sq_quantize_act", "sq_linear"]
+LAUNCHES = {"sq_calibrate": 2, "sq_prepare_weight": 1, "sq_quantize_act": 1, "sq_linear": 1}
+
+
+def _report(name, ms):
+    wl = workloads.get(name)
+    per_call = dict(zip(NAMES, ms))
+    return wl, bench.kernel_report(wl, NAMES, per_call, per_call, LAUNCHES)
+
+
+def test_bounds_follow_the_rooflines():
+    for name in ("tiny", "proj", "mlp", "prefill", "decode"):
+        wl, (kernels, roof) = _report(name, [0.01, 0.012, 0.006, 0.02])
+        for n in NAMES[:3]:
+            assert kernels[n]["bound"] == "hbm"
+        want = "hbm" if name in ("tiny", "decode") else "tensor"
+        assert kernels["sq_linear"]["bound"] == want, name
+        assert roof["kernel"] == "sq_linear"
+        assert roof["bound"] == want
+
+
+def test_fractions_are_achieved_over_peak():
+    hbm, bf16, bf16_sus, _ = bench.peaks()
+    wl, (kernels, roof) = _report("proj", [0.010, 0.012, 0.006, 0.0125])
+    k = kernels["sq_linear"]
+    assert abs(k["achieved_tops"] - 2 * 512 * 4096 * 4096 / 12.5e-6 / 1e12) < 1e-6
+    assert abs(roof["frac"] - k["achieved_tops"] / (bf16 * 2)) < 1e-9
+    c = kernels["sq_calibrate"]
+    assert c["algorithmic_bytes"] == 2 * 512 * 4096 + 2 * 4096 * 4096 + 8 * 4096
+    assert abs(c["frac_of_measured_hbm"] - c["algorithmic_bytes"] / 10e-6 / 1e9 / hbm) < 1e-9
+    wl, (kernels, roof) = _report("decode", [0.030, 0.040, 0.010, 0.014])
+    assert roof["kernel"] == "sq_prepare_weight" and roof["unit"] == "GB/s"
+    assert kernels["sq_linear"]["algorithmic_bytes"] == 8 * 8192 + 8192 * 8192 + 2 * 8 * 8192 + 4 * 8 + 4 * 8192
+
+
+def test_long_kernels_use_the_sustained_peak():
+    hbm, bf16, bf16_sus, _ = bench.peaks()
+    wl, (kernels, roof) = _report("prefill", [0.08, 0.14, 0.06, 1.5])
+    if bf16_sus is not None:
+        assert kernels["sq_linear"]["peak"] == "sustained"
+        assert abs(roof["peak"] - bf16_sus * 2) < 1e-9
+    wl, (kernels, roof) = _report("mlp", [0.02, 0.03, 0.01, 0.08])
+    assert kernels["sq_linear"]["peak"] == "burst"
