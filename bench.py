@@ -67,6 +67,8 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default="proj", choices=sorted(workloads.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--path", default="smoothquant", choices=["smoothquant", "per-tensor"],
+                    help="per-tensor: the baseline W8A8 path (one scale per tensor) on the same workload")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=50)
@@ -76,14 +78,17 @@ def parse_args():
     return ap.parse_args()
 
 
-def workload_config(wl):
-    return {
+def workload_config(wl, path="smoothquant"):
+    c = {
         "workload": f"{wl.name}: X[{wl.M}x{wl.K}] W[{wl.N}x{wl.K}] bf16, alpha {wl.alpha_f32:g}, "
                     f"{wl.outliers} outlier channels x{wl.outlier_scale:g}, calibration {wl.R} rows, "
                     f"{'bias' if wl.has_bias else 'no bias'}",
         "M": wl.M, "N": wl.N, "K": wl.K, "R": wl.R,
         "l2": "flushed before every timed step (256 MiB write, then 512 MiB read); inputs smaller than L2",
     }
+    if path != "smoothquant":
+        c["workload"] = "per-tensor W8A8 baseline (one scale per tensor), " + c["workload"]
+    return c
 
 
 def peaks():
@@ -102,6 +107,9 @@ def algorithmic_work(wl):
         "sq_prepare_weight": (3 * N * K + 4 * N + 4 * K, 0),
         "sq_quantize_act": (3 * M * K + 4 * M + 4 * K, 0),
         "sq_linear": (M * K + N * K + 2 * M * N + 4 * M + 4 * N, 2 * M * N * K),
+        # one scale per tensor: the data once in, the codes and the scale row out
+        "sq_quantize_per_tensor(W)": (3 * N * K + 4 * N, 0),
+        "sq_quantize_per_tensor(X)": (3 * M * K + 4 * M, 0),
     }
 
 
@@ -212,8 +220,12 @@ class ClockSampler:
 
 
 # --------------------------------------------------------------- CPU oracle
-def oracle_step(inp, wl, rows=None):
+def oracle_step(inp, wl, rows=None, path="smoothquant"):
     from oracle import smoothquant as O
+    if path == "per-tensor":
+        from oracle import per_tensor as PT
+        X = inp["X"] if rows is None else inp["X"][:rows]
+        return PT.linear_per_tensor(X, inp["W"], inp["bias"])[0]
     s, _ = O.calibrate(inp["C"], inp["W"], wl.alpha_f32)
     Wq, ws = O.fold_and_quantize_weight(inp["W"], s)
     X = inp["X"] if rows is None else inp["X"][:rows]
@@ -232,13 +244,13 @@ def cpu_threads():
     return len(os.sched_getaffinity(0))
 
 
-def cpu_oracle_rate(wl, seconds, max_steps=None):
+def cpu_oracle_rate(wl, seconds, max_steps=None, path="smoothquant"):
     """Tokens/s of the oracle on whole steps, run until `seconds` pass."""
     inp = workloads.make_inputs(wl)
-    oracle_step(inp, wl)  # warm (page-in, BLAS threads)
+    oracle_step(inp, wl, path=path)  # warm (page-in, BLAS threads)
     n, t0 = 0, time.perf_counter()
     while True:
-        oracle_step(inp, wl)
+        oracle_step(inp, wl, path=path)
         n += 1
         el = time.perf_counter() - t0
         if el >= seconds or (max_steps and n >= max_steps):
@@ -337,14 +349,26 @@ def run_ours(args, wl, rank, world, local_rank):
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     flush_read = torch.ones(FLUSH_READ_BYTES // 4, dtype=torch.int32, device=dev)
 
-    calls = {
-        "sq_calibrate": lambda: sq.sq_calibrate(C, W, wl.alpha_f32, s=s, workspace=ws_cal),
-        "sq_prepare_weight": lambda: sq.sq_prepare_weight(W, s, Wq=Wq, w_scale=w_scale),
-        "sq_quantize_act": lambda: sq.sq_quantize_act(X, s, Xq=Xq, x_scale=x_scale),
-        "sq_linear": lambda: sq.sq_linear(Xq, x_scale, Wq, w_scale, b, Y=Y, workspace=ws_lin),
-    }
-    # kernels per call: calibration clears its workspace with a small kernel first
-    launches_per_call = {"sq_calibrate": 2, "sq_prepare_weight": 1, "sq_quantize_act": 1, "sq_linear": 1}
+    if args.path == "per-tensor":
+        ws_pt = torch.empty(sq.sq_quantize_per_tensor_workspace_bytes(), dtype=torch.uint8, device=dev)
+        ws_pt2 = torch.empty_like(ws_pt)
+        calls = {
+            "sq_quantize_per_tensor(W)": lambda: sq.sq_quantize_per_tensor(W, Aq=Wq, scale_rows=w_scale,
+                                                                           workspace=ws_pt),
+            "sq_quantize_per_tensor(X)": lambda: sq.sq_quantize_per_tensor(X, Aq=Xq, scale_rows=x_scale,
+                                                                           workspace=ws_pt2),
+            "sq_linear": lambda: sq.sq_linear(Xq, x_scale, Wq, w_scale, b, Y=Y, workspace=ws_lin),
+        }
+        launches_per_call = {"sq_quantize_per_tensor(W)": 2, "sq_quantize_per_tensor(X)": 2, "sq_linear": 1}
+    else:
+        calls = {
+            "sq_calibrate": lambda: sq.sq_calibrate(C, W, wl.alpha_f32, s=s, workspace=ws_cal),
+            "sq_prepare_weight": lambda: sq.sq_prepare_weight(W, s, Wq=Wq, w_scale=w_scale),
+            "sq_quantize_act": lambda: sq.sq_quantize_act(X, s, Xq=Xq, x_scale=x_scale),
+            "sq_linear": lambda: sq.sq_linear(Xq, x_scale, Wq, w_scale, b, Y=Y, workspace=ws_lin),
+        }
+        # kernels per call: calibration clears its workspace with a small kernel first
+        launches_per_call = {"sq_calibrate": 2, "sq_prepare_weight": 1, "sq_quantize_act": 1, "sq_linear": 1}
     names = list(calls)
     # initialise library caches outside capture, then capture the step twice:
     # as one graph with no nodes between the calls (the kernels overlap each
@@ -461,9 +485,14 @@ def run_ours(args, wl, rank, world, local_rank):
             dX.copy_(hX, non_blocking=True)
             if db is not None:
                 db.copy_(hb, non_blocking=True)
-            sq.sq_calibrate(dC, dW, wl.alpha_f32, s=s, workspace=ws_cal)
-            sq.sq_prepare_weight(dW, s, Wq=Wq, w_scale=w_scale)
-            sq.sq_forward(dX, s, Wq, w_scale, db, Y=Y, workspace=ws_fwd)
+            if args.path == "per-tensor":
+                sq.sq_quantize_per_tensor(dW, Aq=Wq, scale_rows=w_scale, workspace=ws_pt)
+                sq.sq_quantize_per_tensor(dX, Aq=Xq, scale_rows=x_scale, workspace=ws_pt2)
+                sq.sq_linear(Xq, x_scale, Wq, w_scale, db, Y=Y, workspace=ws_lin)
+            else:
+                sq.sq_calibrate(dC, dW, wl.alpha_f32, s=s, workspace=ws_cal)
+                sq.sq_prepare_weight(dW, s, Wq=Wq, w_scale=w_scale)
+                sq.sq_forward(dX, s, Wq, w_scale, db, Y=Y, workspace=ws_fwd)
             hY.copy_(Y, non_blocking=True)
 
         for _ in range(3):
@@ -481,7 +510,8 @@ def run_ours(args, wl, rank, world, local_rank):
         h2d = sum(t.numel() * t.element_size() for t in (hC, hW, hX) + ((hb,) if hb is not None else ()))
         e2e = {"value": whole_job_rate(wl.M, world, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": hY.numel() * hY.element_size(), "ms_per_step": e2e_ms,
-               "call": "sq_calibrate + sq_prepare_weight + sq_forward"}
+               "call": ("sq_quantize_per_tensor(W) + sq_quantize_per_tensor(X) + sq_linear"
+                        if args.path == "per-tensor" else "sq_calibrate + sq_prepare_weight + sq_forward")}
 
     if rank != 0:
         return
@@ -490,15 +520,17 @@ def run_ours(args, wl, rank, world, local_rank):
 
     cpu = None
     if not args.no_cpu_baseline and world == 1:
-        v, n, el = cpu_oracle_rate(wl, args.cpu_seconds)
+        v, n, el = cpu_oracle_rate(wl, args.cpu_seconds, path=args.path)
         cpu = {"value": v, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
-               "sample": f"{n} whole {wl.name} steps in {el:.1f} s (calibrate, fold+quantise W, forward)"}
+               "sample": f"{n} whole {wl.name} steps in {el:.1f} s ("
+                         + ("quantise W and X per tensor, product" if args.path == "per-tensor"
+                            else "calibrate, fold+quantise W, forward") + ")"}
 
     value = whole_job_rate(wl.M, world, step_ms)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "int8", "data": "synthetic", "config": workload_config(wl),
+        "vs_baseline": None, "dtype": "int8", "data": "synthetic", "config": workload_config(wl, args.path),
         "tops_per_step": 2.0 * wl.M * wl.N * wl.K * world / (step_ms * 1e-3) / 1e12,
         "gemm_tops": 2 * wl.M * wl.N * wl.K / (per_call["sq_linear"] * 1e-3) / 1e12,
         "roofline": roof, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,

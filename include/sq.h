@@ -153,6 +153,30 @@ SQ_API sq_status sq_prepare_weight(const sq_bf16* W, int64_t N, int64_t K, const
 SQ_API sq_status sq_quantize_act(const sq_bf16* X, int64_t M, int64_t K, const float* s,
                           int8_t* Xq, float* x_scale, void* stream);
 
+/* ------------------------------------------- per-tensor baseline quantiser
+ * sq_quantize_per_tensor -- one scale for a whole tensor, the W8A8 variant the
+ * SmoothQuant path is compared with.  Page: "quantized_linear.py --
+ * QuantizedLinear + apply_w8a8", quantize_tensor (scale = max|x| / 127 on fp32
+ * values, replaced by 1.0 when below 1e-8; codes round-half-even of the fp32
+ * quotient x / scale, clamped to [-128, 127]) and QuantizedLinear.forward (the
+ * product of the two dequantised tensors plus the bias).  With the weight and
+ * the activations each quantised this way, sq_linear(Xq, x_scale, Wq,
+ * w_scale, bias) computes that forward with an exact int8 product.
+ *   A[rows][K]       bf16 tensor (weight or activations), K % 16 == 0
+ *   Aq[rows][K]      OUT int8 codes (always within [-127, 127]: the maximum
+ *                    maps to +-127)
+ *   scale_rows[rows] OUT fp32: every entry holds the tensor's scale, the form
+ *                    sq_linear takes for x_scale / w_scale
+ *   workspace        at least sq_quantize_per_tensor_workspace_bytes() bytes,
+ *                    16-byte aligned; contents on entry are ignored
+ * Launches two kernels (block maxima of |A|, then the scale and the codes);
+ * A is read twice from HBM.
+ */
+SQ_API size_t sq_quantize_per_tensor_workspace_bytes(void);
+SQ_API sq_status sq_quantize_per_tensor(const sq_bf16* A, int64_t rows, int64_t K, int8_t* Aq,
+                                        float* scale_rows, void* workspace, size_t workspace_bytes,
+                                        void* stream);
+
 /* ----------------------------------------------------------- int8 linear
  * sq_linear -- Y = bf16( (Xq Wq^T)[m][n] * x_scale[m] * w_scale[n] + bias[n] ).
  * Page: forward ("INT8 x INT8 -> INT32 -> fp32"; bias added after the product).

@@ -35,6 +35,14 @@ def test_every_declared_symbol_is_exported(sq):
     assert not missing, missing
 
 
+def test_binding_has_every_entry_point(sq):
+    """The Python binding carries the C names (sq_last_error and
+    sq_status_string are surfaced through SqError instead)."""
+    missing = [n for n in declared_symbols()
+               if n not in ("sq_last_error", "sq_status_string") and not callable(getattr(sq, n, None))]
+    assert not missing, missing
+
+
 def test_version_and_sizes(sq):
     assert sq.sq_version() == 100
     assert sq.sq_calibrate_workspace_bytes(4096) >= 2 * 4096 * 4
@@ -62,6 +70,13 @@ def test_validation_before_device(sq):
     assert lib.sq_linear(a, a, a, a, None, 4, 8, 200000, a, None, 0, None) == 2
     assert lib.sq_forward(a, a, a, a, None, 4, 8, 64, a, a, 16, None) == 8
     assert lib.sq_gemm_s32(a, a, 4, 0, 64, a, None) == 2
+    ws = lib.sq_quantize_per_tensor_workspace_bytes()
+    assert ws >= 4
+    assert lib.sq_quantize_per_tensor(a, 4, 64, a, a, None, 0, None) == 8
+    assert lib.sq_quantize_per_tensor(a, 4, 64, a, a, a, ws - 4, None) == 8
+    assert lib.sq_quantize_per_tensor(a, 4, 40, a, a, a, ws, None) == 3
+    assert lib.sq_quantize_per_tensor(None, 4, 64, a, a, a, ws, None) == 1
+    assert lib.sq_quantize_per_tensor(a, 0, 64, a, a, a, ws, None) == 2
 
 
 def test_valid_call_without_gpu_fails_cleanly(sq):

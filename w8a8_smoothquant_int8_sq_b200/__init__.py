@@ -22,7 +22,7 @@ import torch
 __all__ = [
     "SqError", "lib", "library_path",
     "sq_version", "sq_calibrate", "sq_calibrate_workspace_bytes", "sq_calibrate_noalloc", "sq_prepare_weight",
-    "sq_quantize_act", "sq_linear", "sq_workspace_bytes", "sq_forward",
+    "sq_quantize_act", "sq_quantize_per_tensor", "sq_quantize_per_tensor_workspace_bytes", "sq_linear", "sq_workspace_bytes", "sq_forward",
     "sq_forward_workspace_bytes", "sq_gemm_s32", "sq_device_status", "sq_debug_fail_after",
     "sq_debug_pipeline_stall",
     "STATUS",
@@ -50,6 +50,8 @@ _SIGNATURES = [
     ("sq_calibrate_noalloc", ctypes.c_int, (_P, _I64, _I64, _P, _I64, ctypes.c_float, _P, _P, _P)),
     ("sq_prepare_weight", ctypes.c_int, (_P, _I64, _I64, _P, _P, _P, _P)),
     ("sq_quantize_act", ctypes.c_int, (_P, _I64, _I64, _P, _P, _P, _P)),
+    ("sq_quantize_per_tensor_workspace_bytes", _SZ, ()),
+    ("sq_quantize_per_tensor", ctypes.c_int, (_P, _I64, _I64, _P, _P, _P, _SZ, _P)),
     ("sq_workspace_bytes", _SZ, (_I64, _I64, _I64)),
     ("sq_linear", ctypes.c_int, (_P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _SZ, _P)),
     ("sq_forward_workspace_bytes", _SZ, (_I64, _I64, _I64)),
@@ -231,6 +233,25 @@ def sq_quantize_act(X: torch.Tensor, s: torch.Tensor, Xq: Optional[torch.Tensor]
     x_scale = _out(x_scale, (M,), torch.float32, X.device, "x_scale")
     _check(_load().sq_quantize_act(_ptr(X), M, K, _ptr(s), _ptr(Xq), _ptr(x_scale), _stream(stream)))
     return Xq, x_scale
+
+
+def sq_quantize_per_tensor_workspace_bytes() -> int:
+    return int(_load().sq_quantize_per_tensor_workspace_bytes())
+
+
+def sq_quantize_per_tensor(A: torch.Tensor, Aq: Optional[torch.Tensor] = None,
+                           scale_rows: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                           stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """(Aq[rows,K] int8, scale_rows[rows] fp32) with one scale for the whole of
+    A[rows,K] bf16 -- the per-tensor baseline; feed the pair to sq_linear."""
+    _want(A, "A", torch.bfloat16, 2)
+    rows, K = A.shape
+    Aq = _out(Aq, (rows, K), torch.int8, A.device, "Aq")
+    scale_rows = _out(scale_rows, (rows,), torch.float32, A.device, "scale_rows")
+    ws = _workspace(workspace, sq_quantize_per_tensor_workspace_bytes(), A.device)
+    _check(_load().sq_quantize_per_tensor(_ptr(A), rows, K, _ptr(Aq), _ptr(scale_rows), _ptr(ws), ws.numel(),
+                                          _stream(stream)))
+    return Aq, scale_rows
 
 
 def sq_linear(Xq: torch.Tensor, x_scale: torch.Tensor, Wq: torch.Tensor, w_scale: torch.Tensor,

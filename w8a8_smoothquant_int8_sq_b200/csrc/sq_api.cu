@@ -216,6 +216,27 @@ sq_status sq_quantize_act(const sq_bf16* X, int64_t M, int64_t K, const float* s
                      "quantize_act launch");
 }
 
+// --------------------------------------------- per-tensor baseline quantiser
+size_t sq_quantize_per_tensor_workspace_bytes(void) { return sq::per_tensor_workspace_bytes(); }
+
+sq_status sq_quantize_per_tensor(const sq_bf16* A, int64_t rows, int64_t K, int8_t* Aq, float* scale_rows,
+                                 void* workspace, size_t workspace_bytes, void* stream) {
+  SQ_TRY(check_k(K, INT32_MAX - 15));
+  SQ_TRY(check_rows(rows, "rows"));
+  SQ_NONNULL(A);
+  SQ_NONNULL(Aq);
+  SQ_NONNULL(scale_rows);
+  if (workspace == nullptr || workspace_bytes < sq::per_tensor_workspace_bytes())
+    return fail(SQ_ERR_WORKSPACE, "workspace must hold sq_quantize_per_tensor_workspace_bytes() = " +
+                                      std::to_string(sq::per_tensor_workspace_bytes()) + " bytes");
+  if (!aligned16(workspace)) return fail(SQ_ERR_ALIGN, "workspace is not 16-byte aligned");
+  sq::DeviceInfo dev;
+  SQ_TRY(prologue(&dev));
+  return cuda_status(sq::launch_quantize_per_tensor(A, rows, K, Aq, scale_rows, workspace,
+                                                    static_cast<cudaStream_t>(stream), dev),
+                     "quantize_per_tensor launch");
+}
+
 // ------------------------------------------------------------- int8 linear
 // SMs assumed when no device can be queried (a B200), so that sizes asked
 // before a device is current are the ones a B200 will want.

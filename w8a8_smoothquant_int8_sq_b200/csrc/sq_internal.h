@@ -95,6 +95,14 @@ cudaError_t launch_calibrate_noalloc(const uint16_t* C, int64_t R, int64_t K, co
 cudaError_t launch_row_quant(bool multiply, const uint16_t* src, int64_t rows, int64_t K, const float* s,
                              int8_t* q, float* scale, cudaStream_t st, const DeviceInfo& dev);
 
+// ---- per-tensor quantisation, the baseline beside SmoothQuant (sq_quant.cu)
+// Workspace: one partial maximum per pass-1 block.
+size_t per_tensor_workspace_bytes();
+// Aq = clamp(rne(fl(A / scale)), -128, 127) with scale = fl(max|A| / 127)
+// (1.0 below 1e-8); every entry of scale_rows[rows] receives the scale.
+cudaError_t launch_quantize_per_tensor(const uint16_t* src, int64_t rows, int64_t K, int8_t* q, float* scale_rows,
+                                       void* ws, cudaStream_t st, const DeviceInfo& dev);
+
 // ---- GEMM (sq_gemm.cu)
 enum class Epilogue { kBf16Dequant = 0, kS32 = 1 };
 

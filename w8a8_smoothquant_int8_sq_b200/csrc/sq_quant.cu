@@ -5,6 +5,9 @@
 //                        s_j = max(mx_j,1e-8)^a / max(mw_j,1e-8)^(1-a), >= 1e-8
 //   row_quant_kernel     per-row symmetric int8 quantisation of W*s (weight
 //                        prep, per output channel) or X/s (activations, per token)
+//   pt_absmax_kernel,    one scale for a whole tensor (the per-tensor W8A8
+//   pt_quant_kernel      baseline: page "quantized_linear.py -- QuantizedLinear
+//                        + apply_w8a8", quantize_tensor)
 //
 // Page: "w8a8_smoothquant.py -- W8A8 com SmoothQuant e alpha APRENDIVEL (V5)",
 // functions _per_channel_max_abs, calibrate_smoothquant,
@@ -579,6 +582,116 @@ static cudaError_t dispatch_rq(const uint16_t* src, int64_t rows, int K, const f
   if (nvec <= 128 * V) return launch_rq<kMul, 4, V>(src, rows, K, s, q, scale, st, dev);
   if (nvec <= 256 * V) return launch_rq<kMul, 8, V>(src, rows, K, s, q, scale, st, dev);
   return launch_rq<kMul, 8, 8>(src, rows, K, s, q, scale, st, dev);  // K up to 16384
+}
+
+// ============================================ per-tensor quantisation (baseline)
+// quantize_tensor of the QuantizedLinear page: scale = max|x| / 127 in fp32
+// (1.0 when below 1e-8), codes rne(fl(x / scale)) clamped to [-128, 127].
+// Since scale = fl(max|x| / 127), |x / scale| exceeds 127 by at most one ulp
+// and every code already lies in [-127, 127]: the clamp is implied.
+// Pass 1 writes one partial maximum per block (plain stores, no atomics and so
+// nothing to clear); pass 2 reduces them in every block and quantises.  The
+// tensor is read as a flat array of 16-byte vectors (rows * K is a multiple
+// of 8), four vectors in flight per thread.
+constexpr int kPtThreads = 256;
+constexpr int kPtVecs = 4;  // vectors per thread per iteration
+constexpr int kPtMaxBlocks = 1024;
+
+__device__ __forceinline__ uint32_t block_max_u32(uint32_t v, uint32_t* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = max(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  if (warp == 0) {
+    v = lane < static_cast<int>(blockDim.x >> 5) ? red[lane] : 0u;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = max(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+    if (lane == 0) red[0] = v;
+  }
+  __syncthreads();
+  return red[0];
+}
+
+__global__ void __launch_bounds__(kPtThreads) pt_absmax_kernel(const uint4* __restrict__ x, int64_t nvec,
+                                                               uint32_t* __restrict__ part) {
+  __shared__ uint32_t red[kPtThreads / 32];
+  griddep_wait();
+  griddep_launch_dependents();
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * kPtThreads;
+  uint32_t m = 0;  // packed pair of |bf16| patterns
+  for (int64_t v0 = static_cast<int64_t>(blockIdx.x) * kPtThreads + threadIdx.x; v0 < nvec; v0 += kPtVecs * stride) {
+    uint4 a[kPtVecs];
+#pragma unroll
+    for (int i = 0; i < kPtVecs; ++i) {
+      const int64_t v = v0 + i * stride;
+      a[i] = v < nvec ? __ldcs(x + v) : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int i = 0; i < kPtVecs; ++i) {
+      m = __vmaxu2(m, a[i].x & 0x7FFF7FFFu);
+      m = __vmaxu2(m, a[i].y & 0x7FFF7FFFu);
+      m = __vmaxu2(m, a[i].z & 0x7FFF7FFFu);
+      m = __vmaxu2(m, a[i].w & 0x7FFF7FFFu);
+    }
+  }
+  const uint32_t h = block_max_u32(max(m & 0xFFFFu, m >> 16), red);
+  if (threadIdx.x == 0) part[blockIdx.x] = h << 16;  // fp32 pattern of the bf16 maximum
+}
+
+__global__ void __launch_bounds__(kPtThreads) pt_quant_kernel(const uint4* __restrict__ x, int64_t nvec,
+                                                              const uint32_t* __restrict__ part, int nparts,
+                                                              int64_t rows, uint2* __restrict__ q,
+                                                              float* __restrict__ scale_rows) {
+  __shared__ uint32_t red[kPtThreads / 32];
+  griddep_wait();
+  griddep_launch_dependents();
+  uint32_t m = 0;
+  for (int i = threadIdx.x; i < nparts; i += kPtThreads) m = max(m, __ldcg(part + i));
+  const float mx = __uint_as_float(block_max_u32(m, red));
+  float sc = __fdiv_rn(mx, kQmax);
+  if (sc < kClampFloor) sc = 1.0f;
+  const float rsc = __frcp_rn(sc);
+  const f2x nsc2 = f2_pack(-sc, -sc), rsc2 = f2_pack(rsc, rsc);
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * kPtThreads;
+  for (int64_t v0 = static_cast<int64_t>(blockIdx.x) * kPtThreads + threadIdx.x; v0 < nvec; v0 += kPtVecs * stride) {
+    uint4 a[kPtVecs];
+#pragma unroll
+    for (int i = 0; i < kPtVecs; ++i) {
+      const int64_t v = v0 + i * stride;
+      a[i] = v < nvec ? __ldcs(x + v) : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int i = 0; i < kPtVecs; ++i) {
+      const int64_t v = v0 + i * stride;
+      if (v < nvec) {
+        f2x c[4];
+        c[0] = f2_round_codes(f2_div_rn(f2_from_bf16x2(a[i].x), nsc2, rsc2));
+        c[1] = f2_round_codes(f2_div_rn(f2_from_bf16x2(a[i].y), nsc2, rsc2));
+        c[2] = f2_round_codes(f2_div_rn(f2_from_bf16x2(a[i].z), nsc2, rsc2));
+        c[3] = f2_round_codes(f2_div_rn(f2_from_bf16x2(a[i].w), nsc2, rsc2));
+        q[v] = pack8_codes(c[0], c[1], c[2], c[3]);
+      }
+    }
+  }
+  for (int64_t r = static_cast<int64_t>(blockIdx.x) * kPtThreads + threadIdx.x; r < rows; r += stride)
+    scale_rows[r] = sc;
+}
+
+size_t per_tensor_workspace_bytes() { return kPtMaxBlocks * sizeof(uint32_t); }
+
+cudaError_t launch_quantize_per_tensor(const uint16_t* src, int64_t rows, int64_t K, int8_t* q, float* scale_rows,
+                                       void* ws, cudaStream_t st, const DeviceInfo& dev) {
+  const int64_t nvec = rows * K / 8;
+  const int64_t want = (nvec + kPtVecs * kPtThreads - 1) / (kPtVecs * kPtThreads);
+  const int blocks = static_cast<int>(std::max<int64_t>(
+      1, std::min<int64_t>({want, static_cast<int64_t>(4) * dev.sm_count, static_cast<int64_t>(kPtMaxBlocks)})));
+  uint32_t* part = static_cast<uint32_t*>(ws);
+  const uint4* x = reinterpret_cast<const uint4*>(src);
+  cudaError_t e = launch_pdl(pt_absmax_kernel, dim3(blocks), dim3(kPtThreads), 0, st, x, nvec, part);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(pt_quant_kernel, dim3(blocks), dim3(kPtThreads), 0, st, x, nvec,
+                    static_cast<const uint32_t*>(part), blocks, rows, reinterpret_cast<uint2*>(q), scale_rows);
 }
 
 cudaError_t launch_row_quant(bool multiply, const uint16_t* src, int64_t rows, int64_t K, const float* s, int8_t* q,
