@@ -177,6 +177,22 @@ SQ_API sq_status sq_quantize_per_tensor(const sq_bf16* A, int64_t rows, int64_t 
                                         float* scale_rows, void* workspace, size_t workspace_bytes,
                                         void* stream);
 
+/* ------------------------------------------------ int8 weight-only linear
+ * sq_linear_weight_only -- the decode comparison point beside W8A8: the
+ * activations stay bf16 and only the weight is int8.  Page: torchao,
+ * Int8WeightOnlyQuantizedLinearWeight._quantized_op:
+ *     Y[m][n] = bf16( (sum_k X[m][k] * Wq[n][k]) * w_scale[n] + bias[n] ).
+ *   X[M][K] bf16, Wq[N][K] int8 and w_scale[N] fp32 (per output channel, e.g.
+ *   from sq_prepare_weight with s = 1), bias[N] bf16 or NULL -> Y[M][N] bf16.
+ * The sum runs in fp32 on the CUDA cores (there is no int8 x bf16 tensor-core
+ * product), in an order of its own, and is rounded once to bf16 after the
+ * scale and bias: the result is within one bf16 ulp plus the fp32 summation
+ * error of the exact value.  Built for few tokens (groups of 8 re-read Wq).
+ * K <= 16384, a multiple of 16.
+ */
+SQ_API sq_status sq_linear_weight_only(const sq_bf16* X, int64_t M, const int8_t* Wq, const float* w_scale,
+                                       const sq_bf16* bias, int64_t N, int64_t K, sq_bf16* Y, void* stream);
+
 /* ----------------------------------------------------------- int8 linear
  * sq_linear -- Y = bf16( (Xq Wq^T)[m][n] * x_scale[m] * w_scale[n] + bias[n] ).
  * Page: forward ("INT8 x INT8 -> INT32 -> fp32"; bias added after the product).

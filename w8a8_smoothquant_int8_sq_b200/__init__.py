@@ -22,7 +22,7 @@ import torch
 __all__ = [
     "SqError", "lib", "library_path",
     "sq_version", "sq_calibrate", "sq_calibrate_workspace_bytes", "sq_calibrate_noalloc", "sq_prepare_weight",
-    "sq_quantize_act", "sq_quantize_per_tensor", "sq_quantize_per_tensor_workspace_bytes", "sq_linear", "sq_workspace_bytes", "sq_forward",
+    "sq_quantize_act", "sq_quantize_per_tensor", "sq_quantize_per_tensor_workspace_bytes", "sq_linear_weight_only", "sq_linear", "sq_workspace_bytes", "sq_forward",
     "sq_forward_workspace_bytes", "sq_gemm_s32", "sq_device_status", "sq_debug_fail_after",
     "sq_debug_pipeline_stall",
     "STATUS",
@@ -52,6 +52,7 @@ _SIGNATURES = [
     ("sq_quantize_act", ctypes.c_int, (_P, _I64, _I64, _P, _P, _P, _P)),
     ("sq_quantize_per_tensor_workspace_bytes", _SZ, ()),
     ("sq_quantize_per_tensor", ctypes.c_int, (_P, _I64, _I64, _P, _P, _P, _SZ, _P)),
+    ("sq_linear_weight_only", ctypes.c_int, (_P, _I64, _P, _P, _P, _I64, _I64, _P, _P)),
     ("sq_workspace_bytes", _SZ, (_I64, _I64, _I64)),
     ("sq_linear", ctypes.c_int, (_P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _SZ, _P)),
     ("sq_forward_workspace_bytes", _SZ, (_I64, _I64, _I64)),
@@ -252,6 +253,25 @@ def sq_quantize_per_tensor(A: torch.Tensor, Aq: Optional[torch.Tensor] = None,
     _check(_load().sq_quantize_per_tensor(_ptr(A), rows, K, _ptr(Aq), _ptr(scale_rows), _ptr(ws), ws.numel(),
                                           _stream(stream)))
     return Aq, scale_rows
+
+
+def sq_linear_weight_only(X: torch.Tensor, Wq: torch.Tensor, w_scale: torch.Tensor,
+                          bias: Optional[torch.Tensor] = None, Y: Optional[torch.Tensor] = None,
+                          stream=None) -> torch.Tensor:
+    """Y[M,N] bf16 = bf16((X Wq^T) * w_scale[n] + bias[n]) with X[M,K] bf16 (weight-only int8)."""
+    _want(X, "X", torch.bfloat16, 2)
+    _want(Wq, "Wq", torch.int8, 2)
+    _want(w_scale, "w_scale", torch.float32, 1)
+    M, K = X.shape
+    N = Wq.shape[0]
+    if Wq.shape[1] != K or w_scale.shape[0] != N:
+        raise ValueError("inconsistent shapes")
+    if bias is not None:
+        _want(bias, "bias", torch.bfloat16, 1)
+    Y = _out(Y, (M, N), torch.bfloat16, X.device, "Y")
+    _check(_load().sq_linear_weight_only(_ptr(X), M, _ptr(Wq), _ptr(w_scale), _ptr(bias), N, K, _ptr(Y),
+                                         _stream(stream)))
+    return Y
 
 
 def sq_linear(Xq: torch.Tensor, x_scale: torch.Tensor, Wq: torch.Tensor, w_scale: torch.Tensor,

@@ -237,6 +237,23 @@ sq_status sq_quantize_per_tensor(const sq_bf16* A, int64_t rows, int64_t K, int8
                      "quantize_per_tensor launch");
 }
 
+// ------------------------------------------------- int8 weight-only linear
+sq_status sq_linear_weight_only(const sq_bf16* X, int64_t M, const int8_t* Wq, const float* w_scale,
+                                const sq_bf16* bias, int64_t N, int64_t K, sq_bf16* Y, void* stream) {
+  SQ_TRY(check_k(K, sq::kMaxQuantK));
+  SQ_TRY(check_rows(M, "M"));
+  SQ_TRY(check_rows(N, "N"));
+  SQ_NONNULL(X);
+  SQ_NONNULL(Wq);
+  SQ_NONNULL(w_scale);
+  SQ_NONNULL(Y);
+  if (bias != nullptr && !aligned16(bias)) return fail(SQ_ERR_ALIGN, "bias is not 16-byte aligned");
+  sq::DeviceInfo dev;
+  SQ_TRY(prologue(&dev));
+  return cuda_status(sq::launch_weight_only(X, M, Wq, w_scale, bias, N, K, Y, static_cast<cudaStream_t>(stream), dev),
+                     "weight-only linear launch");
+}
+
 // ------------------------------------------------------------- int8 linear
 // SMs assumed when no device can be queried (a B200), so that sizes asked
 // before a device is current are the ones a B200 will want.

@@ -695,10 +695,11 @@ cudaError_t read_device_status(uint32_t* flags, bool clear) {
     e = cudaMemcpyToSymbol(g_sq_device_status, &z, sizeof(z));
     if (e != cudaSuccess) return e;
   }
-  uint32_t q = 0;
+  uint32_t q = 0, w = 0;
   e = read_quant_status(&q, clear);
+  if (e == cudaSuccess) e = read_weight_only_status(&w, clear);
   if (e != cudaSuccess) return e;
-  *flags = v | q;
+  *flags = v | q | w;
   return cudaSuccess;
 }
 

@@ -103,6 +103,16 @@ size_t per_tensor_workspace_bytes();
 cudaError_t launch_quantize_per_tensor(const uint16_t* src, int64_t rows, int64_t K, int8_t* q, float* scale_rows,
                                        void* ws, cudaStream_t st, const DeviceInfo& dev);
 
+// ---- int8 weight-only linear, the decode comparison point (sq_weight_only.cu)
+// Y = bf16((X Wq^T) * w_scale + bias) with X in bf16; cudaErrorNotSupported
+// when K exceeds the kernel's 4 x 4096 columns.
+cudaError_t launch_weight_only(const uint16_t* X, int64_t M, const int8_t* Wq, const float* w_scale,
+                               const uint16_t* bias, int64_t N, int64_t K, uint16_t* Y, cudaStream_t st,
+                               const DeviceInfo& dev);
+
+// Status word of the weight-only kernel (bit 0: a wait timed out).
+cudaError_t read_weight_only_status(uint32_t* flags, bool clear);
+
 // ---- GEMM (sq_gemm.cu)
 enum class Epilogue { kBf16Dequant = 0, kS32 = 1 };
 
