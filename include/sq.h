@@ -193,6 +193,53 @@ SQ_API sq_status sq_quantize_per_tensor(const sq_bf16* A, int64_t rows, int64_t 
 SQ_API sq_status sq_linear_weight_only(const sq_bf16* X, int64_t M, const int8_t* Wq, const float* w_scale,
                                        const sq_bf16* bias, int64_t N, int64_t K, sq_bf16* Y, void* stream);
 
+/* ---------------------------------- learnable-alpha straight-through backward
+ * sq_ste_backward -- gradients of the quantised-mode forward of the
+ * learnable-alpha layer.  Page: "w8a8_smoothquant.py -- W8A8 com SmoothQuant e
+ * alpha APRENDIVEL (V5)": SmoothQuantW8A8.alpha (alpha = sigmoid(eta_alpha)),
+ * SmoothQuantW8A8.forward (s recomputed from the running activation max and
+ * the detached weight max with the trainable alpha, X / s and weight * s
+ * fake-quantised per token and per output channel, Y = X_q_deq W_q_deq^T + b)
+ * and STEQuantize.backward (the gradient passes through round and clamp; the
+ * scales receive none).  With G = dL/dY:
+ *     dX[m][k] = (G Wdq)[m][k] / s[k]           Wdq = Wq * w_scale (per row n)
+ *     dW[n][k] = (G^T Xdq)[n][k] * s[k]         Xdq = Xq * x_scale (per row m)
+ *     db[n]    = sum_m G[m][n]
+ *     d_eta    = alpha (1 - alpha) sum_k ds[k] raw[k] (ln mx[k] + ln mw[k]),
+ * where ds[k] = sum_n dL/dW_smooth[n][k] W[n][k] - sum_m dL/dX_smooth[m][k]
+ * X[m][k] / s[k]^2, raw[k] = mx[k]^alpha / mw[k]^(1-alpha) (mx, mw clamped at
+ * 1e-8; channels with raw[k] < 1e-8 sit on the clamp of s and contribute
+ * nothing) and mw[k] = max_n |W[n][k]|.
+ *   G[M][N] bf16        dL/dY (an auxiliary loss on Y enters through it)
+ *   X[M][K], W[N][K]    the layer's bf16 input and weight
+ *   s[K]                the forward's smoothing factor (sq_calibrate with
+ *                       mx_inout = mx, R = 0 and this alpha)
+ *   mx[K]               the running activation max (calib_max_abs)
+ *   alpha               the fp32 alpha of the forward, in [0, 1]
+ *   Xq, x_scale, Wq, w_scale   the forward's codes and scales
+ *                       (sq_quantize_act and sq_prepare_weight with s)
+ *   dX[M][K], dW[N][K]  OUT fp32
+ *   db[N]               OUT fp32, or NULL
+ *   ds[K]               OUT fp32: dL/ds (the gradient reaching s), or NULL
+ *   d_eta[1]            OUT fp32: dL/d eta_alpha
+ *   workspace           sq_ste_backward_workspace_bytes(M, N, K) bytes,
+ *                       16-byte aligned, contents ignored on entry
+ * Requirements beyond the general ones: N % 8 == 0 (G is read by TMA rows).
+ * The two products run on the tensor cores with the codes as exact bf16
+ * operands and G times the scale split into two bf16 halves (2^-16 relative),
+ * accumulating in fp32: each element of dX and dW is within
+ * 2^-16 + 2^-23 + 2C * 2^-22 of the sum of its absolute products (C the
+ * contraction length).  ds is formed from the quantisation errors W*s - Wdq
+ * and X/s - Xdq, so it carries that relative error without cancellation.
+ * Launches 7 kernels; reads G once.
+ */
+SQ_API size_t sq_ste_backward_workspace_bytes(int64_t M, int64_t N, int64_t K);
+SQ_API sq_status sq_ste_backward(const sq_bf16* G, const sq_bf16* X, const sq_bf16* W, const float* s,
+                                 const float* mx, float alpha, const int8_t* Xq, const float* x_scale,
+                                 const int8_t* Wq, const float* w_scale, int64_t M, int64_t N, int64_t K,
+                                 float* dX, float* dW, float* db, float* ds, float* d_eta, void* workspace,
+                                 size_t workspace_bytes, void* stream);
+
 /* ----------------------------------------------------------- int8 linear
  * sq_linear -- Y = bf16( (Xq Wq^T)[m][n] * x_scale[m] * w_scale[n] + bias[n] ).
  * Page: forward ("INT8 x INT8 -> INT32 -> fp32"; bias added after the product).

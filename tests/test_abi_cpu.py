@@ -77,6 +77,21 @@ def test_validation_before_device(sq):
     assert lib.sq_quantize_per_tensor(a, 4, 40, a, a, a, ws, None) == 3
     assert lib.sq_quantize_per_tensor(None, 4, 64, a, a, a, ws, None) == 1
     assert lib.sq_quantize_per_tensor(a, 0, 64, a, a, a, ws, None) == 2
+    # straight-through backward: N % 8, alpha, NULL, workspace size
+    wsb = lib.sq_ste_backward_workspace_bytes(4, 64, 64)
+    assert wsb >= 64 * 64 * 2 + 64 * 8 * 2 + 4 * 64 * 8 * 2 + 3 * 64 * 4
+    f = ctypes.c_float
+
+    def bwd(G=a, N=64, alpha=0.5, db=None, ds=None, ws=a, nbytes=wsb, K=64):
+        return lib.sq_ste_backward(G, a, a, a, a, f(alpha), a, a, a, a, 4, N, K, a, a, db, ds, a, ws, nbytes, None)
+    assert bwd(N=60) == 3
+    assert bwd(alpha=1.5) == 4
+    assert bwd(alpha=float("nan")) == 4
+    assert bwd(G=None) == 1
+    assert bwd(db=mis) == 3
+    assert bwd(ds=mis) == 3
+    assert bwd(nbytes=wsb - 1) == 8
+    assert bwd(K=40) == 3
 
 
 def test_valid_call_without_gpu_fails_cleanly(sq):

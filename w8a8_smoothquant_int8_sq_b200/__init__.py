@@ -22,7 +22,8 @@ import torch
 __all__ = [
     "SqError", "lib", "library_path",
     "sq_version", "sq_calibrate", "sq_calibrate_workspace_bytes", "sq_calibrate_noalloc", "sq_prepare_weight",
-    "sq_quantize_act", "sq_quantize_per_tensor", "sq_quantize_per_tensor_workspace_bytes", "sq_linear_weight_only", "sq_linear", "sq_workspace_bytes", "sq_forward",
+    "sq_quantize_act", "sq_quantize_per_tensor", "sq_quantize_per_tensor_workspace_bytes", "sq_linear_weight_only", "sq_ste_backward",
+    "sq_ste_backward_workspace_bytes", "sq_linear", "sq_workspace_bytes", "sq_forward",
     "sq_forward_workspace_bytes", "sq_gemm_s32", "sq_device_status", "sq_debug_fail_after",
     "sq_debug_pipeline_stall",
     "STATUS",
@@ -53,6 +54,9 @@ _SIGNATURES = [
     ("sq_quantize_per_tensor_workspace_bytes", _SZ, ()),
     ("sq_quantize_per_tensor", ctypes.c_int, (_P, _I64, _I64, _P, _P, _P, _SZ, _P)),
     ("sq_linear_weight_only", ctypes.c_int, (_P, _I64, _P, _P, _P, _I64, _I64, _P, _P)),
+    ("sq_ste_backward_workspace_bytes", _SZ, (_I64, _I64, _I64)),
+    ("sq_ste_backward", ctypes.c_int, (_P, _P, _P, _P, _P, ctypes.c_float, _P, _P, _P, _P, _I64, _I64, _I64,
+                                       _P, _P, _P, _P, _P, _P, _SZ, _P)),
     ("sq_workspace_bytes", _SZ, (_I64, _I64, _I64)),
     ("sq_linear", ctypes.c_int, (_P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _SZ, _P)),
     ("sq_forward_workspace_bytes", _SZ, (_I64, _I64, _I64)),
@@ -272,6 +276,51 @@ def sq_linear_weight_only(X: torch.Tensor, Wq: torch.Tensor, w_scale: torch.Tens
     _check(_load().sq_linear_weight_only(_ptr(X), M, _ptr(Wq), _ptr(w_scale), _ptr(bias), N, K, _ptr(Y),
                                          _stream(stream)))
     return Y
+
+
+def sq_ste_backward_workspace_bytes(M: int, N: int, K: int) -> int:
+    return int(_load().sq_ste_backward_workspace_bytes(M, N, K))
+
+
+def sq_ste_backward(G: torch.Tensor, X: torch.Tensor, W: torch.Tensor, s: torch.Tensor, mx: torch.Tensor,
+                    alpha: float, Xq: torch.Tensor, x_scale: torch.Tensor, Wq: torch.Tensor,
+                    w_scale: torch.Tensor, with_db: bool = True, with_ds: bool = False,
+                    dX: Optional[torch.Tensor] = None, dW: Optional[torch.Tensor] = None,
+                    db: Optional[torch.Tensor] = None, ds: Optional[torch.Tensor] = None,
+                    d_eta: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                    stream=None):
+    """Straight-through backward of the learnable-alpha layer: returns
+    ``(dX [M,K] fp32, dW [N,K] fp32, db [N] fp32 or None, ds [K] fp32 or None,
+    d_eta [1] fp32)`` from G = dL/dY [M,N] bf16 and the forward's inputs, s,
+    running max, alpha, codes and scales."""
+    _want(G, "G", torch.bfloat16, 2)
+    _want(X, "X", torch.bfloat16, 2)
+    _want(W, "W", torch.bfloat16, 2)
+    _want(s, "s", torch.float32, 1)
+    _want(mx, "mx", torch.float32, 1)
+    _want(Xq, "Xq", torch.int8, 2)
+    _want(x_scale, "x_scale", torch.float32, 1)
+    _want(Wq, "Wq", torch.int8, 2)
+    _want(w_scale, "w_scale", torch.float32, 1)
+    M, K = X.shape
+    N = W.shape[0]
+    if (G.shape != (M, N) or W.shape[1] != K or s.shape[0] != K or mx.shape[0] != K or Xq.shape != (M, K)
+            or x_scale.shape[0] != M or Wq.shape != (N, K) or w_scale.shape[0] != N):
+        raise ValueError("inconsistent shapes")
+    dX = _out(dX, (M, K), torch.float32, X.device, "dX")
+    dW = _out(dW, (N, K), torch.float32, X.device, "dW")
+    if with_db or db is not None:
+        db = _out(db, (N,), torch.float32, X.device, "db")
+    if with_ds or ds is not None:
+        ds = _out(ds, (K,), torch.float32, X.device, "ds")
+    d_eta = _out(d_eta, (1,), torch.float32, X.device, "d_eta")
+    nbytes = sq_ste_backward_workspace_bytes(M, N, K)
+    ws = _workspace(workspace, nbytes, X.device)
+    _check(_load().sq_ste_backward(_ptr(G), _ptr(X), _ptr(W), _ptr(s), _ptr(mx), ctypes.c_float(alpha), _ptr(Xq),
+                                   _ptr(x_scale), _ptr(Wq), _ptr(w_scale), M, N, K, _ptr(dX), _ptr(dW), _ptr(db),
+                                   _ptr(ds), _ptr(d_eta), _ptr(ws), nbytes if workspace is None else ws.numel(),
+                                   _stream(stream)))
+    return dX, dW, db, ds, d_eta
 
 
 def sq_linear(Xq: torch.Tensor, x_scale: torch.Tensor, Wq: torch.Tensor, w_scale: torch.Tensor,

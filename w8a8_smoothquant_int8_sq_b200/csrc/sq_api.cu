@@ -254,6 +254,70 @@ sq_status sq_linear_weight_only(const sq_bf16* X, int64_t M, const int8_t* Wq, c
                      "weight-only linear launch");
 }
 
+// ------------------------------------- learnable-alpha straight-through backward
+size_t sq_ste_backward_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  if (M <= 0 || N <= 0 || K <= 0) return 0;
+  return sq::ste_workspace_bytes(M, N, K);
+}
+
+sq_status sq_ste_backward(const sq_bf16* G, const sq_bf16* X, const sq_bf16* W, const float* s, const float* mx,
+                          float alpha, const int8_t* Xq, const float* x_scale, const int8_t* Wq,
+                          const float* w_scale, int64_t M, int64_t N, int64_t K, float* dX, float* dW, float* db,
+                          float* ds, float* d_eta, void* workspace, size_t workspace_bytes, void* stream) {
+  SQ_TRY(check_k(K, sq::kMaxQuantK));
+  SQ_TRY(check_rows(M, "M"));
+  SQ_TRY(check_rows(N, "N"));
+  if (N % 8 != 0) return fail(SQ_ERR_ALIGN, "N=" + std::to_string(N) + " is not a multiple of 8");
+  if (!(alpha >= 0.0f && alpha <= 1.0f)) return fail(SQ_ERR_ARG, "alpha outside [0, 1]");
+  SQ_NONNULL(G);
+  SQ_NONNULL(X);
+  SQ_NONNULL(W);
+  SQ_NONNULL(s);
+  SQ_NONNULL(mx);
+  SQ_NONNULL(Xq);
+  SQ_NONNULL(x_scale);
+  SQ_NONNULL(Wq);
+  SQ_NONNULL(w_scale);
+  SQ_NONNULL(dX);
+  SQ_NONNULL(dW);
+  SQ_NONNULL(d_eta);
+  SQ_NONNULL(workspace);
+  if (db != nullptr && !aligned16(db)) return fail(SQ_ERR_ALIGN, "db is not 16-byte aligned");
+  if (ds != nullptr && !aligned16(ds)) return fail(SQ_ERR_ALIGN, "ds is not 16-byte aligned");
+  const size_t need = sq::ste_workspace_bytes(M, N, K);
+  if (workspace_bytes < need)
+    return fail(SQ_ERR_WORKSPACE, "workspace of " + std::to_string(workspace_bytes) + " bytes; " +
+                                      std::to_string(need) + " needed");
+  sq::DeviceInfo dev;
+  SQ_TRY(prologue(&dev));
+  sq::SteArgs a;
+  a.G = G;
+  a.X = X;
+  a.W = W;
+  a.s = s;
+  a.mx = mx;
+  a.alpha = alpha;
+  a.Xq = Xq;
+  a.x_scale = x_scale;
+  a.Wq = Wq;
+  a.w_scale = w_scale;
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.dX = dX;
+  a.dW = dW;
+  a.db = db;
+  a.ds = ds;
+  a.d_eta = d_eta;
+  a.ws = workspace;
+  a.ws_bytes = workspace_bytes;
+  const char* why = "launch";
+  cudaError_t e = sq::launch_ste_backward(a, static_cast<cudaStream_t>(stream), dev, &why);
+  if (e != cudaSuccess) return fail(SQ_ERR_CUDA, std::string("straight-through backward: ") + why + ": " +
+                                                     cudaGetErrorString(e));
+  return SQ_OK;
+}
+
 // ------------------------------------------------------------- int8 linear
 // SMs assumed when no device can be queried (a B200), so that sizes asked
 // before a device is current are the ones a B200 will want.

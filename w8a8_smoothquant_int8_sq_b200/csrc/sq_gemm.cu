@@ -695,16 +695,17 @@ cudaError_t read_device_status(uint32_t* flags, bool clear) {
     e = cudaMemcpyToSymbol(g_sq_device_status, &z, sizeof(z));
     if (e != cudaSuccess) return e;
   }
-  uint32_t q = 0, w = 0;
+  uint32_t q = 0, w = 0, b = 0;
   e = read_quant_status(&q, clear);
   if (e == cudaSuccess) e = read_weight_only_status(&w, clear);
+  if (e == cudaSuccess) e = read_ste_status(&b, clear);
   if (e != cudaSuccess) return e;
-  *flags = v | q | w;
+  *flags = v | q | w | b;
   return cudaSuccess;
 }
 
 bool make_tmap_2d(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int elem_bytes, int box_cols,
-                  int box_rows, int swizzle_bytes) {
+                  int box_rows, int swizzle_bytes, int64_t pitch_bytes) {
   EncodeTiledFn enc = get_encode_fn();
   if (enc == nullptr) return false;
   CUtensorMapDataType dt;
@@ -715,7 +716,8 @@ bool make_tmap_2d(CUtensorMap* map, const void* base, int64_t rows, int64_t cols
     default: return false;
   }
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
-  cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * static_cast<cuuint64_t>(elem_bytes)};
+  cuuint64_t strides[1] = {pitch_bytes > 0 ? static_cast<cuuint64_t>(pitch_bytes)
+                                           : static_cast<cuuint64_t>(cols) * static_cast<cuuint64_t>(elem_bytes)};
   cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows)};
   cuuint32_t estr[2] = {1, 1};
   CUtensorMapSwizzle sw;

@@ -61,12 +61,13 @@ struct DeviceInfo {
 cudaError_t current_device_info(DeviceInfo* out);
 
 // 2-D tensor map over a row-major [rows][cols] matrix of elem_bytes-wide
-// elements (row pitch cols * elem_bytes), box box_cols x box_rows, zero fill
-// outside the matrix; swizzle_bytes 0 (none), 32, 64 or 128 (the shared-memory
-// box's 16-byte units permuted as the hardware swizzle mode of that span).
-// False when the driver's encoder is unavailable or rejects the arguments.
+// elements (row pitch pitch_bytes, or cols * elem_bytes when 0), box
+// box_cols x box_rows, zero fill outside the matrix; swizzle_bytes 0 (none),
+// 32, 64 or 128 (the shared-memory box's 16-byte units permuted as the
+// hardware swizzle mode of that span).  False when the driver's encoder is
+// unavailable or rejects the arguments.
 bool make_tmap_2d(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int elem_bytes, int box_cols,
-                  int box_rows, int swizzle_bytes = 0);
+                  int box_rows, int swizzle_bytes = 0, int64_t pitch_bytes = 0);
 
 // Status word of the HBM-bound kernels (bit 0: a wait timed out).  Clearing a
 // set word also re-zeroes the no-allocation calibration scratch.
@@ -165,5 +166,30 @@ void debug_pipeline_stall(bool enable, unsigned long long timeout_ns);
 
 // Device status word (bit 0: pipeline wait timeout).
 cudaError_t read_device_status(uint32_t* flags, bool clear);
+
+// ---- straight-through backward of the learnable-alpha layer (sq_ste.cu)
+struct SteArgs {
+  const uint16_t* G;      // [M][N] bf16, dL/dY
+  const uint16_t* X;      // [M][K] bf16
+  const uint16_t* W;      // [N][K] bf16
+  const float* s;         // [K]
+  const float* mx;        // [K] running activation max
+  float alpha;
+  const int8_t* Xq;       // [M][K]
+  const float* x_scale;   // [M]
+  const int8_t* Wq;       // [N][K]
+  const float* w_scale;   // [N]
+  int64_t M, N, K;
+  float* dX;              // [M][K]
+  float* dW;              // [N][K]
+  float* db;              // [N] or null
+  float* ds;              // [K] or null
+  float* d_eta;           // [1]
+  void* ws;
+  size_t ws_bytes;
+};
+size_t ste_workspace_bytes(int64_t M, int64_t N, int64_t K);
+cudaError_t launch_ste_backward(const SteArgs& a, cudaStream_t st, const DeviceInfo& dev, const char** why);
+cudaError_t read_ste_status(uint32_t* flags, bool clear);
 
 }  // namespace sq
