@@ -67,8 +67,10 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default="proj", choices=sorted(workloads.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--path", default="smoothquant", choices=["smoothquant", "per-tensor"],
-                    help="per-tensor: the baseline W8A8 path (one scale per tensor) on the same workload")
+    ap.add_argument("--path", default="smoothquant", choices=["smoothquant", "per-tensor", "ste-train"],
+                    help="per-tensor: the baseline W8A8 path (one scale per tensor) on the same workload; "
+                         "ste-train: a learnable-alpha training step (s from the running max, forward, "
+                         "straight-through backward to X, W, bias and eta_alpha)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=50)
@@ -76,6 +78,12 @@ def parse_args():
     ap.add_argument("--settle-s", type=float, default=1.0,
                     help="untimed replays after warm-up until this much wall time has passed (clock sampling)")
     return ap.parse_args()
+
+
+def metric_for(path):
+    if path == "ste-train":
+        return "learnable-alpha W8A8 training step (forward + straight-through backward) tokens/s at 1 B200"
+    return METRIC
 
 
 def workload_config(wl, path="smoothquant"):
@@ -86,8 +94,11 @@ def workload_config(wl, path="smoothquant"):
         "M": wl.M, "N": wl.N, "K": wl.K, "R": wl.R,
         "l2": "flushed before every timed step (256 MiB write, then 512 MiB read); inputs smaller than L2",
     }
-    if path != "smoothquant":
+    if path == "per-tensor":
         c["workload"] = "per-tensor W8A8 baseline (one scale per tensor), " + c["workload"]
+    elif path == "ste-train":
+        c["workload"] = ("learnable-alpha training step (s from the running max of the calibration batch, "
+                         "forward, straight-through backward of a seeded bf16 dL/dY), " + c["workload"])
     return c
 
 
@@ -100,9 +111,10 @@ def peaks():
 
 
 def algorithmic_work(wl):
-    """Per call: (minimum HBM bytes per launch, int8 ops per launch or 0)."""
+    """Per call: (minimum HBM bytes per launch, tensor ops per launch or 0,
+    their operand type)."""
     M, N, K, R = wl.M, wl.N, wl.K, wl.R
-    return {
+    work = {
         "sq_calibrate": (2 * R * K + 2 * N * K + 8 * K, 0),
         "sq_prepare_weight": (3 * N * K + 4 * N + 4 * K, 0),
         "sq_quantize_act": (3 * M * K + 4 * M + 4 * K, 0),
@@ -110,7 +122,14 @@ def algorithmic_work(wl):
         # one scale per tensor: the data once in, the codes and the scale row out
         "sq_quantize_per_tensor(W)": (3 * N * K + 4 * N, 0),
         "sq_quantize_per_tensor(X)": (3 * M * K + 4 * M, 0),
+        # s from the running max alone: W read, mx read, s written
+        "sq_calibrate(mx)": (2 * N * K + 8 * K, 0),
+        # G, X, W, Xq, Wq and the scales in; dX, dW (fp32), db, ds out; two
+        # contractions of 2MNK each (counted once, whatever the kernel's split)
+        "sq_ste_backward": (2 * M * N + 7 * M * K + 7 * N * K + 8 * M + 12 * N + 12 * K, 4 * M * N * K),
     }
+    typ = {"sq_ste_backward": "bf16"}
+    return {n: (b, o, typ.get(n, "int8")) for n, (b, o) in work.items()}
 
 
 # Per-call kernel durations are spans over this many back-to-back launches.
@@ -222,6 +241,15 @@ class ClockSampler:
 # --------------------------------------------------------------- CPU oracle
 def oracle_step(inp, wl, rows=None, path="smoothquant"):
     from oracle import smoothquant as O
+    if path == "ste-train":
+        from oracle import ste_backward as STE
+        X = inp["X"] if rows is None else inp["X"][:rows]
+        G = inp["G"] if rows is None else inp["G"][:rows]
+        mx = O.column_max_abs(O.widen_bf16(inp["C"]))
+        s, _ = O.calibrate(inp["C"][:0], inp["W"], wl.alpha_f32, mx_prev=mx)
+        Wq, ws = O.fold_and_quantize_weight(inp["W"], s)
+        Y, _, _, _ = O.forward(X, s, Wq, ws, inp["bias"])
+        return Y, STE.ste_backward(G, X, inp["W"], mx, wl.alpha_f32)
     if path == "per-tensor":
         from oracle import per_tensor as PT
         X = inp["X"] if rows is None else inp["X"][:rows]
@@ -244,9 +272,16 @@ def cpu_threads():
     return len(os.sched_getaffinity(0))
 
 
+def train_gradient(wl):
+    """Seeded synthetic dL/dY [M, N] (bf16 bits) for the training step."""
+    return workloads.random_bf16((wl.M, wl.N), seed=1000 * wl.index + 9, scale=1e-3)
+
+
 def cpu_oracle_rate(wl, seconds, max_steps=None, path="smoothquant"):
     """Tokens/s of the oracle on whole steps, run until `seconds` pass."""
     inp = workloads.make_inputs(wl)
+    if path == "ste-train":
+        inp["G"] = train_gradient(wl)
     oracle_step(inp, wl, path=path)  # warm (page-in, BLAS threads)
     n, t0 = 0, time.perf_counter()
     while True:
@@ -262,21 +297,23 @@ def run_reference(args, wl, rank, world):
     if rank != 0:
         return
     inp = workloads.make_inputs(wl)
+    if args.path == "ste-train":
+        inp["G"] = train_gradient(wl)
     for _ in range(args.warmup):
-        oracle_step(inp, wl)
+        oracle_step(inp, wl, path=args.path)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        oracle_step(inp, wl)
+        oracle_step(inp, wl, path=args.path)
     el = time.perf_counter() - t0
     v = wl.M * args.steps / el
     cores = cpu_threads()
     line = {
-        "impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus,
+        "impl": "reference", "metric": metric_for(args.path), "value": v, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * el / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64+fp32 (numpy)",
-        "data": "synthetic", "config": workload_config(wl),
+        "data": "synthetic", "config": workload_config(wl, args.path),
         "cpu_baseline": {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
-                         "sample": f"{args.steps} whole {wl.name} steps (calibrate, fold+quantise W, forward)"},
+                         "sample": f"{args.steps} whole {wl.name} steps ({args.path} path of the oracle)"},
         "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -289,10 +326,10 @@ def kernel_report(wl, names, per_call, per_call_single, launches_per_call):
     work = algorithmic_work(wl)
     kernels = {}
     for n in names:
-        nbytes, ops = work[n]
+        nbytes, ops, op_type = work[n]
         ms = per_call[n]
         sustained = ms >= SUSTAINED_AFTER_MS and bf16_tf_sus is not None
-        int8_peak_tops = (bf16_tf_sus if sustained else bf16_tf) * INT8_OVER_BF16
+        int8_peak_tops = (bf16_tf_sus if sustained else bf16_tf) * (INT8_OVER_BF16 if op_type == "int8" else 1.0)
         # the bound is whichever roofline takes longer for this call's work
         t_hbm = nbytes / (hbm_gbs * 1e9)
         t_tensor = ops / (int8_peak_tops * 1e12)
@@ -307,6 +344,8 @@ def kernel_report(wl, names, per_call, per_call_single, launches_per_call):
                           "achieved_tops": ach,
                           "int8_peak_tops": int8_peak_tops, "frac_of_int8_peak": ach / int8_peak_tops,
                           "peak": "sustained" if sustained else "burst", "launches": launches_per_call[n]}
+            if op_type != "int8":
+                kernels[n]["operands"] = op_type
     dom = max(names, key=lambda n: per_call[n])
     kd = kernels[dom]
     if kd["bound"] == "hbm":
@@ -316,7 +355,8 @@ def kernel_report(wl, names, per_call, per_call_single, launches_per_call):
     else:
         roof = {"bound": "tensor", "achieved": kd["achieved_tops"], "peak": kd["int8_peak_tops"], "unit": "TFLOP/s",
                 "frac": kd["achieved_tops"] / kd["int8_peak_tops"]}
-        roof["peak_source"] = f"{peak_kind} cuBLAS bf16 {kd['peak']} x2 (nominal dense int8/bf16 ratio)"
+        roof["peak_source"] = (f"{peak_kind} cuBLAS bf16 {kd['peak']}" if kd.get("operands") == "bf16" else
+                               f"{peak_kind} cuBLAS bf16 {kd['peak']} x2 (nominal dense int8/bf16 ratio)")
     roof["kernel"] = dom
     roof["traffic"] = ncu_traffic(dom, wl.name)
     return kernels, roof
@@ -349,7 +389,31 @@ def run_ours(args, wl, rank, world, local_rank):
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     flush_read = torch.ones(FLUSH_READ_BYTES // 4, dtype=torch.int32, device=dev)
 
-    if args.path == "per-tensor":
+    if args.path == "ste-train":
+        # the training step of the learnable-alpha layer: s recomputed from the
+        # running activation max (taken once from the calibration batch) and
+        # the weight, the forward, and the straight-through backward
+        G = d(train_gradient(wl))
+        mx = torch.empty(K, dtype=torch.float32, device=dev).zero_()
+        sq.sq_calibrate(C, W, wl.alpha_f32, s=s, mx_inout=mx, workspace=ws_cal)
+        dXg = torch.empty(M, K, dtype=torch.float32, device=dev)
+        dWg = torch.empty(N, K, dtype=torch.float32, device=dev)
+        dbg = torch.empty(N, dtype=torch.float32, device=dev) if b is not None else None
+        dsg = torch.empty(K, dtype=torch.float32, device=dev)
+        d_eta = torch.empty(1, dtype=torch.float32, device=dev)
+        ws_bwd = torch.empty(sq.sq_ste_backward_workspace_bytes(M, N, K), dtype=torch.uint8, device=dev)
+        calls = {
+            "sq_calibrate(mx)": lambda: sq.sq_calibrate(None, W, wl.alpha_f32, s=s, mx_inout=mx, workspace=ws_cal),
+            "sq_prepare_weight": lambda: sq.sq_prepare_weight(W, s, Wq=Wq, w_scale=w_scale),
+            "sq_quantize_act": lambda: sq.sq_quantize_act(X, s, Xq=Xq, x_scale=x_scale),
+            "sq_linear": lambda: sq.sq_linear(Xq, x_scale, Wq, w_scale, b, Y=Y, workspace=ws_lin),
+            "sq_ste_backward": lambda: sq.sq_ste_backward(G, X, W, s, mx, wl.alpha_f32, Xq, x_scale, Wq, w_scale,
+                                                          with_db=b is not None, dX=dXg, dW=dWg, db=dbg, ds=dsg,
+                                                          d_eta=d_eta, workspace=ws_bwd),
+        }
+        launches_per_call = {"sq_calibrate(mx)": 2, "sq_prepare_weight": 1, "sq_quantize_act": 1, "sq_linear": 1,
+                             "sq_ste_backward": 7}
+    elif args.path == "per-tensor":
         ws_pt = torch.empty(sq.sq_quantize_per_tensor_workspace_bytes(), dtype=torch.uint8, device=dev)
         ws_pt2 = torch.empty_like(ws_pt)
         calls = {
@@ -478,6 +542,11 @@ def run_ours(args, wl, rank, world, local_rank):
         hY = torch.empty(M, N, dtype=torch.bfloat16).pin_memory()
         dC, dW, dX = torch.empty_like(C), torch.empty_like(W), torch.empty_like(X)
         db = torch.empty_like(b) if b is not None else None
+        if args.path == "ste-train":
+            hG = torch.from_numpy(train_gradient(wl).view(np.int16)).view(torch.bfloat16).pin_memory()
+            hmx = mx.cpu().pin_memory()
+            h_eta = torch.empty(1, dtype=torch.float32).pin_memory()
+            dG, dmx = torch.empty_like(G), torch.empty_like(mx)
 
         def e2e_step():
             dC.copy_(hC, non_blocking=True)
@@ -485,7 +554,18 @@ def run_ours(args, wl, rank, world, local_rank):
             dX.copy_(hX, non_blocking=True)
             if db is not None:
                 db.copy_(hb, non_blocking=True)
-            if args.path == "per-tensor":
+            if args.path == "ste-train":
+                dG.copy_(hG, non_blocking=True)
+                dmx.copy_(hmx, non_blocking=True)
+                sq.sq_calibrate(None, dW, wl.alpha_f32, s=s, mx_inout=dmx, workspace=ws_cal)
+                sq.sq_prepare_weight(dW, s, Wq=Wq, w_scale=w_scale)
+                sq.sq_quantize_act(dX, s, Xq=Xq, x_scale=x_scale)
+                sq.sq_linear(Xq, x_scale, Wq, w_scale, db, Y=Y, workspace=ws_lin)
+                sq.sq_ste_backward(dG, dX, dW, s, dmx, wl.alpha_f32, Xq, x_scale, Wq, w_scale,
+                                   with_db=db is not None, dX=dXg, dW=dWg, db=dbg, ds=dsg, d_eta=d_eta,
+                                   workspace=ws_bwd)
+                h_eta.copy_(d_eta, non_blocking=True)
+            elif args.path == "per-tensor":
                 sq.sq_quantize_per_tensor(dW, Aq=Wq, scale_rows=w_scale, workspace=ws_pt)
                 sq.sq_quantize_per_tensor(dX, Aq=Xq, scale_rows=x_scale, workspace=ws_pt2)
                 sq.sq_linear(Xq, x_scale, Wq, w_scale, db, Y=Y, workspace=ws_lin)
@@ -507,11 +587,20 @@ def run_ours(args, wl, rank, world, local_rank):
         e1.record(stream)
         torch.cuda.synchronize()
         e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, world, dev)
-        h2d = sum(t.numel() * t.element_size() for t in (hC, hW, hX) + ((hb,) if hb is not None else ()))
-        e2e = {"value": whole_job_rate(wl.M, world, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
-               "d2h_bytes_per_step": hY.numel() * hY.element_size(), "ms_per_step": e2e_ms,
-               "call": ("sq_quantize_per_tensor(W) + sq_quantize_per_tensor(X) + sq_linear"
-                        if args.path == "per-tensor" else "sq_calibrate + sq_prepare_weight + sq_forward")}
+        if args.path == "ste-train":
+            ins = (hW, hX, hG, hmx) + ((hb,) if hb is not None else ())
+            outs = (hY, h_eta)
+            call = ("sq_calibrate(mx) + sq_prepare_weight + sq_quantize_act + sq_linear + sq_ste_backward, "
+                    "Y and d eta read back")
+        else:
+            ins = (hC, hW, hX) + ((hb,) if hb is not None else ())
+            outs = (hY,)
+            call = ("sq_quantize_per_tensor(W) + sq_quantize_per_tensor(X) + sq_linear"
+                    if args.path == "per-tensor" else "sq_calibrate + sq_prepare_weight + sq_forward")
+        e2e = {"value": whole_job_rate(wl.M, world, e2e_ms), "unit": UNIT,
+               "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in ins),
+               "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in outs), "ms_per_step": e2e_ms,
+               "call": call}
 
     if rank != 0:
         return
@@ -521,14 +610,15 @@ def run_ours(args, wl, rank, world, local_rank):
     cpu = None
     if not args.no_cpu_baseline and world == 1:
         v, n, el = cpu_oracle_rate(wl, args.cpu_seconds, path=args.path)
+        what = {"per-tensor": "quantise W and X per tensor, product",
+                "ste-train": "s from the running max, fold+quantise W, forward, straight-through backward"}
         cpu = {"value": v, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
                "sample": f"{n} whole {wl.name} steps in {el:.1f} s ("
-                         + ("quantise W and X per tensor, product" if args.path == "per-tensor"
-                            else "calibrate, fold+quantise W, forward") + ")"}
+                         + what.get(args.path, "calibrate, fold+quantise W, forward") + ")"}
 
     value = whole_job_rate(wl.M, world, step_ms)
     line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "metric": metric_for(args.path), "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "int8", "data": "synthetic", "config": workload_config(wl, args.path),
         "tops_per_step": 2.0 * wl.M * wl.N * wl.K * world / (step_ms * 1e-3) / 1e12,
