@@ -8,7 +8,7 @@ kernels' arithmetic allows.  The two products take the codes as exact bf16
 operands and G times a scale split into two bf16 halves (2^-16 relative, after
 the scale's own fp32 product), accumulated in fp32 over 2C products (at most
 2C * 2^-22 of the sum of absolute products, a worst-case bound that allows
-round-toward-zero accumulation), then one fp32 division or product.
+round-toward-zero accumulation), then one fp32 product (dW) or a product with the rounded reciprocal of s (dX).
 ds_k s_k is formed from the quantisation errors, so its bound is that
 relative error times sum |dWs| |W s - Wdq| + sum |dXs| |X/s - Xdq|, plus the
 fp32 rounding of W s and X / s and the fp32 sums of N and M such terms.
@@ -73,7 +73,8 @@ def compare(G, X, W, mx, alpha, r, dX, dW, db, ds, d_eta, label, with_db=True):
         worst[name] = float(ratio.max()) if ratio.size else 0.0
         assert worst[name] <= 1.0, f"{label}: {name} error {worst[name]:.3f} of the bound"
 
-    check("dX", dX, r["dX"], gx * e["aXs"] / s64[None, :] + 2.0 ** -24 * np.abs(r["dX"]))
+    # dX = dXs * RN(1/s): two roundings after the product
+    check("dX", dX, r["dX"], gx * e["aXs"] / s64[None, :] * (1 + 2.0 ** -22) + 2.0 ** -22 * np.abs(r["dX"]))
     check("dW", dW, r["dW"], gw * e["aWs"] * s64[None, :] + 2.0 ** -24 * np.abs(r["dW"]))
     if with_db:
         Ga = np.abs(O.widen_bf16(G).astype(np.float64)).sum(axis=0)
@@ -87,7 +88,8 @@ def compare(G, X, W, mx, alpha, r, dX, dW, db, ds, d_eta, label, with_db=True):
     round_terms = (e["aWs"] * np.abs(Wv) * s64[None, :]).sum(axis=0) + (e["aXs"] * np.abs(Xv) / s64[None, :]).sum(axis=0)
     aT_w = (e["aWs"] * np.abs(e["dW_q"])).sum(axis=0)
     aT_x = (e["aXs"] * np.abs(e["dX_q"])).sum(axis=0)
-    bT = gw * aT_w + gx * aT_x + 2.0 ** -23 * round_terms + (N + M + 4) * 2.0 ** -24 * (aT_w + aT_x)
+    # (X/s is formed as X * RN(1/s): two roundings, hence 2^-22 on the X terms)
+    bT = gw * aT_w + gx * aT_x + 2.0 ** -22 * round_terms + (N + M + 4) * 2.0 ** -24 * (aT_w + aT_x)
     check("ds", ds, r["ds"], bT / s64 + 2.0 ** -23 * np.abs(r["ds"]))
     raw, mxc, mwc = STE.raw_smoothing(mx, r["mw"], alpha)
     Ls = np.log(mxc) + np.log(mwc)

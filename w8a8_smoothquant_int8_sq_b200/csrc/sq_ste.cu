@@ -58,17 +58,25 @@ constexpr int kSBN = 128;          // GEMM tile columns (tokens or output rows) 
 constexpr int kSBK = 64;           // contraction elements per stage (128 bytes of bf16)
 constexpr int kSUmmaK = 16;        // contraction per tcgen05.mma kind::f16
 constexpr int kSStages = 4;
-constexpr int kSThreads = 192;
+constexpr int kSEpiWarps = 8;     // two per TMEM lane quarter, each taking half of the tile's columns
+constexpr int kSThreads = 64 + 32 * kSEpiWarps;
 constexpr int kSABytes = kSBM * kSBK * 2;
 constexpr int kSBBytes = kSBN * kSBK * 2;  // one half (hi or lo)
 constexpr int kSStageBytes = kSABytes + 2 * kSBBytes;
 constexpr int kSBarOffset = kSStages * kSStageBytes;
 constexpr int kSNumBars = 2 * kSStages + 4 + 1;
-constexpr int kSEpiOffset = (kSBarOffset + kSNumBars * 8 + 15) / 16 * 16;
-constexpr int kSEpiBytes = 4 * kSBN * 4;
-constexpr int kSMiscOffset = kSEpiOffset + kSEpiBytes;
+// per epilogue warp: a 32 x 32 block of src (bf16, 80-byte rows) and of q
+// (int8, 48-byte rows) staged for the transposed read, and the block's 32
+// column scales; the row pitches keep the 16-byte stores of 8 consecutive
+// lanes on distinct bank groups
+constexpr int kStgSrcPitch = 80;
+constexpr int kStgQPitch = 48;
+constexpr int kStgBytes = 32 * kStgSrcPitch + 32 * kStgQPitch + 32 * 4;
+constexpr int kSStgOffset = (kSBarOffset + kSNumBars * 8 + 15) / 16 * 16;
+constexpr int kSMiscOffset = kSStgOffset + kSEpiWarps * kStgBytes;
 constexpr int kSAlloc = kSMiscOffset + 16 + 1024;
-constexpr uint32_t kSTmemCols = 2 * kSBN;
+constexpr int kSAccCols = 2 * kSBN;         // one accumulator: A Bh^T in columns [0, 128), A Bl^T in [128, 256)
+constexpr uint32_t kSTmemCols = 2 * kSAccCols;
 constexpr unsigned long long kSWaitNs = 2000000000ull;
 constexpr int kEpiDX = 0;
 constexpr int kEpiDW = 1;
@@ -87,9 +95,11 @@ __device__ __forceinline__ void store4(uint16_t* dst, int n, uint16_t v0, uint16
   }
 }
 
-__global__ void ste_init_kernel(float* tx, float* tw, unsigned int* mwbits, int K, float* db, int N) {
+__global__ void ste_init_kernel(float* tx, float* tw, unsigned int* mwbits, int K, float* db, int N,
+                                unsigned int* counter) {
   griddep_wait();
   griddep_launch_dependents();
+  if (blockIdx.x == 0 && threadIdx.x == 0) *counter = 0u;
   const int stride = gridDim.x * blockDim.x;
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < K; i += stride) {
     tx[i] = 0.0f;
@@ -222,13 +232,17 @@ __device__ __forceinline__ void ste_flag_timeout(volatile int* abort_flag) {
 // D[i][j] = sum_c A[i][c] (Bh[j][c] + Bl[j][c]) with A [I][C], Bh and Bl
 // [J][C] bf16 (row-major, loaded by TMA in 128 x 64-element boxes with the
 // 128-byte swizzle), one CTA per SM persistent over 128 x 128 tiles: warp 0
-// loads, warp 1 issues tcgen05.mma kind::f16 (A Bh, then A Bl) into one of two
-// TMEM accumulators, warps 2..5 run the epilogue of EPI on TMEM lanes (rows i)
-// 32 (warp % 4) .. + 31.
+// loads (and prefetches the tile's src and q blocks into L2 for the
+// epilogue), warp 1 issues tcgen05.mma kind::f16 with N = 256 -- the Bh and
+// Bl boxes sit back to back in shared memory and form one 256-row operand, so
+// one MMA yields A Bh^T and A Bl^T side by side -- into one of two TMEM
+// accumulators, warps 2..5 run the epilogue of EPI on TMEM lanes (rows i)
+// 32 (warp % 4) .. + 31, adding the two halves.
 template <int EPI>
 __global__ void __launch_bounds__(kSThreads, 1)
     ste_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmBh,
-                    const __grid_constant__ CUtensorMap tmBl, const SteGemmParams p) {
+                    const __grid_constant__ CUtensorMap tmBl, const __grid_constant__ CUtensorMap tmSrc,
+                    const __grid_constant__ CUtensorMap tmQ, const SteGemmParams p) {
   extern __shared__ uint8_t ste_smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(ste_smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kSBarOffset);
@@ -249,7 +263,7 @@ __global__ void __launch_bounds__(kSThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&tfull[i], 1);
-      mbar_init(&tempty[i], 4);
+      mbar_init(&tempty[i], kSEpiWarps);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -260,6 +274,8 @@ __global__ void __launch_bounds__(kSThreads, 1)
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmBh);
     tma_prefetch_desc(&tmBl);
+    tma_prefetch_desc(&tmSrc);
+    tma_prefetch_desc(&tmQ);
   }
   if (warp == 1) {
     __syncwarp();
@@ -288,6 +304,9 @@ __global__ void __launch_bounds__(kSThreads, 1)
       for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
         const int i_blk = tile % p.num_i_blocks;
         const int j_blk = tile / p.num_i_blocks;
+        // the epilogue's src and q blocks of this tile, into L2
+        tma_prefetch_l2_2d(&tmSrc, i_blk * kSBM, j_blk * kSBN);
+        tma_prefetch_l2_2d(&tmQ, i_blk * kSBM, j_blk * kSBN);
         for (int kb = 0; kb < nk; ++kb) {
           if (*abort_flag || !mbar_wait_bounded(&empty[stage], phase ^ 1u, kSWaitNs)) {
             if (!*abort_flag) ste_flag_timeout(abort_flag);
@@ -316,7 +335,7 @@ __global__ void __launch_bounds__(kSThreads, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16(kSBM, kSBN);
+      constexpr uint32_t idesc = idesc_bf16(kSBM, 2 * kSBN);
       int stage = 0;
       uint32_t phase = 0;
       int it = 0;
@@ -329,7 +348,7 @@ __global__ void __launch_bounds__(kSThreads, 1)
           break;
         }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kSBN);
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kSAccCols);
         for (int kb = 0; kb < nk; ++kb) {
           if (*abort_flag || !mbar_wait_bounded(&full[stage], phase, kSWaitNs)) {
             if (!*abort_flag) ste_flag_timeout(abort_flag);
@@ -340,14 +359,11 @@ __global__ void __launch_bounds__(kSThreads, 1)
           const uint32_t sa = smem_u32(smem + stage * kSStageBytes);
           const uint32_t sb = sa + kSABytes;
           const uint64_t adesc = smem_desc_k_sw128(sa);
-          const uint64_t bhdesc = smem_desc_k_sw128(sb);
-          const uint64_t bldesc = smem_desc_k_sw128(sb + kSBBytes);
+          const uint64_t bdesc = smem_desc_k_sw128(sb);  // Bh rows 0..127, Bl rows 128..255
 #pragma unroll
-          for (int kk = 0; kk < kSBK / kSUmmaK; ++kk) {  // 32 bytes per step inside the swizzle atom
-            mma_bf16(d_tmem, adesc + static_cast<uint64_t>(kk * 2), bhdesc + static_cast<uint64_t>(kk * 2), idesc,
+          for (int kk = 0; kk < kSBK / kSUmmaK; ++kk)  // 32 bytes per step inside the swizzle atom
+            mma_bf16(d_tmem, adesc + static_cast<uint64_t>(kk * 2), bdesc + static_cast<uint64_t>(kk * 2), idesc,
                      (kb != 0 || kk != 0) ? 1u : 0u);
-            mma_bf16(d_tmem, adesc + static_cast<uint64_t>(kk * 2), bldesc + static_cast<uint64_t>(kk * 2), idesc, 1u);
-          }
           mma_commit(&empty[stage]);
           if (++stage == kSStages) {
             stage = 0;
@@ -361,23 +377,57 @@ __global__ void __launch_bounds__(kSThreads, 1)
       (void)mbar_wait_bounded(drain, 0, kSWaitNs);
     }
   } else {
-    const int quarter = warp & 3;
-    float* ep_qs = reinterpret_cast<float*>(smem + kSEpiOffset) + (warp - 2) * kSBN;
+    const int quarter = warp & 3;          // TMEM lanes 32 quarter .. + 31
+    const int ew = warp - 2;               // epilogue warp 0 .. kSEpiWarps - 1
+    const int half = ew / 4;               // columns [64 half, 64 half + 64) of each tile
+    uint8_t* stg = smem + kSStgOffset + ew * kStgBytes;
+    uint16_t* stg_src = reinterpret_cast<uint16_t*>(stg);                 // [32 j][kStgSrcPitch bytes]
+    int8_t* stg_q = reinterpret_cast<int8_t*>(stg + 32 * kStgSrcPitch);  // [32 j][kStgQPitch bytes]
+    float* stg_qs = reinterpret_cast<float*>(stg + 32 * (kStgSrcPitch + kStgQPitch));  // [32 j]
+    constexpr int kChunks = kSBN / 32 / 2;  // 32-column chunks per warp and tile
     int it = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
       const int acc = it & 1;
       const uint32_t acc_phase = (it >> 1) & 1;
       const int i_blk = tile % p.num_i_blocks;
       const int j_blk = tile / p.num_i_blocks;
-      const int i = i_blk * kSBM + quarter * 32 + lane;
+      const int i0 = i_blk * kSBM + quarter * 32;  // this warp's first row
+      const int i = i0 + lane;
       const bool row_ok = i < p.I;
+      // rows of this warp that exist: 0, 16 or 32 (I % 16 == 0, i0 % 32 == 0)
+      const int ni = max(0, min(32, p.I - i0));
       const float s_i = row_ok ? __ldg(p.s + i) : 1.0f;
-      __syncwarp();
-      for (int c = lane; c < kSBN; c += 32) {
-        const int j = j_blk * kSBN + c;
-        ep_qs[c] = j < p.J ? __ldg(p.qscale + j) : 0.0f;
+      const float rs_i = __frcp_rn(s_i);
+      // this warp's 32 x 64 block of src and q and its column scales, fetched
+      // before the accumulator is ready so that the loads overlap the tile's
+      // MMAs: lane l holds row j_blk * 128 + 64 half + 32 cc + l, columns
+      // i0 .. i0 + ni - 1
+      uint4 ra[kChunks][4], rb[kChunks][2];
+      float rq[kChunks];
+#pragma unroll
+      for (int cc = 0; cc < kChunks; ++cc) {
+        const int j = j_blk * kSBN + half * 64 + cc * 32 + lane;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) ra[cc][u] = make_uint4(0u, 0u, 0u, 0u);
+        rb[cc][0] = rb[cc][1] = make_uint4(0u, 0u, 0u, 0u);
+        rq[cc] = 0.0f;
+        if (j < p.J) {
+          rq[cc] = __ldg(p.qscale + j);
+          if (ni > 0) {
+            const int64_t e = static_cast<int64_t>(j) * p.I + i0;
+            const uint4* sv = reinterpret_cast<const uint4*>(p.src + e);
+            const uint4* qv = reinterpret_cast<const uint4*>(p.q + e);
+            ra[cc][0] = sv[0];
+            ra[cc][1] = sv[1];
+            rb[cc][0] = qv[0];
+            if (ni > 16) {
+              ra[cc][2] = sv[2];
+              ra[cc][3] = sv[3];
+              rb[cc][1] = qv[1];
+            }
+          }
+        }
       }
-      __syncwarp();
       const bool mine = !*abort_flag && mbar_wait_bounded(&tfull[acc], acc_phase, kSWaitNs);
       if (!__all_sync(0xFFFFFFFFu, mine)) {
         if (lane == 0 && !*abort_flag) ste_flag_timeout(abort_flag);
@@ -385,43 +435,50 @@ __global__ void __launch_bounds__(kSThreads, 1)
       }
       tc_fence_after();
       const uint32_t t_base =
-          tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * kSBN);
+          tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * kSAccCols);
       float tsum = 0.0f;
       uint32_t mbits = 0u;
-#pragma unroll 1
-      for (int c0 = 0; c0 < kSBN; c0 += 32) {
-        uint32_t r[32];
-        tmem_ld_32cols(t_base + static_cast<uint32_t>(c0), r);
-        tmem_ld_wait();
-        const int j0 = j_blk * kSBN + c0;
-        if (j0 >= p.J) continue;  // warp-uniform
-        const int jn = min(32, p.J - j0);
-        if (row_ok) {
-          uint16_t sv[32];
-          int8_t qv[32];
 #pragma unroll
-          for (int jj = 0; jj < 32; ++jj) {
-            const int64_t e = static_cast<int64_t>(j0 + jj) * p.I + i;
-            sv[jj] = jj < jn ? p.src[e] : static_cast<uint16_t>(0);
-            qv[jj] = jj < jn ? p.q[e] : static_cast<int8_t>(0);
-          }
+      for (int cc = 0; cc < kChunks; ++cc) {
+        const int c0 = half * 64 + cc * 32;
+        uint32_t r[32], rl[32];
+        tmem_ld_32cols(t_base + static_cast<uint32_t>(c0), r);           // A Bh^T
+        tmem_ld_32cols(t_base + static_cast<uint32_t>(kSBN + c0), rl);   // A Bl^T
+        const int j0 = j_blk * kSBN + c0;
+        const int jn = min(32, p.J - j0);
+        __syncwarp();  // the previous chunk's reads of the staging area are done
+        {
+          uint4* ds = reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(stg_src) + lane * kStgSrcPitch);
+#pragma unroll
+          for (int u = 0; u < 4; ++u) ds[u] = ra[cc][u];
+          uint4* dq = reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(stg_q) + lane * kStgQPitch);
+          dq[0] = rb[cc][0];
+          dq[1] = rb[cc][1];
+          stg_qs[lane] = rq[cc];
+        }
+        tmem_ld_wait();
+        __syncwarp();
+        if (j0 < p.J && row_ok) {
+          float* o = p.out + static_cast<int64_t>(j0) * p.I + i;
 #pragma unroll
           for (int jj = 0; jj < 32; ++jj) {
             if (jj >= jn) break;
-            const float v = __uint_as_float(r[jj]);
-            const float x = __uint_as_float(static_cast<uint32_t>(sv[jj]) << 16);
-            const float dq = static_cast<float>(qv[jj]);
-            float* o = p.out + static_cast<int64_t>(j0 + jj) * p.I + i;
+            const float v = __fadd_rn(__uint_as_float(r[jj]), __uint_as_float(rl[jj]));
+            const uint16_t xb = *reinterpret_cast<const uint16_t*>(reinterpret_cast<const uint8_t*>(stg_src) +
+                                                                  jj * kStgSrcPitch + lane * 2);
+            const float x = __uint_as_float(static_cast<uint32_t>(xb) << 16);
+            const float dq = static_cast<float>(stg_q[jj * kStgQPitch + lane]);
             if (EPI == kEpiDX) {
-              *o = __fdiv_rn(v, s_i);
-              const float err = __fmaf_rn(-dq, ep_qs[c0 + jj], __fdiv_rn(x, s_i));  // X/s - Xdq
+              *o = __fmul_rn(v, rs_i);                                          // dXs / s
+              const float err = __fmaf_rn(-dq, stg_qs[jj], __fmul_rn(x, rs_i));  // X/s - Xdq
               tsum = __fmaf_rn(v, err, tsum);
             } else {
-              *o = __fmul_rn(v, s_i);
-              const float err = __fmaf_rn(-dq, ep_qs[c0 + jj], __fmul_rn(x, s_i));  // W*s - Wdq
+              *o = __fmul_rn(v, s_i);                                           // dWs * s
+              const float err = __fmaf_rn(-dq, stg_qs[jj], __fmul_rn(x, s_i));   // W*s - Wdq
               tsum = __fmaf_rn(v, err, tsum);
-              mbits = max(mbits, static_cast<uint32_t>(sv[jj] & 0x7FFFu) << 16);
+              mbits = max(mbits, static_cast<uint32_t>(xb & 0x7FFFu) << 16);
             }
+            o += p.I;
           }
         }
       }
@@ -444,36 +501,49 @@ __global__ void __launch_bounds__(kSThreads, 1)
 
 // ds_k = T_k / s_k with T_k = tw_k - tx_k, and d eta = alpha (1 - alpha)
 // sum_k ds_k raw_k (ln mx_k + ln mw_k) over the channels whose raw_k =
-// mx_k^alpha / mw_k^(1-alpha) (both clamped at 1e-8) is not below 1e-8.  One
-// block; float64.
-constexpr int kFinishThreads = 1024;
+// mx_k^alpha / mw_k^(1-alpha) (both clamped at 1e-8) is not below 1e-8.
+// float64; one channel per thread, block sums in `partial`, and the last
+// block to finish (arrival counter, zeroed by ste_init_kernel) adds the block
+// sums in block order and writes d eta.
+constexpr int kFinishThreads = 256;
 __global__ void __launch_bounds__(kFinishThreads) ste_finish_kernel(const float* tx, const float* tw,
                                                                      const unsigned int* mwbits, const float* mx,
                                                                      const float* s, float alpha, int K,
-                                                                     float* ds_out, float* d_eta) {
+                                                                     float* ds_out, double* partial,
+                                                                     unsigned int* counter, float* d_eta) {
   __shared__ double part[kFinishThreads / 32];
+  __shared__ bool last;
   griddep_wait();
   griddep_launch_dependents();
   const double a = static_cast<double>(alpha);
   const double floor_v = static_cast<double>(kClampFloor);
   double acc = 0.0;
-  for (int k = threadIdx.x; k < K; k += kFinishThreads) {
+  const int k = blockIdx.x * kFinishThreads + threadIdx.x;
+  if (k < K) {
     const double mxc = fmax(static_cast<double>(mx[k]), floor_v);
     const double mwc = fmax(static_cast<double>(__uint_as_float(mwbits[k])), floor_v);
     const double raw = pow(mxc, a) / pow(mwc, 1.0 - a);
     const double ds = (static_cast<double>(tw[k]) - static_cast<double>(tx[k])) / static_cast<double>(s[k]);
     if (ds_out != nullptr) ds_out[k] = static_cast<float>(ds);
-    if (raw >= floor_v) acc += ds * raw * (log(mxc) + log(mwc));
+    if (raw >= floor_v) acc = ds * raw * (log(mxc) + log(mwc));
   }
 #pragma unroll
   for (int o = 16; o >= 1; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
   if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = acc;
   __syncthreads();
-  if (threadIdx.x < 32) {
-    double v = part[threadIdx.x];
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
-    if (threadIdx.x == 0) d_eta[0] = static_cast<float>(a * (1.0 - a) * v);
+  if (threadIdx.x == 0) {
+    double v = 0.0;
+    for (int w = 0; w < kFinishThreads / 32; ++w) v += part[w];
+    partial[blockIdx.x] = v;
+    __threadfence();
+    last = atomicAdd(counter, 1u) == gridDim.x - 1;
+  }
+  __syncthreads();
+  if (last && threadIdx.x == 0) {
+    __threadfence();
+    double v = 0.0;
+    for (unsigned b = 0; b < gridDim.x; ++b) v += *(volatile double*)(partial + b);
+    d_eta[0] = static_cast<float>(a * (1.0 - a) * v);
   }
 }
 
@@ -481,7 +551,7 @@ int64_t round_up64(int64_t v, int64_t a) { return (v + a - 1) / a * a; }
 
 struct SteLayout {
   int64_t Mp;
-  size_t wt, xt, gh, gl, gth, gtl, tx, tw, mw, total;
+  size_t wt, xt, gh, gl, gth, gtl, tx, tw, mw, fin, total;
 };
 
 SteLayout ste_layout(int64_t M, int64_t N, int64_t K) {
@@ -502,6 +572,7 @@ SteLayout ste_layout(int64_t M, int64_t N, int64_t K) {
   L.tx = take(static_cast<size_t>(K) * 4);
   L.tw = take(static_cast<size_t>(K) * 4);
   L.mw = take(static_cast<size_t>(K) * 4);
+  L.fin = take(static_cast<size_t>((K + kFinishThreads - 1) / kFinishThreads) * 8 + 16);  // block sums, counter
   L.total = off;
   return L;
 }
@@ -510,10 +581,12 @@ template <int EPI>
 cudaError_t run_ste_gemm(const void* A, const void* Bh, const void* Bl, int64_t I, int64_t J, int64_t C,
                          int64_t pitch_elems, const SteGemmParams& base, cudaStream_t st, const DeviceInfo& dev,
                          const char** why) {
-  CUtensorMap tmA, tmBh, tmBl;
+  CUtensorMap tmA, tmBh, tmBl, tmSrc, tmQ;
   if (!make_tmap_2d(&tmA, A, I, C, 2, kSBK, kSBM, 128, pitch_elems * 2) ||
       !make_tmap_2d(&tmBh, Bh, J, C, 2, kSBK, kSBN, 128, pitch_elems * 2) ||
-      !make_tmap_2d(&tmBl, Bl, J, C, 2, kSBK, kSBN, 128, pitch_elems * 2)) {
+      !make_tmap_2d(&tmBl, Bl, J, C, 2, kSBK, kSBN, 128, pitch_elems * 2) ||
+      !make_tmap_2d(&tmSrc, base.src, J, I, 2, kSBM, kSBN, 0) ||
+      !make_tmap_2d(&tmQ, base.q, J, I, 1, kSBM, kSBN, 0)) {
     *why = "cuTensorMapEncodeTiled failed or unavailable";
     return cudaErrorInvalidValue;
   }
@@ -533,7 +606,7 @@ cudaError_t run_ste_gemm(const void* A, const void* Bh, const void* Bl, int64_t 
   }
   const int tiles = p.num_i_blocks * p.num_j_blocks;
   const int grid = std::min(tiles, dev.sm_count);
-  return launch_pdl(kern, dim3(grid), dim3(kSThreads), kSAlloc, st, tmA, tmBh, tmBl, p);
+  return launch_pdl(kern, dim3(grid), dim3(kSThreads), kSAlloc, st, tmA, tmBh, tmBl, tmSrc, tmQ, p);
 }
 
 }  // namespace
@@ -569,11 +642,14 @@ cudaError_t launch_ste_backward(const SteArgs& a, cudaStream_t st, const DeviceI
   float* tx = reinterpret_cast<float*>(ws + L.tx);
   float* tw = reinterpret_cast<float*>(ws + L.tw);
   unsigned int* mw = reinterpret_cast<unsigned int*>(ws + L.mw);
+  const int fin_blocks = (static_cast<int>(a.K) + kFinishThreads - 1) / kFinishThreads;
+  double* fin_partial = reinterpret_cast<double*>(ws + L.fin);
+  unsigned int* fin_counter = reinterpret_cast<unsigned int*>(ws + L.fin + static_cast<size_t>(fin_blocks) * 8);
   const int M = static_cast<int>(a.M), N = static_cast<int>(a.N), K = static_cast<int>(a.K);
   const int Mp = static_cast<int>(L.Mp);
 
   cudaError_t e = launch_pdl(ste_init_kernel, dim3(std::max(1, std::min(dev.sm_count, (std::max(K, N) + 255) / 256))),
-                             dim3(256), 0, st, tx, tw, mw, K, a.db, N);
+                             dim3(256), 0, st, tx, tw, mw, K, a.db, N, fin_counter);
   if (e != cudaSuccess) return *why = "init launch", e;
   e = launch_pdl(split_g_kernel, dim3((N + kTT - 1) / kTT, (M + kTT - 1) / kTT), dim3(kTThreads), 0, st, a.G, M, N,
                  a.w_scale, a.x_scale, Gh, Gl, Gth, Gtl, Mp, a.db);
@@ -605,8 +681,9 @@ cudaError_t launch_ste_backward(const SteArgs& a, cudaStream_t st, const DeviceI
   // dWs^T[k][n] = sum_m Xt[k][m] (Gth + Gtl)[n][m]
   e = run_ste_gemm<kEpiDW>(Xt, Gth, Gtl, a.K, a.N, a.M, L.Mp, p, st, dev, why);
   if (e != cudaSuccess) return e;
-  e = launch_pdl(ste_finish_kernel, dim3(1), dim3(kFinishThreads), 0, st, static_cast<const float*>(tx),
-                 static_cast<const float*>(tw), static_cast<const unsigned int*>(mw), a.mx, a.s, a.alpha, K, a.ds, a.d_eta);
+  e = launch_pdl(ste_finish_kernel, dim3(fin_blocks), dim3(kFinishThreads), 0, st, static_cast<const float*>(tx),
+                 static_cast<const float*>(tw), static_cast<const unsigned int*>(mw), a.mx, a.s, a.alpha, K, a.ds,
+                 fin_partial, fin_counter, a.d_eta);
   if (e != cudaSuccess) return *why = "finish launch", e;
   return cudaSuccess;
 }
