@@ -58,6 +58,8 @@ FLUSH_READ_BYTES = 512 << 20   # then read, leaving L2 clean
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 INT8_OVER_BF16 = 2.0  # nominal dense int8 / bf16 ratio (4.5 / 2.25 PFLOP/s)
+# fp32 multiply-add peak of the CUDA cores: 148 SMs x 128 lanes x 2 flops x 1.965 GHz
+FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 
 
 def parse_args():
@@ -67,10 +69,12 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default="proj", choices=sorted(workloads.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--path", default="smoothquant", choices=["smoothquant", "per-tensor", "ste-train"],
+    ap.add_argument("--path", default="smoothquant", choices=["smoothquant", "per-tensor", "ste-train", "weight-only"],
                     help="per-tensor: the baseline W8A8 path (one scale per tensor) on the same workload; "
                          "ste-train: a learnable-alpha training step (s from the running max, forward, "
-                         "straight-through backward to X, W, bias and eta_alpha)")
+                         "straight-through backward to X, W, bias and eta_alpha); weight-only: the int8 "
+                         "weight-only comparison (weight quantised per output channel with s = 1, bf16 "
+                         "activations)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=50)
@@ -96,6 +100,9 @@ def workload_config(wl, path="smoothquant"):
     }
     if path == "per-tensor":
         c["workload"] = "per-tensor W8A8 baseline (one scale per tensor), " + c["workload"]
+    elif path == "weight-only":
+        c["workload"] = ("int8 weight-only comparison (W quantised per output channel with s = 1, activations "
+                         "bf16), " + c["workload"])
     elif path == "ste-train":
         c["workload"] = ("learnable-alpha training step (s from the running max of the calibration batch, "
                          "forward, straight-through backward of a seeded bf16 dL/dY), " + c["workload"])
@@ -127,8 +134,10 @@ def algorithmic_work(wl):
         # G, X, W, Xq, Wq and the scales in; dX, dW (fp32), db, ds out; two
         # contractions of 2MNK each (counted once, whatever the kernel's split)
         "sq_ste_backward": (2 * M * N + 7 * M * K + 7 * N * K + 8 * M + 12 * N + 12 * K, 4 * M * N * K),
+        # X (bf16) and the codes in, Y out; 2MNK multiply-add operations on the fp32 CUDA cores
+        "sq_linear_weight_only": (2 * M * K + N * K + 4 * N + 2 * M * N, 2 * M * N * K),
     }
-    typ = {"sq_ste_backward": "bf16"}
+    typ = {"sq_ste_backward": "bf16", "sq_linear_weight_only": "fp32-alu"}
     return {n: (b, o, typ.get(n, "int8")) for n, (b, o) in work.items()}
 
 
@@ -250,6 +259,11 @@ def oracle_step(inp, wl, rows=None, path="smoothquant"):
         Wq, ws = O.fold_and_quantize_weight(inp["W"], s)
         Y, _, _, _ = O.forward(X, s, Wq, ws, inp["bias"])
         return Y, STE.ste_backward(G, X, inp["W"], mx, wl.alpha_f32)
+    if path == "weight-only":
+        from oracle import weight_only as WO
+        X = inp["X"] if rows is None else inp["X"][:rows]
+        Wq, ws = O.fold_and_quantize_weight(inp["W"], np.ones(wl.K, np.float32))
+        return WO.weight_only_linear(X, Wq, ws, inp["bias"])[0]
     if path == "per-tensor":
         from oracle import per_tensor as PT
         X = inp["X"] if rows is None else inp["X"][:rows]
@@ -330,6 +344,8 @@ def kernel_report(wl, names, per_call, per_call_single, launches_per_call):
         ms = per_call[n]
         sustained = ms >= SUSTAINED_AFTER_MS and bf16_tf_sus is not None
         int8_peak_tops = (bf16_tf_sus if sustained else bf16_tf) * (INT8_OVER_BF16 if op_type == "int8" else 1.0)
+        if op_type == "fp32-alu":
+            int8_peak_tops = FP32_ALU_TFLOPS
         # the bound is whichever roofline takes longer for this call's work
         t_hbm = nbytes / (hbm_gbs * 1e9)
         t_tensor = ops / (int8_peak_tops * 1e12)
@@ -346,9 +362,15 @@ def kernel_report(wl, names, per_call, per_call_single, launches_per_call):
                           "peak": "sustained" if sustained else "burst", "launches": launches_per_call[n]}
             if op_type != "int8":
                 kernels[n]["operands"] = op_type
+            if op_type == "fp32-alu":
+                kernels[n]["bound"] = "alu"
     dom = max(names, key=lambda n: per_call[n])
     kd = kernels[dom]
-    if kd["bound"] == "hbm":
+    if kd["bound"] == "alu":
+        roof = {"bound": "alu", "achieved": kd["achieved_tops"], "peak": kd["int8_peak_tops"], "unit": "TFLOP/s",
+                "frac": kd["achieved_tops"] / kd["int8_peak_tops"],
+                "peak_source": "fp32 FMA peak of the CUDA cores from unit counts and the 1965 MHz clock"}
+    elif kd["bound"] == "hbm":
         roof = {"bound": "hbm", "achieved": kd["achieved_gbs"], "peak": hbm_gbs, "unit": "GB/s",
                 "frac": kd["achieved_gbs"] / hbm_gbs}
         roof["peak_source"] = f"{peak_kind} HBM copy"
@@ -389,7 +411,14 @@ def run_ours(args, wl, rank, world, local_rank):
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     flush_read = torch.ones(FLUSH_READ_BYTES // 4, dtype=torch.int32, device=dev)
 
-    if args.path == "ste-train":
+    if args.path == "weight-only":
+        ones = torch.ones(K, dtype=torch.float32, device=dev)
+        calls = {
+            "sq_prepare_weight": lambda: sq.sq_prepare_weight(W, ones, Wq=Wq, w_scale=w_scale),
+            "sq_linear_weight_only": lambda: sq.sq_linear_weight_only(X, Wq, w_scale, b, Y=Y),
+        }
+        launches_per_call = {"sq_prepare_weight": 1, "sq_linear_weight_only": 1}
+    elif args.path == "ste-train":
         # the training step of the learnable-alpha layer: s recomputed from the
         # running activation max (taken once from the calibration batch) and
         # the weight, the forward, and the straight-through backward
@@ -549,12 +578,16 @@ def run_ours(args, wl, rank, world, local_rank):
             dG, dmx = torch.empty_like(G), torch.empty_like(mx)
 
         def e2e_step():
-            dC.copy_(hC, non_blocking=True)
+            if args.path == "smoothquant":
+                dC.copy_(hC, non_blocking=True)
             dW.copy_(hW, non_blocking=True)
             dX.copy_(hX, non_blocking=True)
             if db is not None:
                 db.copy_(hb, non_blocking=True)
-            if args.path == "ste-train":
+            if args.path == "weight-only":
+                sq.sq_prepare_weight(dW, ones, Wq=Wq, w_scale=w_scale)
+                sq.sq_linear_weight_only(dX, Wq, w_scale, db, Y=Y)
+            elif args.path == "ste-train":
                 dG.copy_(hG, non_blocking=True)
                 dmx.copy_(hmx, non_blocking=True)
                 sq.sq_calibrate(None, dW, wl.alpha_f32, s=s, mx_inout=dmx, workspace=ws_cal)
@@ -592,8 +625,12 @@ def run_ours(args, wl, rank, world, local_rank):
             outs = (hY, h_eta)
             call = ("sq_calibrate(mx) + sq_prepare_weight + sq_quantize_act + sq_linear + sq_ste_backward, "
                     "Y and d eta read back")
+        elif args.path == "weight-only":
+            ins = (hW, hX) + ((hb,) if hb is not None else ())
+            outs = (hY,)
+            call = "sq_prepare_weight (s = 1) + sq_linear_weight_only"
         else:
-            ins = (hC, hW, hX) + ((hb,) if hb is not None else ())
+            ins = ((hC,) if args.path == "smoothquant" else ()) + (hW, hX) + ((hb,) if hb is not None else ())
             outs = (hY,)
             call = ("sq_quantize_per_tensor(W) + sq_quantize_per_tensor(X) + sq_linear"
                     if args.path == "per-tensor" else "sq_calibrate + sq_prepare_weight + sq_forward")
@@ -611,6 +648,7 @@ def run_ours(args, wl, rank, world, local_rank):
     if not args.no_cpu_baseline and world == 1:
         v, n, el = cpu_oracle_rate(wl, args.cpu_seconds, path=args.path)
         what = {"per-tensor": "quantise W and X per tensor, product",
+                "weight-only": "quantise W per output channel, bf16 x int8 product",
                 "ste-train": "s from the running max, fold+quantise W, forward, straight-through backward"}
         cpu = {"value": v, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
                "sample": f"{n} whole {wl.name} steps in {el:.1f} s ("
@@ -622,7 +660,8 @@ def run_ours(args, wl, rank, world, local_rank):
         "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "int8", "data": "synthetic", "config": workload_config(wl, args.path),
         "tops_per_step": 2.0 * wl.M * wl.N * wl.K * world / (step_ms * 1e-3) / 1e12,
-        "gemm_tops": 2 * wl.M * wl.N * wl.K / (per_call["sq_linear"] * 1e-3) / 1e12,
+        "gemm_tops": 2 * wl.M * wl.N * wl.K / (per_call.get("sq_linear", per_call.get("sq_linear_weight_only"))
+                                                * 1e-3) / 1e12,
         "roofline": roof, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": args.steps * sum(launches_per_call.values()),  # the timed step replays
         "clocks": clocks, "wall_s_timed": wall,

@@ -48,3 +48,24 @@ def test_long_kernels_use_the_sustained_peak():
         assert abs(roof["peak"] - bf16_sus * 2) < 1e-9
     wl, (kernels, roof) = _report("mlp", [0.02, 0.03, 0.01, 0.08])
     assert kernels["sq_linear"]["peak"] == "burst"
+
+
+def test_other_paths_take_their_own_peaks():
+    """The backward's products are bf16 (the measured bf16 peak, not x2); the
+    weight-only product runs on the fp32 CUDA cores (the ALU peak)."""
+    hbm, bf16, bf16_sus, _ = bench.peaks()
+    wl = workloads.get("proj")
+    names = ["sq_linear", "sq_ste_backward"]
+    per = {"sq_linear": 0.0125, "sq_ste_backward": 0.030}
+    kernels, roof = bench.kernel_report(wl, names, per, per, {"sq_linear": 1, "sq_ste_backward": 7})
+    k = kernels["sq_ste_backward"]
+    assert k["bound"] == "tensor" and k["operands"] == "bf16"
+    assert abs(k["int8_peak_tops"] - bf16) < 1e-9
+    assert abs(k["achieved_tops"] - 4 * 512 * 4096 * 4096 / 30e-6 / 1e12) < 1e-6
+    wl = workloads.get("decode")
+    names = ["sq_prepare_weight", "sq_linear_weight_only"]
+    per = {"sq_prepare_weight": 0.0115, "sq_linear_weight_only": 0.054}
+    kernels, roof = bench.kernel_report(wl, names, per, per, {n: 1 for n in names})
+    assert roof["bound"] == "alu" and roof["kernel"] == "sq_linear_weight_only"
+    assert abs(roof["peak"] - 148 * 128 * 2 * 1.965e9 / 1e12) < 1e-9
+    assert abs(roof["frac"] - 2 * 8 * 8192 * 8192 / 54e-6 / 1e12 / roof["peak"]) < 1e-9
