@@ -54,3 +54,21 @@ def test_reference_arm_runs_on_rank_zero_only(capsys):
     args = types.SimpleNamespace(steps=1, warmup=0, gpus=2)
     bench.run_reference(args, workloads.get("tiny"), rank=1, world=2)
     assert capsys.readouterr().out == ""
+
+
+@pytest.mark.parametrize("path", ["smoothquant", "per-tensor", "ste-train", "weight-only"])
+def test_reference_arm_line_on_rank_zero(capsys, path):
+    """The reference arm (the CPU oracle) prints one JSON line per run with
+    the keys the driver reads, for every bench path."""
+    import json
+    import types
+    import bench
+    import workloads
+    args = types.SimpleNamespace(steps=1, warmup=0, gpus=1, path=path)
+    bench.run_reference(args, workloads.get("tiny"), rank=0, world=1)
+    line = json.loads(capsys.readouterr().out.strip())
+    assert line["impl"] == "reference" and line["metric"] == bench.metric_for(path)
+    for k in ("value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better", "config",
+              "cpu_baseline", "e2e"):
+        assert k in line
+    assert line["value"] > 0 and line["e2e"]["h2d_bytes_per_step"] == 0
