@@ -149,10 +149,11 @@ REPS = 8
 SUSTAINED_AFTER_MS = 0.5
 
 
-def source_sha():
+def source_sha(files=None):
+    """Hash of the kernel sources (all of csrc/, or the listed files of it)."""
     h = hashlib.sha256()
     cs = os.path.join(ROOT, "w8a8_smoothquant_int8_sq_b200", "csrc")
-    for f in sorted(os.listdir(cs)):
+    for f in sorted(files if files else os.listdir(cs)):
         h.update(open(os.path.join(cs, f), "rb").read())
     return h.hexdigest()[:16]
 
@@ -168,7 +169,7 @@ def ncu_traffic(kernel_call, wl_name):
     except Exception:
         return None
     e = d.get(wl_name, {}).get(kernel_call)
-    if not e or e.get("source_sha") != source_sha():
+    if not e or e.get("source_sha") != source_sha(e.get("sources")):
         return None
     return e.get("dram_bytes_per_launch")
 
