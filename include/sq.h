@@ -13,6 +13,15 @@
  *                  quantize_per_token_symmetric)
  *   int8 linear    acc = Xq Wq^T (int32) ; Y = bf16(acc * x_scale[m] * w_scale[n] + bias[n])
  *                  (forward: "INT8 x INT8 -> INT32 -> fp32" on real hardware)
+ *   backward       straight-through gradients of the learnable-alpha layer's
+ *                  quantised-mode forward: dX, dW, db, ds, d eta_alpha
+ *                  (STEQuantize, SmoothQuantW8A8.alpha / forward)
+ *
+ * and two comparison points from other pages:
+ *
+ *   per-tensor     one scale per tensor (quantized_linear.py, quantize_tensor)
+ *   weight-only    bf16 activations times int8 weights (torchao,
+ *                  Int8WeightOnlyQuantizedLinearWeight)
  *
  * Conventions shared by every entry point
  *   - Layouts are row-major and dense: X[M][K], C[R][K], W[N][K] (nn.Linear
