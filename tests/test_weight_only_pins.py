@@ -51,3 +51,46 @@ def test_closed_form_ones():
     assert np.all(SQ.widen_bf16(Y) == np.float32(K * 127 * 2.0 ** -7))
     S = WO.abs_product_sum(X, -Wq, ws)
     assert np.all(S == K * 127 * 2.0 ** -7)
+
+
+# --------------------------------------------------------------- planted mistakes
+import pytest  # noqa: E402
+
+
+def _mut(kind):
+    def linear(X_bits, Wq, w_scale, bias_bits=None):
+        X = SQ.widen_bf16(np.asarray(X_bits)).astype(np.float64)
+        Q = np.asarray(Wq).astype(np.float64)
+        ws = np.asarray(w_scale, dtype=np.float64)
+        if kind == "scale_per_input_channel":
+            y = (X * np.resize(ws, X.shape[1])[None, :]) @ Q.T
+        elif kind == "transposed_codes":
+            y = (X @ Q[:, ::-1].T) * ws[None, :]
+        elif kind == "dropped_bias":
+            y = (X @ Q.T) * ws[None, :]
+            return SQ.bf16_round(y), y
+        elif kind == "bf16_per_product":
+            y = np.zeros((X.shape[0], Q.shape[0]))
+            for k in range(X.shape[1]):
+                y = SQ.widen_bf16(SQ.bf16_round(y + np.outer(X[:, k], Q[:, k]))).astype(np.float64)
+            y = y * ws[None, :]
+        else:
+            y = (X @ Q.T) * ws[None, :]
+        if bias_bits is not None:
+            y = y + SQ.widen_bf16(np.asarray(bias_bits)).astype(np.float64)[None, :]
+        return SQ.bf16_round(y), y
+    return linear
+
+
+@pytest.mark.parametrize("kind", ["scale_per_input_channel", "transposed_codes", "dropped_bias", "bf16_per_product"])
+def test_mutant_is_caught(kind, monkeypatch):
+    caught = []
+    for pin in (test_brute_force_small, test_matches_dequantised_weight_form, test_closed_form_ones):
+        monkeypatch.setattr(WO, "weight_only_linear", _mut(kind))
+        try:
+            pin()
+        except AssertionError:
+            caught.append(pin.__name__)
+        finally:
+            monkeypatch.undo()
+    assert caught, f"no pin catches {kind}"
