@@ -102,3 +102,29 @@ def test_valid_call_without_gpu_fails_cleanly(sq):
     st = sq.lib.sq_quantize_act(a, 4, 64, a, a, a, None)
     assert st in (5, 6)          # no sm_100 device: UNSUPPORTED or CUDA error, never a crash
     assert sq.lib.sq_last_error()
+
+
+def test_binding_refuses_host_tensors(sq):
+    """No CPU fallback: every entry point of the binding rejects host tensors
+    before calling the library."""
+    import torch
+    bf = torch.zeros(4, 64, dtype=torch.bfloat16)
+    i8 = torch.zeros(4, 64, dtype=torch.int8)
+    f1 = torch.zeros(64, dtype=torch.float32)
+    f4 = torch.zeros(4, dtype=torch.float32)
+    G = torch.zeros(4, 8, dtype=torch.bfloat16)
+    W8 = torch.zeros(8, 64, dtype=torch.bfloat16)
+    calls = [
+        lambda: sq.sq_calibrate(bf, bf, 0.5),
+        lambda: sq.sq_prepare_weight(bf, f1),
+        lambda: sq.sq_quantize_act(bf, f1),
+        lambda: sq.sq_quantize_per_tensor(bf),
+        lambda: sq.sq_linear(i8, f4, i8, f4),
+        lambda: sq.sq_forward(bf, f1, i8, f4),
+        lambda: sq.sq_linear_weight_only(bf, i8, f4),
+        lambda: sq.sq_ste_backward(G, bf, W8, f1, f1, 0.5, i8, f4, torch.zeros(8, 64, dtype=torch.int8),
+                                   torch.zeros(8, dtype=torch.float32)),
+    ]
+    for c in calls:
+        with pytest.raises(ValueError, match="CUDA tensor"):
+            c()
