@@ -1,6 +1,7 @@
 """Benchmark of the SmoothQuant W8A8 int8 linear layer on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload proj]
+                    [--path smoothquant|per-tensor|ste-train|weight-only] [--serial]
                     [--impl ours|reference] [--no-e2e] [--no-cpu-baseline]
 
 A step is one pass of the whole path over one batch of seeded synthetic input:
@@ -27,6 +28,12 @@ nodes between the single calls gives `ms_single_launch`.  With N > 1
 (one process per GPU under torchrun) every rank runs an independent replica
 (the layer shards by tokens with no exchange): the value is the tokens all
 ranks processed divided by the slowest rank's time.
+
+Other paths time the comparison points and the training step on the same
+workloads: `per-tensor` (one scale per tensor for W and X, then the int8
+GEMM), `ste-train` (s from the running max, the forward, and the
+straight-through backward to X, W, bias and eta_alpha of a seeded dL/dY),
+`weight-only` (W quantised per output channel with s = 1, bf16 activations).
 
 The JSON line adds: `e2e` (the same step through the Python binding with the
 inputs copied from pinned host memory and Y copied back, every step),
