@@ -72,3 +72,9 @@ def test_reference_arm_line_on_rank_zero(capsys, path):
               "cpu_baseline", "e2e"):
         assert k in line
     assert line["value"] > 0 and line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_step_stats():
+    import bench
+    mean, median = bench.step_stats([1.0, 2.0, 10.0])
+    assert mean == pytest.approx(13.0 / 3) and median == 2.0
