@@ -16,6 +16,7 @@ with:
   depend on s, so ds = 0 and d eta = 0;
 * the algebraic form ds_j s_j = sum_n dWs (W s - Wdq) - sum_m dXs (X/s - Xdq)
   (the two ways of writing it agree whatever the codes are);
+* linearity in G (the forward fixed, the gradients of G1 + G2 are the sums);
 * sigmoid at points where its value is exact.
 """
 from __future__ import annotations
@@ -133,6 +134,25 @@ def pin_error_form(bwd, seed=81):
     assert np.max(np.abs(T)) > 1e-6 * np.max(big), "the case must be lossy"
 
 
+def pin_linear_in_G(bwd, seed=91):
+    """With the forward fixed, every straight-through gradient is linear in
+    G = dL/dY: the gradients of G1 + G2 are the sums of those of G1 and G2
+    (G1, G2 small integers times 2^-10, so that G1 + G2 is exact in bf16)."""
+    wl = workloads.get("tiny")
+    inp = workloads.make_inputs(wl, ("X", "W", "C"))
+    mx = SQ.column_max_abs(SQ.widen_bf16(inp["C"]))
+    rng = np.random.default_rng(seed)
+    g1 = rng.integers(-60, 61, size=(wl.M, wl.N)) * 2.0 ** -10
+    g2 = rng.integers(-60, 61, size=(wl.M, wl.N)) * 2.0 ** -10
+    a = np.float32(wl.alpha_f32)
+    r1 = bwd(bits(g1), inp["X"], inp["W"], mx, a)
+    r2 = bwd(bits(g2), inp["X"], inp["W"], mx, a)
+    r12 = bwd(bits(g1 + g2), inp["X"], inp["W"], mx, a)
+    for k in ("dX", "dW", "db", "ds"):
+        _close(r12[k], r1[k] + r2[k], 1e-12, scale=np.max(np.abs(r1[k])) + np.max(np.abs(r2[k])))
+    _close(r12["deta"], r1["deta"] + r2["deta"], 1e-9, scale=abs(r1["deta"]) + abs(r2["deta"]))
+
+
 def pin_sigmoid():
     assert STE.alpha_from_logit(0.0) == np.float32(0.5)
     assert STE.alpha_from_logit(math.log(3.0)) == np.float32(0.75)
@@ -141,4 +161,4 @@ def pin_sigmoid():
     assert STE.alpha_from_logit(800.0) == np.float32(1.0)
 
 
-ALL_PINS = [pin_autograd, pin_lossless, pin_error_form]
+ALL_PINS = [pin_autograd, pin_lossless, pin_error_form, pin_linear_in_G]
