@@ -1,43 +1,53 @@
 """Benchmark of the SmoothQuant W8A8 int8 linear layer on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload proj]
-                    [--path smoothquant|per-tensor|ste-train|weight-only] [--serial]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload prefill]
+                    [--path smoothquant|forward|per-tensor|ste-train|weight-only] [--serial]
                     [--impl ours|reference] [--no-e2e] [--no-cpu-baseline]
 
 A step is one pass of the whole path over one batch of seeded synthetic input:
 calibration (column max-abs of the calibration batch and of W, smoothing
 factor s), weight fold + int8 quantisation, per-token activation quantisation
 and the int8 tcgen05 GEMM with its dequant + bias epilogue.  The default
-workload is the projection-shaped layer: X[512x4096] bf16 with 41 outlier
-channels x50, W[4096x4096] bf16 ~N(0,0.02), no bias, alpha 0.5, calibration
-batch of 512 rows.
+workload is the largest layer, the prefill GEMM: X[8192x8192] bf16 with 41
+outlier channels x100, W[28672x8192] bf16 ~N(0,0.01), no bias, alpha 0.5,
+calibration batch of 512 rows.  `--workload tiny|proj|mlp|decode` selects the
+other layer shapes.
 
-Timing: every step is preceded by an L2 flush (the inputs are smaller than
-L2): a 256 MiB write, then a 512 MiB read, so that L2 holds neither the
+Paths (`--path`):
+  smoothquant  the whole path above (default, except for decode);
+  forward      the per-call path once the weight is prepared: sq_forward on
+               pre-quantised weights (default for decode: every call streams
+               the 64 MiB of int8 W from HBM -- the calls rotate over enough
+               prepared weight copies, >= 256 MiB, that L2 cannot serve them);
+  per-tensor   one scale per tensor for W and X, then the int8 GEMM;
+  ste-train    s from the running max, the forward, and the straight-through
+               backward to X, W, bias and eta_alpha of a seeded dL/dY;
+  weight-only  W quantised per output channel with s = 1, bf16 activations.
+
+Timing.  Whole steps (all paths but forward): every step is preceded by an L2
+flush (a 256 MiB write, then a 512 MiB read, so that L2 holds neither the
 step's inputs nor dirty lines whose write-back would land inside the timed
-step.  The step (the four library calls) is captured as a CUDA graph with timing-event
+step); the step's calls are captured as one CUDA graph with timing-event
 nodes before and after it; the kernels overlap each other's launch through
 programmatic dependent launch, and calls that depend only on earlier calls
-of the step (the weight prep and the activation quantiser both need s alone)
-run on forked streams (`--serial` captures them in order instead).  Per call, a capture of 8 back-to-back
-launches of that call between two event nodes, replayed after the same flush,
-gives its kernel duration (the span / 8, so the event node's launch latency is
-amortised; the first launch reads its operands from HBM, the rest find them in
-L2, as the step's later calls do) used for the roofline; a capture with event
-nodes between the single calls gives `ms_single_launch`.  With N > 1
-(one process per GPU under torchrun) every rank runs an independent replica
-(the layer shards by tokens with no exchange): the value is the tokens all
-ranks processed divided by the slowest rank's time.
+(the weight prep and the activation quantiser both need s alone) run on
+forked streams (`--serial` captures them in order).  The forward path captures
+the K timed calls as one graph between two event nodes (the span / K is the
+step time), each call on the next weight copy of the rotation.
 
-Other paths time the comparison points and the training step on the same
-workloads: `per-tensor` (one scale per tensor for W and X, then the int8
-GEMM), `ste-train` (s from the running max, the forward, and the
-straight-through backward to X, W, bias and eta_alpha of a seeded dL/dY),
-`weight-only` (W quantised per output channel with s = 1, bf16 activations).
+Per call (the roofline and the `kernels` breakdown): a graph of back-to-back
+launches of that call between two event nodes, replayed after the L2 flush;
+consecutive launches take their inputs from different copies (a rotation whose
+copies add up to at least 256 MiB, twice the L2), so every launch reads its
+inputs from HBM.  The span / launches is the call's duration; a graph with
+event nodes between single calls gives `ms_single_launch`.  With N > 1 (one
+process per GPU under torchrun) every rank runs an independent replica (the
+layer shards by tokens with no exchange): the value is the tokens all ranks
+processed divided by the slowest rank's time.
 
 The JSON line adds: `e2e` (the same step through the Python binding with the
 inputs copied from pinned host memory and Y copied back, every step),
-`roofline` of the dominant kernel, `cpu_baseline` (the CPU oracle timed on a
+`roofline` of the dominant call, `cpu_baseline` (the CPU oracle timed on a
 bounded sample, rank 0 only), sampled `clocks`, and per-call `kernels` times.
 `--impl reference` times the CPU oracle itself as the reference arm.
 """
@@ -46,6 +56,7 @@ from __future__ import annotations
 import argparse
 import hashlib
 import json
+import math
 import os
 import subprocess
 import sys
@@ -63,37 +74,51 @@ METRIC = "W8A8 linear int8 TOPS & tokens/s at 1 B200; % of INT8 tensor peak / HB
 UNIT = "tokens/s"
 FLUSH_BYTES = 256 << 20        # written before each step
 FLUSH_READ_BYTES = 512 << 20   # then read, leaving L2 clean
+L2_BYTES = 126 << 20
+ROTATE_BYTES = 256 << 20       # inputs of a rotation add up to at least this (2x L2)
+MAX_ROTATION = 128             # copies at most (tiny inputs stay partly L2-resident)
 # fallback peaks (only if MEASURED_PEAKS.json is absent)
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 INT8_OVER_BF16 = 2.0  # nominal dense int8 / bf16 ratio (4.5 / 2.25 PFLOP/s)
 # fp32 multiply-add peak of the CUDA cores: 148 SMs x 128 lanes x 2 flops x 1.965 GHz
 FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+PATHS = ["smoothquant", "forward", "per-tensor", "ste-train", "weight-only"]
+# sq_forward fuses the activation quantisation into the weight-streaming
+# kernel up to this many tokens (one launch), else runs the quantiser first
+FORWARD_FUSED_MAX_M = 8
 
 
-def parse_args():
+def parse_args(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=3000)
-    ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--workload", default="proj", choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="prefill", choices=sorted(workloads.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--path", default="smoothquant", choices=["smoothquant", "per-tensor", "ste-train", "weight-only"],
-                    help="per-tensor: the baseline W8A8 path (one scale per tensor) on the same workload; "
+    ap.add_argument("--path", default=None, choices=PATHS,
+                    help="smoothquant: the whole path (default); forward: sq_forward on prepared weights "
+                         "(default for decode); per-tensor: the baseline W8A8 path (one scale per tensor); "
                          "ste-train: a learnable-alpha training step (s from the running max, forward, "
-                         "straight-through backward to X, W, bias and eta_alpha); weight-only: the int8 "
-                         "weight-only comparison (weight quantised per output channel with s = 1, bf16 "
-                         "activations)")
+                         "straight-through backward); weight-only: the int8 weight-only comparison")
     ap.add_argument("--serial", action="store_true",
                     help="capture the step's calls strictly in order (by default calls that depend only on "
                          "earlier stages run on forked streams)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--settle-s", type=float, default=1.0,
                     help="untimed replays after warm-up until this much wall time has passed (clock sampling)")
-    return ap.parse_args()
+    args = ap.parse_args(argv)
+    if args.path is None:
+        args.path = default_path(args.workload)
+    return args
+
+
+def default_path(workload_name):
+    """The decode layer is timed as a per-call layer on prepared weights."""
+    return "forward" if workload_name == "decode" else "smoothquant"
 
 
 def metric_for(path):
@@ -108,7 +133,7 @@ def workload_config(wl, path="smoothquant"):
                     f"{wl.outliers} outlier channels x{wl.outlier_scale:g}, calibration {wl.R} rows, "
                     f"{'bias' if wl.has_bias else 'no bias'}",
         "M": wl.M, "N": wl.N, "K": wl.K, "R": wl.R,
-        "l2": "flushed before every timed step (256 MiB write, then 512 MiB read); inputs smaller than L2",
+        "l2": "flushed before every timed step (256 MiB write, then 512 MiB read)",
     }
     if path == "per-tensor":
         c["workload"] = "per-tensor W8A8 baseline (one scale per tensor), " + c["workload"]
@@ -118,7 +143,18 @@ def workload_config(wl, path="smoothquant"):
     elif path == "ste-train":
         c["workload"] = ("learnable-alpha training step (s from the running max of the calibration batch, "
                          "forward, straight-through backward of a seeded bf16 dL/dY), " + c["workload"])
+    elif path == "forward":
+        c["workload"] = ("per-call forward on pre-quantised weights (sq_forward: activation quantisation + "
+                         "int8 GEMM + epilogue; calibration and weight prep done once, untimed), " + c["workload"])
+        c["l2"] = (f"calls rotate over {forward_rotation(wl)} prepared weight copies "
+                   f"({forward_rotation(wl) * wl.N * wl.K / 2**20:.0f} MiB of int8 W), so every call streams "
+                   f"its weight from HBM")
     return c
+
+
+def forward_rotation(wl):
+    """Prepared weight copies the forward path rotates over (>= 4, >= 256 MiB)."""
+    return max(4, min(MAX_ROTATION, -(-ROTATE_BYTES // (wl.N * wl.K + 4 * wl.N))))
 
 
 def peaks():
@@ -138,6 +174,9 @@ def algorithmic_work(wl):
         "sq_prepare_weight": (3 * N * K + 4 * N + 4 * K, 0),
         "sq_quantize_act": (3 * M * K + 4 * M + 4 * K, 0),
         "sq_linear": (M * K + N * K + 2 * M * N + 4 * M + 4 * N, 2 * M * N * K),
+        # X in (bf16), s, the codes and scales of W in, Y out; the codes of X
+        # need not leave the chip
+        "sq_forward": (2 * M * K + 4 * K + N * K + 4 * N + 2 * M * N, 2 * M * N * K),
         # one scale per tensor: the data once in, the codes and the scale row out
         "sq_quantize_per_tensor(W)": (3 * N * K + 4 * N, 0),
         "sq_quantize_per_tensor(X)": (3 * M * K + 4 * M, 0),
@@ -153,7 +192,7 @@ def algorithmic_work(wl):
     return {n: (b, o, typ.get(n, "int8")) for n, (b, o) in work.items()}
 
 
-# Per-call kernel durations are spans over this many back-to-back launches.
+# Per-call kernel durations are spans over at least this many back-to-back launches.
 REPS = 8
 
 # A kernel running this long sits in a power-capped stretch of work: its
@@ -184,6 +223,14 @@ def ncu_traffic(kernel_call, wl_name):
     if not e or e.get("source_sha") != source_sha(e.get("sources")):
         return None
     return e.get("dram_bytes_per_launch")
+
+
+def rotation_count(footprint_bytes):
+    """Input copies that make back-to-back launches read from HBM: their
+    inputs add up to at least ROTATE_BYTES (at most MAX_ROTATION copies)."""
+    if footprint_bytes <= 0:
+        return 1
+    return int(max(1, min(MAX_ROTATION, -(-ROTATE_BYTES // footprint_bytes))))
 
 
 # ------------------------------------------------------------- multi-rank
@@ -267,31 +314,100 @@ class ClockSampler:
 
 
 # --------------------------------------------------------------- CPU oracle
-def oracle_step(inp, wl, rows=None, path="smoothquant"):
+# Largest whole step the CPU legs run; beyond it the smoothquant step is timed
+# on a sample of rows and extrapolated phase by phase.
+WHOLE_STEP_MAX_MNK = 1.0e11
+WHOLE_STEP_MAX_NK = 64 << 20
+SAMPLE_X_ROWS = 256
+SAMPLE_W_ROWS = 4096
+
+
+def sample_plan(wl, path):
+    """(rows of X, rows of W) the oracle's step runs on: all of them for the
+    smaller layers, a seeded-input prefix for the prefill layer."""
+    if path != "smoothquant" or (wl.M * wl.N * wl.K <= WHOLE_STEP_MAX_MNK and wl.N * wl.K <= WHOLE_STEP_MAX_NK):
+        return wl.M, wl.N
+    return min(wl.M, SAMPLE_X_ROWS), min(wl.N, SAMPLE_W_ROWS)
+
+
+def oracle_inputs(wl, path, inp=None):
+    """The seeded inputs of `wl` (or a copy of `inp`) plus what the path's
+    untimed set-up needs."""
+    inp = dict(workloads.make_inputs(wl) if inp is None else inp)
+    if path == "ste-train":
+        inp["G"] = train_gradient(wl)
+    if path == "forward":
+        # the weight is prepared once, outside the timed calls (as on the GPU)
+        from oracle import smoothquant as O
+        s, _ = O.calibrate(inp["C"], inp["W"], wl.alpha_f32)
+        inp["s"] = s
+        inp["Wq"], inp["ws"] = O.fold_and_quantize_weight(inp["W"], s)
+    return inp
+
+
+def oracle_step_seconds(inp, wl, path="smoothquant"):
+    """Seconds the oracle takes for one whole step of `path` on `wl`.
+
+    For the prefill layer the smoothquant step is timed on a sample and
+    extrapolated per phase, each phase linear in what it processes:
+    calibration in full (it reads all of C and W); the weight fold +
+    quantisation on the first m_w rows of W (x N / m_w); the activation
+    quantisation on the first m_x rows of X (x M / m_x); the int8 product and
+    the epilogue on that m_x x m_w block (x M N / (m_x m_w))."""
     from oracle import smoothquant as O
+    pc = time.perf_counter
     if path == "ste-train":
         from oracle import ste_backward as STE
-        X = inp["X"] if rows is None else inp["X"][:rows]
-        G = inp["G"] if rows is None else inp["G"][:rows]
+        t0 = pc()
         mx = O.column_max_abs(O.widen_bf16(inp["C"]))
         s, _ = O.calibrate(inp["C"][:0], inp["W"], wl.alpha_f32, mx_prev=mx)
         Wq, ws = O.fold_and_quantize_weight(inp["W"], s)
-        Y, _, _, _ = O.forward(X, s, Wq, ws, inp["bias"])
-        return Y, STE.ste_backward(G, X, inp["W"], mx, wl.alpha_f32)
+        O.forward(inp["X"], s, Wq, ws, inp["bias"])
+        STE.ste_backward(inp["G"], inp["X"], inp["W"], mx, wl.alpha_f32)
+        return pc() - t0
     if path == "weight-only":
         from oracle import weight_only as WO
-        X = inp["X"] if rows is None else inp["X"][:rows]
+        t0 = pc()
         Wq, ws = O.fold_and_quantize_weight(inp["W"], np.ones(wl.K, np.float32))
-        return WO.weight_only_linear(X, Wq, ws, inp["bias"])[0]
+        WO.weight_only_linear(inp["X"], Wq, ws, inp["bias"])
+        return pc() - t0
     if path == "per-tensor":
         from oracle import per_tensor as PT
-        X = inp["X"] if rows is None else inp["X"][:rows]
-        return PT.linear_per_tensor(X, inp["W"], inp["bias"])[0]
+        t0 = pc()
+        PT.linear_per_tensor(inp["X"], inp["W"], inp["bias"])
+        return pc() - t0
+    if path == "forward":
+        t0 = pc()
+        O.forward(inp["X"], inp["s"], inp["Wq"], inp["ws"], inp["bias"])
+        return pc() - t0
+    mx_rows, mw_rows = sample_plan(wl, path)
+    b = inp["bias"]
+    t0 = pc()
     s, _ = O.calibrate(inp["C"], inp["W"], wl.alpha_f32)
-    Wq, ws = O.fold_and_quantize_weight(inp["W"], s)
-    X = inp["X"] if rows is None else inp["X"][:rows]
-    Y, _, _, _ = O.forward(X, s, Wq, ws, inp["bias"])
-    return Y
+    t1 = pc()
+    Wq, ws = O.fold_and_quantize_weight(inp["W"][:mw_rows], s)
+    t2 = pc()
+    Xq, xs = O.quantize_activation(inp["X"][:mx_rows], s)
+    t3 = pc()
+    acc = O.int8_gemm(Xq, Wq)
+    O.dequant_epilogue(acc, xs, ws, None if b is None else b[:mw_rows])
+    t4 = pc()
+    return ((t1 - t0) + (t2 - t1) * wl.N / mw_rows + (t3 - t2) * wl.M / mx_rows
+            + (t4 - t3) * (wl.M * wl.N) / (mx_rows * mw_rows))
+
+
+def oracle_sample_text(wl, path):
+    mx_rows, mw_rows = sample_plan(wl, path)
+    what = {"per-tensor": "quantise W and X per tensor, product",
+            "weight-only": "quantise W per output channel, bf16 x int8 product",
+            "ste-train": "s from the running max, fold+quantise W, forward, straight-through backward",
+            "forward": "forward on the prepared weight: quantise X, int8 product, epilogue",
+            "smoothquant": "calibrate, fold+quantise W, quantise X, int8 product, epilogue"}[path]
+    if (mx_rows, mw_rows) == (wl.M, wl.N):
+        return f"whole {wl.name} steps ({what})"
+    return (f"{wl.name} steps ({what}) timed on a sample and extrapolated per phase: calibration in full, "
+            f"weight prep on {mw_rows} of {wl.N} W rows, activation quantisation on {mx_rows} of {wl.M} X rows, "
+            f"product + epilogue on the {mx_rows}x{mw_rows} block (each phase scaled by the rows it covers)")
 
 
 def cpu_threads():
@@ -310,50 +426,49 @@ def train_gradient(wl):
     return workloads.random_bf16((wl.M, wl.N), seed=1000 * wl.index + 9, scale=1e-3)
 
 
-def cpu_oracle_rate(wl, seconds, max_steps=None, path="smoothquant"):
-    """Tokens/s of the oracle on whole steps, run until `seconds` pass."""
-    inp = workloads.make_inputs(wl)
-    if path == "ste-train":
-        inp["G"] = train_gradient(wl)
-    oracle_step(inp, wl, path=path)  # warm (page-in, BLAS threads)
-    n, t0 = 0, time.perf_counter()
+def cpu_oracle_rate(wl, seconds, path="smoothquant", inp=None):
+    """Tokens/s of the oracle on (extrapolated) whole steps, run until `seconds`
+    of CPU work have passed.  Returns (rate, steps, seconds of work)."""
+    inp = oracle_inputs(wl, path, inp)
+    oracle_step_seconds(inp, wl, path)  # warm (page-in, BLAS threads)
+    n, work, t0 = 0, 0.0, time.perf_counter()
+    ext = 0.0
     while True:
-        oracle_step(inp, wl, path=path)
+        ext += oracle_step_seconds(inp, wl, path)
         n += 1
-        el = time.perf_counter() - t0
-        if el >= seconds or (max_steps and n >= max_steps):
+        work = time.perf_counter() - t0
+        if work >= seconds:
             break
-    return wl.M * n / el, n, el
+    return wl.M * n / ext, n, work
 
 
 def run_reference(args, wl, rank, world):
     if rank != 0:
         return
-    inp = workloads.make_inputs(wl)
-    if args.path == "ste-train":
-        inp["G"] = train_gradient(wl)
+    path = getattr(args, "path", "smoothquant") or default_path(wl.name)
+    inp = oracle_inputs(wl, path)
     for _ in range(args.warmup):
-        oracle_step(inp, wl, path=args.path)
-    t0 = time.perf_counter()
+        oracle_step_seconds(inp, wl, path)
+    ext, t0 = 0.0, time.perf_counter()
     for _ in range(args.steps):
-        oracle_step(inp, wl, path=args.path)
-    el = time.perf_counter() - t0
-    v = wl.M * args.steps / el
+        ext += oracle_step_seconds(inp, wl, path)
+    work = time.perf_counter() - t0
+    v = wl.M * args.steps / ext
     cores = cpu_threads()
     line = {
-        "impl": "reference", "metric": metric_for(args.path), "value": v, "unit": UNIT, "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * el / args.steps,
+        "impl": "reference", "metric": metric_for(path), "value": v, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * ext / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64+fp32 (numpy)",
-        "data": "synthetic", "config": workload_config(wl, args.path),
+        "data": "synthetic", "config": workload_config(wl, path),
         "cpu_baseline": {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
-                         "sample": f"{args.steps} whole {wl.name} steps ({args.path} path of the oracle)"},
+                         "sample": f"{args.steps} {oracle_sample_text(wl, path)}; {work:.1f} s of CPU work"},
         "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
 
 
 # -------------------------------------------------------------------- GPU arm
-def kernel_report(wl, names, per_call, per_call_single, launches_per_call):
+def kernel_report(wl, names, per_call, per_call_single, launches_per_call, rotations=None):
     """Per-call roofline figures and the roofline object of the longest call."""
     hbm_gbs, bf16_tf, bf16_tf_sus, peak_kind = peaks()
     work = algorithmic_work(wl)
@@ -383,6 +498,8 @@ def kernel_report(wl, names, per_call, per_call_single, launches_per_call):
                 kernels[n]["operands"] = op_type
             if op_type == "fp32-alu":
                 kernels[n]["bound"] = "alu"
+        if rotations is not None and n in rotations:
+            kernels[n]["input_copies"], kernels[n]["l2_cold"] = rotations[n]
     dom = max(names, key=lambda n: per_call[n])
     kd = kernels[dom]
     if kd["bound"] == "alu":
@@ -403,6 +520,19 @@ def kernel_report(wl, names, per_call, per_call_single, launches_per_call):
     return kernels, roof
 
 
+class Call:
+    """One library call of the step: fn(T) enqueues it with the tensors of T;
+    `reads` names the tensors of T it reads from HBM (copied for the rotation
+    of the per-call timing); `launches` is its number of kernels."""
+
+    def __init__(self, fn, reads, launches):
+        self.fn, self.reads, self.launches = fn, reads, launches
+
+
+def nbytes(t):
+    return 0 if t is None else t.numel() * t.element_size()
+
+
 def run_ours(args, wl, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -415,141 +545,182 @@ def run_ours(args, wl, rank, world, local_rank):
     def d(bits):
         return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
 
-    C, W, X = d(inp["C"]), d(inp["W"]), d(inp["X"])
-    b = d(inp["bias"]) if inp["bias"] is not None else None
     K, N, M = wl.K, wl.N, wl.M
-    s = torch.empty(K, dtype=torch.float32, device=dev)
-    Wq = torch.empty(N, K, dtype=torch.int8, device=dev)
-    w_scale = torch.empty(N, dtype=torch.float32, device=dev)
-    Xq = torch.empty(M, K, dtype=torch.int8, device=dev)
-    x_scale = torch.empty(M, dtype=torch.float32, device=dev)
-    Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
-    ws_cal = torch.empty(sq.sq_calibrate_workspace_bytes(K), dtype=torch.uint8, device=dev)
-    ws_fwd = torch.empty(max(sq.sq_forward_workspace_bytes(M, N, K), 16), dtype=torch.uint8, device=dev)
-    ws_lin = torch.empty(max(sq.sq_workspace_bytes(M, N, K), 16), dtype=torch.uint8, device=dev)
+    T = {"C": d(inp["C"]), "W": d(inp["W"]), "X": d(inp["X"]),
+         "b": d(inp["bias"]) if inp["bias"] is not None else None,
+         "s": torch.empty(K, dtype=torch.float32, device=dev),
+         "Wq": torch.empty(N, K, dtype=torch.int8, device=dev),
+         "w_scale": torch.empty(N, dtype=torch.float32, device=dev),
+         "Xq": torch.empty(M, K, dtype=torch.int8, device=dev),
+         "x_scale": torch.empty(M, dtype=torch.float32, device=dev),
+         "Y": torch.empty(M, N, dtype=torch.bfloat16, device=dev),
+         "ws_cal": torch.empty(sq.sq_calibrate_workspace_bytes(K), dtype=torch.uint8, device=dev),
+         "ws_fwd": torch.empty(max(sq.sq_forward_workspace_bytes(M, N, K), 16), dtype=torch.uint8, device=dev),
+         "ws_lin": torch.empty(max(sq.sq_workspace_bytes(M, N, K), 16), dtype=torch.uint8, device=dev)}
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     flush_read = torch.ones(FLUSH_READ_BYTES // 4, dtype=torch.int32, device=dev)
+    a = wl.alpha_f32
+    fwd_launches = 1 if M <= FORWARD_FUSED_MAX_M else 2
 
     if args.path == "weight-only":
-        ones = torch.ones(K, dtype=torch.float32, device=dev)
+        T["ones"] = torch.ones(K, dtype=torch.float32, device=dev)
         calls = {
-            "sq_prepare_weight": lambda: sq.sq_prepare_weight(W, ones, Wq=Wq, w_scale=w_scale),
-            "sq_linear_weight_only": lambda: sq.sq_linear_weight_only(X, Wq, w_scale, b, Y=Y),
+            "sq_prepare_weight": Call(lambda T: sq.sq_prepare_weight(T["W"], T["ones"], Wq=T["Wq"],
+                                                                     w_scale=T["w_scale"]), ["W"], 1),
+            "sq_linear_weight_only": Call(lambda T: sq.sq_linear_weight_only(T["X"], T["Wq"], T["w_scale"], T["b"],
+                                                                             Y=T["Y"]),
+                                          ["X", "Wq", "w_scale", "b"], 1),
         }
-        launches_per_call = {"sq_prepare_weight": 1, "sq_linear_weight_only": 1}
+        stages = [["sq_prepare_weight"], ["sq_linear_weight_only"]]
     elif args.path == "ste-train":
         # the training step of the learnable-alpha layer: s recomputed from the
         # running activation max (taken once from the calibration batch) and
         # the weight, the forward, and the straight-through backward
-        G = d(train_gradient(wl))
-        mx = torch.empty(K, dtype=torch.float32, device=dev).zero_()
-        sq.sq_calibrate(C, W, wl.alpha_f32, s=s, mx_inout=mx, workspace=ws_cal)
-        dXg = torch.empty(M, K, dtype=torch.float32, device=dev)
-        dWg = torch.empty(N, K, dtype=torch.float32, device=dev)
-        dbg = torch.empty(N, dtype=torch.float32, device=dev) if b is not None else None
-        dsg = torch.empty(K, dtype=torch.float32, device=dev)
-        d_eta = torch.empty(1, dtype=torch.float32, device=dev)
-        ws_bwd = torch.empty(sq.sq_ste_backward_workspace_bytes(M, N, K), dtype=torch.uint8, device=dev)
+        T["G"] = d(train_gradient(wl))
+        T["mx"] = torch.zeros(K, dtype=torch.float32, device=dev)
+        sq.sq_calibrate(T["C"], T["W"], a, s=T["s"], mx_inout=T["mx"], workspace=T["ws_cal"])
+        T.update(dXg=torch.empty(M, K, dtype=torch.float32, device=dev),
+                 dWg=torch.empty(N, K, dtype=torch.float32, device=dev),
+                 dbg=torch.empty(N, dtype=torch.float32, device=dev) if T["b"] is not None else None,
+                 dsg=torch.empty(K, dtype=torch.float32, device=dev),
+                 d_eta=torch.empty(1, dtype=torch.float32, device=dev),
+                 ws_bwd=torch.empty(sq.sq_ste_backward_workspace_bytes(M, N, K), dtype=torch.uint8, device=dev))
+
+        def bwd(T):
+            sq.sq_ste_backward(T["G"], T["X"], T["W"], T["s"], T["mx"], a, T["Xq"], T["x_scale"], T["Wq"],
+                               T["w_scale"], with_db=T["b"] is not None, dX=T["dXg"], dW=T["dWg"], db=T["dbg"],
+                               ds=T["dsg"], d_eta=T["d_eta"], workspace=T["ws_bwd"])
         calls = {
-            "sq_calibrate(mx)": lambda: sq.sq_calibrate(None, W, wl.alpha_f32, s=s, mx_inout=mx, workspace=ws_cal),
-            "sq_prepare_weight": lambda: sq.sq_prepare_weight(W, s, Wq=Wq, w_scale=w_scale),
-            "sq_quantize_act": lambda: sq.sq_quantize_act(X, s, Xq=Xq, x_scale=x_scale),
-            "sq_linear": lambda: sq.sq_linear(Xq, x_scale, Wq, w_scale, b, Y=Y, workspace=ws_lin),
-            "sq_ste_backward": lambda: sq.sq_ste_backward(G, X, W, s, mx, wl.alpha_f32, Xq, x_scale, Wq, w_scale,
-                                                          with_db=b is not None, dX=dXg, dW=dWg, db=dbg, ds=dsg,
-                                                          d_eta=d_eta, workspace=ws_bwd),
+            "sq_calibrate(mx)": Call(lambda T: sq.sq_calibrate(None, T["W"], a, s=T["s"], mx_inout=T["mx"],
+                                                               workspace=T["ws_cal"]), ["W", "mx"], 2),
+            "sq_prepare_weight": Call(lambda T: sq.sq_prepare_weight(T["W"], T["s"], Wq=T["Wq"],
+                                                                     w_scale=T["w_scale"]), ["W"], 1),
+            "sq_quantize_act": Call(lambda T: sq.sq_quantize_act(T["X"], T["s"], Xq=T["Xq"], x_scale=T["x_scale"]),
+                                    ["X"], 1),
+            "sq_linear": Call(lambda T: sq.sq_linear(T["Xq"], T["x_scale"], T["Wq"], T["w_scale"], T["b"], Y=T["Y"],
+                                                     workspace=T["ws_lin"]), ["Xq", "Wq", "x_scale", "w_scale"], 1),
+            "sq_ste_backward": Call(bwd, ["G", "X", "W", "Xq", "Wq"], 7),
         }
-        launches_per_call = {"sq_calibrate(mx)": 2, "sq_prepare_weight": 1, "sq_quantize_act": 1, "sq_linear": 1,
-                             "sq_ste_backward": 7}
+        stages = [["sq_calibrate(mx)"], ["sq_prepare_weight", "sq_quantize_act"], ["sq_linear"],
+                  ["sq_ste_backward"]]
     elif args.path == "per-tensor":
-        ws_pt = torch.empty(sq.sq_quantize_per_tensor_workspace_bytes(), dtype=torch.uint8, device=dev)
-        ws_pt2 = torch.empty_like(ws_pt)
+        T["ws_pt"] = torch.empty(sq.sq_quantize_per_tensor_workspace_bytes(), dtype=torch.uint8, device=dev)
+        T["ws_pt2"] = torch.empty_like(T["ws_pt"])
         calls = {
-            "sq_quantize_per_tensor(W)": lambda: sq.sq_quantize_per_tensor(W, Aq=Wq, scale_rows=w_scale,
-                                                                           workspace=ws_pt),
-            "sq_quantize_per_tensor(X)": lambda: sq.sq_quantize_per_tensor(X, Aq=Xq, scale_rows=x_scale,
-                                                                           workspace=ws_pt2),
-            "sq_linear": lambda: sq.sq_linear(Xq, x_scale, Wq, w_scale, b, Y=Y, workspace=ws_lin),
+            "sq_quantize_per_tensor(W)": Call(lambda T: sq.sq_quantize_per_tensor(
+                T["W"], Aq=T["Wq"], scale_rows=T["w_scale"], workspace=T["ws_pt"]), ["W"], 2),
+            "sq_quantize_per_tensor(X)": Call(lambda T: sq.sq_quantize_per_tensor(
+                T["X"], Aq=T["Xq"], scale_rows=T["x_scale"], workspace=T["ws_pt2"]), ["X"], 2),
+            "sq_linear": Call(lambda T: sq.sq_linear(T["Xq"], T["x_scale"], T["Wq"], T["w_scale"], T["b"], Y=T["Y"],
+                                                     workspace=T["ws_lin"]), ["Xq", "Wq", "x_scale", "w_scale"], 1),
         }
-        launches_per_call = {"sq_quantize_per_tensor(W)": 2, "sq_quantize_per_tensor(X)": 2, "sq_linear": 1}
+        # measured slower side by side (41.4 against 40.5 us on proj): in order
+        stages = [["sq_quantize_per_tensor(W)"], ["sq_quantize_per_tensor(X)"], ["sq_linear"]]
+    elif args.path == "forward":
+        # weights prepared once; the timed calls are sq_forward alone
+        sq.sq_calibrate(T["C"], T["W"], a, s=T["s"], workspace=T["ws_cal"])
+        sq.sq_prepare_weight(T["W"], T["s"], Wq=T["Wq"], w_scale=T["w_scale"])
+        calls = {
+            "sq_forward": Call(lambda T: sq.sq_forward(T["X"], T["s"], T["Wq"], T["w_scale"], T["b"], Y=T["Y"],
+                                                       workspace=T["ws_fwd"]), ["Wq", "w_scale"], fwd_launches),
+        }
+        stages = [["sq_forward"]]
     else:
         calls = {
-            "sq_calibrate": lambda: sq.sq_calibrate(C, W, wl.alpha_f32, s=s, workspace=ws_cal),
-            "sq_prepare_weight": lambda: sq.sq_prepare_weight(W, s, Wq=Wq, w_scale=w_scale),
-            "sq_quantize_act": lambda: sq.sq_quantize_act(X, s, Xq=Xq, x_scale=x_scale),
-            "sq_linear": lambda: sq.sq_linear(Xq, x_scale, Wq, w_scale, b, Y=Y, workspace=ws_lin),
+            "sq_calibrate": Call(lambda T: sq.sq_calibrate(T["C"], T["W"], a, s=T["s"], workspace=T["ws_cal"]),
+                                 ["C", "W"], 2),  # a small kernel clears the workspace first
+            "sq_prepare_weight": Call(lambda T: sq.sq_prepare_weight(T["W"], T["s"], Wq=T["Wq"],
+                                                                     w_scale=T["w_scale"]), ["W"], 1),
+            "sq_quantize_act": Call(lambda T: sq.sq_quantize_act(T["X"], T["s"], Xq=T["Xq"], x_scale=T["x_scale"]),
+                                    ["X"], 1),
+            "sq_linear": Call(lambda T: sq.sq_linear(T["Xq"], T["x_scale"], T["Wq"], T["w_scale"], T["b"], Y=T["Y"],
+                                                     workspace=T["ws_lin"]), ["Xq", "Wq", "x_scale", "w_scale"], 1),
         }
-        # kernels per call: calibration clears its workspace with a small kernel first
-        launches_per_call = {"sq_calibrate": 2, "sq_prepare_weight": 1, "sq_quantize_act": 1, "sq_linear": 1}
+        stages = [["sq_calibrate"], ["sq_prepare_weight", "sq_quantize_act"], ["sq_linear"]]
     names = list(calls)
-    # the step's dependency stages: calls within a stage read only what the
-    # earlier stages wrote (the weight prep and the activation quantiser both
-    # need s alone), so they run on forked streams unless --serial
-    stages = {
-        "smoothquant": [["sq_calibrate"], ["sq_prepare_weight", "sq_quantize_act"], ["sq_linear"]],
-        # measured slower side by side (41.4 against 40.5 us on proj): in order
-        "per-tensor": [["sq_quantize_per_tensor(W)"], ["sq_quantize_per_tensor(X)"], ["sq_linear"]],
-        "ste-train": [["sq_calibrate(mx)"], ["sq_prepare_weight", "sq_quantize_act"], ["sq_linear"],
-                      ["sq_ste_backward"]],
-        "weight-only": [["sq_prepare_weight"], ["sq_linear_weight_only"]],
-    }[args.path]
+    launches_per_call = {n: calls[n].launches for n in names}
     assert sorted(n for st in stages for n in st) == sorted(names)
     side = [torch.cuda.Stream(device=dev) for _ in range(max(len(st) for st in stages) - 1)]
 
-    def run_step():
+    def run_step(T):
         main = torch.cuda.current_stream()
         for st in stages:
             if len(st) == 1 or args.serial:
                 for n in st:
-                    calls[n]()
+                    calls[n].fn(T)
                 continue
             fork = torch.cuda.Event()
             fork.record(main)
             for k, n in enumerate(st[1:]):
                 side[k].wait_event(fork)
                 with torch.cuda.stream(side[k]):
-                    calls[n]()
-            calls[st[0]]()
+                    calls[n].fn(T)
+            calls[st[0]].fn(T)
             for k in range(len(st) - 1):
                 join = torch.cuda.Event()
                 join.record(side[k])
                 main.wait_event(join)
 
-    # initialise library caches outside capture, then capture the step twice:
-    # as one graph with no nodes between the calls (the kernels overlap each
-    # other's launch through programmatic dependent launch, independent calls
-    # run side by side) for the step time, and with timing-event nodes
-    # between the calls for the per-call times.
-    for f in calls.values():
-        f()
+    # initialise library caches and the intermediate tensors outside capture
+    for n in names:
+        calls[n].fn(T)
     torch.cuda.synchronize()
+
+    # input copies for the L2-cold per-call timing: consecutive launches read
+    # different copies, whose inputs add up to >= ROTATE_BYTES
+    sets, rotations = {}, {}
+    for n in names:
+        foot = sum(nbytes(T[k]) for k in calls[n].reads)
+        r = rotation_count(foot)
+        lst = [T]
+        for _ in range(r - 1):
+            Ti = dict(T)
+            for k in calls[n].reads:
+                Ti[k] = None if T[k] is None else T[k].clone()
+            lst.append(Ti)
+        sets[n] = lst
+        rotations[n] = (r, r * foot >= ROTATE_BYTES)
+    torch.cuda.synchronize()
+
+    forward_path = args.path == "forward"
     step_evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)]
     g_step = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g_step):
-        step_evs[0].record()
-        run_step()
-        step_evs[1].record()
+    if forward_path:
+        # the K timed calls in one graph, each on the next prepared weight copy
+        fsets = sets["sq_forward"]
+        with torch.cuda.graph(g_step):
+            step_evs[0].record()
+            for k in range(args.steps):
+                calls["sq_forward"].fn(fsets[k % len(fsets)])
+            step_evs[1].record()
+        g_warm = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_warm):
+            for k in range(max(args.warmup, 1)):
+                calls["sq_forward"].fn(fsets[k % len(fsets)])
+    else:
+        with torch.cuda.graph(g_step):
+            step_evs[0].record()
+            run_step(T)
+            step_evs[1].record()
     call_evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(names) + 1)]
     g_calls = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g_calls):
         call_evs[0].record()
         for i, n in enumerate(names):
-            calls[n]()
+            calls[n].fn(T)
             call_evs[i + 1].record()
-    # and each call REPS times back to back between two event nodes: the span
-    # over REPS is that call's kernel duration with the launch latency of the
-    # event node amortised (consecutive launches chain through programmatic
-    # dependent launch, as in the step; the first launch after the flush reads
-    # its operands from HBM, the others find them in L2 -- as the step's later
-    # calls find theirs, written or read by the call before)
+    # each call back to back between two event nodes over its rotation: the
+    # span / launches is that call's kernel duration with the event node's
+    # launch latency amortised, every launch reading its inputs from HBM
     rep_evs = {n: [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)] for n in names}
+    reps = {n: max(REPS, len(sets[n])) for n in names}
     g_reps = {}
     for n in names:
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
             rep_evs[n][0].record()
-            for _ in range(REPS):
-                calls[n]()
+            for i in range(reps[n]):
+                calls[n].fn(sets[n][i % len(sets[n])])
             rep_evs[n][1].record()
         g_reps[n] = g
     torch.cuda.synchronize()
@@ -562,17 +733,17 @@ def run_ours(args, wl, rank, world, local_rank):
     if sampler:
         sampler.start()
     t_settle = time.perf_counter()
-    for _ in range(args.warmup):
+    for _ in range(1 if forward_path else args.warmup):
         flush_l2()
-        g_step.replay()
+        (g_warm if forward_path else g_step).replay()
         flush_l2()
         g_calls.replay()
     torch.cuda.synchronize()
     # keep the GPU under load briefly so the clock sampler sees steady clocks
     while time.perf_counter() - t_settle < args.settle_s:
-        for _ in range(50):
+        for _ in range(20):
             flush_l2()
-            g_step.replay()
+            (g_warm if forward_path else g_step).replay()
         torch.cuda.synchronize()
 
     if world > 1:
@@ -580,18 +751,24 @@ def run_ours(args, wl, rank, world, local_rank):
     torch.cuda.synchronize()
     step_times = []
     t_wall = time.perf_counter()
-    for k in range(args.steps):
+    if forward_path:
         flush_l2()
         g_step.replay()
-        torch.cuda.synchronize()  # the events are read before the next replay re-records them
-        step_times.append(step_evs[0].elapsed_time(step_evs[1]))
+        torch.cuda.synchronize()
+        step_times.append(step_evs[0].elapsed_time(step_evs[1]) / args.steps)
+    else:
+        for k in range(args.steps):
+            flush_l2()
+            g_step.replay()
+            torch.cuda.synchronize()  # the events are read before the next replay re-records them
+            step_times.append(step_evs[0].elapsed_time(step_evs[1]))
     wall = time.perf_counter() - t_wall
     if world > 1:
         dist.barrier()
-    # per-call device times (same flush, same buffers), for the roofline and the breakdown
+    # per-call device times (same flush, inputs rotated), for the roofline and the breakdown
     per_call_single = {n: 0.0 for n in names}
     per_call = {n: 0.0 for n in names}
-    rep_steps = max(1, min(args.steps, 1000))
+    rep_steps = max(1, min(args.steps, 20))
     for k in range(rep_steps):
         flush_l2()
         g_calls.replay()
@@ -602,7 +779,7 @@ def run_ours(args, wl, rank, world, local_rank):
             flush_l2()
             g_reps[n].replay()
             torch.cuda.synchronize()
-            per_call[n] += rep_evs[n][0].elapsed_time(rep_evs[n][1]) / REPS
+            per_call[n] += rep_evs[n][0].elapsed_time(rep_evs[n][1]) / reps[n]
     clocks = sampler.stop() if sampler else None
 
     mean_ms, median_ms = step_stats(step_times)
@@ -611,56 +788,79 @@ def run_ours(args, wl, rank, world, local_rank):
     per_call = {n: v / rep_steps for n, v in per_call.items()}
     per_call_single = {n: v / rep_steps for n, v in per_call_single.items()}
 
-    # correctness guard on the timed buffers (cheap; sq_forward path equals these calls)
+    # no bounded device wait may have run out during the timed work
     assert sq.sq_device_status() == 0, "device-side timeout flagged"
 
     # ------------------------------------------------------------- e2e leg
     stream = torch.cuda.current_stream()
     e2e = None
     if not args.no_e2e:
-        hC = torch.from_numpy(inp["C"].view(np.int16)).view(torch.bfloat16).pin_memory()
-        hW = torch.from_numpy(inp["W"].view(np.int16)).view(torch.bfloat16).pin_memory()
-        hX = torch.from_numpy(inp["X"].view(np.int16)).view(torch.bfloat16).pin_memory()
-        hb = torch.from_numpy(inp["bias"].view(np.int16)).view(torch.bfloat16).pin_memory() if b is not None else None
+        def pinned(bits):
+            return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).pin_memory()
+
+        hX = pinned(inp["X"])
         hY = torch.empty(M, N, dtype=torch.bfloat16).pin_memory()
-        dC, dW, dX = torch.empty_like(C), torch.empty_like(W), torch.empty_like(X)
-        db = torch.empty_like(b) if b is not None else None
+        D = dict(T)
+        D["X"] = torch.empty_like(T["X"])
+        ins = [hX]
+        if not forward_path:
+            hW = pinned(inp["W"])
+            D["W"] = torch.empty_like(T["W"])
+            ins.append(hW)
+        if args.path == "smoothquant":
+            hC = pinned(inp["C"])
+            D["C"] = torch.empty_like(T["C"])
+            ins.append(hC)
+        hb = None
+        if T["b"] is not None and not forward_path:
+            hb = pinned(inp["bias"])
+            D["b"] = torch.empty_like(T["b"])
+            ins.append(hb)
+        outs = [hY]
         if args.path == "ste-train":
-            hG = torch.from_numpy(train_gradient(wl).view(np.int16)).view(torch.bfloat16).pin_memory()
-            hmx = mx.cpu().pin_memory()
+            hG = pinned(train_gradient(wl))
+            hmx = T["mx"].cpu().pin_memory()
             h_eta = torch.empty(1, dtype=torch.float32).pin_memory()
-            dG, dmx = torch.empty_like(G), torch.empty_like(mx)
+            D["G"], D["mx"] = torch.empty_like(T["G"]), torch.empty_like(T["mx"])
+            ins += [hG, hmx]
+            outs.append(h_eta)
+        e2e_count = [0]
 
         def e2e_step():
+            D["X"].copy_(hX, non_blocking=True)
+            if not forward_path:
+                D["W"].copy_(hW, non_blocking=True)
             if args.path == "smoothquant":
-                dC.copy_(hC, non_blocking=True)
-            dW.copy_(hW, non_blocking=True)
-            dX.copy_(hX, non_blocking=True)
-            if db is not None:
-                db.copy_(hb, non_blocking=True)
+                D["C"].copy_(hC, non_blocking=True)
+            if hb is not None:
+                D["b"].copy_(hb, non_blocking=True)
             if args.path == "weight-only":
-                sq.sq_prepare_weight(dW, ones, Wq=Wq, w_scale=w_scale)
-                sq.sq_linear_weight_only(dX, Wq, w_scale, db, Y=Y)
+                sq.sq_prepare_weight(D["W"], D["ones"], Wq=D["Wq"], w_scale=D["w_scale"])
+                sq.sq_linear_weight_only(D["X"], D["Wq"], D["w_scale"], D["b"], Y=D["Y"])
             elif args.path == "ste-train":
-                dG.copy_(hG, non_blocking=True)
-                dmx.copy_(hmx, non_blocking=True)
-                sq.sq_calibrate(None, dW, wl.alpha_f32, s=s, mx_inout=dmx, workspace=ws_cal)
-                sq.sq_prepare_weight(dW, s, Wq=Wq, w_scale=w_scale)
-                sq.sq_quantize_act(dX, s, Xq=Xq, x_scale=x_scale)
-                sq.sq_linear(Xq, x_scale, Wq, w_scale, db, Y=Y, workspace=ws_lin)
-                sq.sq_ste_backward(dG, dX, dW, s, dmx, wl.alpha_f32, Xq, x_scale, Wq, w_scale,
-                                   with_db=db is not None, dX=dXg, dW=dWg, db=dbg, ds=dsg, d_eta=d_eta,
-                                   workspace=ws_bwd)
-                h_eta.copy_(d_eta, non_blocking=True)
+                D["G"].copy_(hG, non_blocking=True)
+                D["mx"].copy_(hmx, non_blocking=True)
+                sq.sq_calibrate(None, D["W"], a, s=D["s"], mx_inout=D["mx"], workspace=D["ws_cal"])
+                sq.sq_prepare_weight(D["W"], D["s"], Wq=D["Wq"], w_scale=D["w_scale"])
+                sq.sq_quantize_act(D["X"], D["s"], Xq=D["Xq"], x_scale=D["x_scale"])
+                sq.sq_linear(D["Xq"], D["x_scale"], D["Wq"], D["w_scale"], D["b"], Y=D["Y"], workspace=D["ws_lin"])
+                sq.sq_ste_backward(D["G"], D["X"], D["W"], D["s"], D["mx"], a, D["Xq"], D["x_scale"], D["Wq"],
+                                   D["w_scale"], with_db=D["b"] is not None, dX=D["dXg"], dW=D["dWg"], db=D["dbg"],
+                                   ds=D["dsg"], d_eta=D["d_eta"], workspace=D["ws_bwd"])
+                h_eta.copy_(D["d_eta"], non_blocking=True)
             elif args.path == "per-tensor":
-                sq.sq_quantize_per_tensor(dW, Aq=Wq, scale_rows=w_scale, workspace=ws_pt)
-                sq.sq_quantize_per_tensor(dX, Aq=Xq, scale_rows=x_scale, workspace=ws_pt2)
-                sq.sq_linear(Xq, x_scale, Wq, w_scale, db, Y=Y, workspace=ws_lin)
+                sq.sq_quantize_per_tensor(D["W"], Aq=D["Wq"], scale_rows=D["w_scale"], workspace=D["ws_pt"])
+                sq.sq_quantize_per_tensor(D["X"], Aq=D["Xq"], scale_rows=D["x_scale"], workspace=D["ws_pt2"])
+                sq.sq_linear(D["Xq"], D["x_scale"], D["Wq"], D["w_scale"], D["b"], Y=D["Y"], workspace=D["ws_lin"])
+            elif forward_path:
+                F = sets["sq_forward"][e2e_count[0] % len(sets["sq_forward"])]
+                sq.sq_forward(D["X"], F["s"], F["Wq"], F["w_scale"], F["b"], Y=D["Y"], workspace=D["ws_fwd"])
             else:
-                sq.sq_calibrate(dC, dW, wl.alpha_f32, s=s, workspace=ws_cal)
-                sq.sq_prepare_weight(dW, s, Wq=Wq, w_scale=w_scale)
-                sq.sq_forward(dX, s, Wq, w_scale, db, Y=Y, workspace=ws_fwd)
-            hY.copy_(Y, non_blocking=True)
+                sq.sq_calibrate(D["C"], D["W"], a, s=D["s"], workspace=D["ws_cal"])
+                sq.sq_prepare_weight(D["W"], D["s"], Wq=D["Wq"], w_scale=D["w_scale"])
+                sq.sq_forward(D["X"], D["s"], D["Wq"], D["w_scale"], D["b"], Y=D["Y"], workspace=D["ws_fwd"])
+            hY.copy_(D["Y"], non_blocking=True)
+            e2e_count[0] += 1
 
         for _ in range(3):
             e2e_step()
@@ -674,54 +874,43 @@ def run_ours(args, wl, rank, world, local_rank):
         e1.record(stream)
         torch.cuda.synchronize()
         e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, world, dev)
-        if args.path == "ste-train":
-            ins = (hW, hX, hG, hmx) + ((hb,) if hb is not None else ())
-            outs = (hY, h_eta)
-            call = ("sq_calibrate(mx) + sq_prepare_weight + sq_quantize_act + sq_linear + sq_ste_backward, "
-                    "Y and d eta read back")
-        elif args.path == "weight-only":
-            ins = (hW, hX) + ((hb,) if hb is not None else ())
-            outs = (hY,)
-            call = "sq_prepare_weight (s = 1) + sq_linear_weight_only"
-        else:
-            ins = ((hC,) if args.path == "smoothquant" else ()) + (hW, hX) + ((hb,) if hb is not None else ())
-            outs = (hY,)
-            call = ("sq_quantize_per_tensor(W) + sq_quantize_per_tensor(X) + sq_linear"
-                    if args.path == "per-tensor" else "sq_calibrate + sq_prepare_weight + sq_forward")
+        call = {"ste-train": "sq_calibrate(mx) + sq_prepare_weight + sq_quantize_act + sq_linear + "
+                             "sq_ste_backward, Y and d eta read back",
+                "weight-only": "sq_prepare_weight (s = 1) + sq_linear_weight_only",
+                "per-tensor": "sq_quantize_per_tensor(W) + sq_quantize_per_tensor(X) + sq_linear",
+                "forward": "sq_forward on a prepared weight (X in, Y out)",
+                "smoothquant": "sq_calibrate + sq_prepare_weight + sq_forward"}[args.path]
         e2e = {"value": whole_job_rate(wl.M, world, e2e_ms), "unit": UNIT,
-               "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in ins),
-               "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in outs), "ms_per_step": e2e_ms,
-               "call": call}
+               "h2d_bytes_per_step": sum(nbytes(t) for t in ins),
+               "d2h_bytes_per_step": sum(nbytes(t) for t in outs), "ms_per_step": e2e_ms, "call": call}
 
     if rank != 0:
         return
 
-    kernels, roof = kernel_report(wl, names, per_call, per_call_single, launches_per_call)
+    kernels, roof = kernel_report(wl, names, per_call, per_call_single, launches_per_call, rotations)
 
     cpu = None
     if not args.no_cpu_baseline and world == 1:
-        v, n, el = cpu_oracle_rate(wl, args.cpu_seconds, path=args.path)
-        what = {"per-tensor": "quantise W and X per tensor, product",
-                "weight-only": "quantise W per output channel, bf16 x int8 product",
-                "ste-train": "s from the running max, fold+quantise W, forward, straight-through backward"}
+        v, n, el = cpu_oracle_rate(wl, args.cpu_seconds, path=args.path, inp=inp)
         cpu = {"value": v, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
-               "sample": f"{n} whole {wl.name} steps in {el:.1f} s ("
-                         + what.get(args.path, "calibrate, fold+quantise W, forward") + ")"}
+               "sample": f"{n} {oracle_sample_text(wl, args.path)}; {el:.1f} s of CPU work"}
 
     value = whole_job_rate(wl.M, world, step_ms)
+    cfg = workload_config(wl, args.path)
+    if not forward_path:
+        cfg["schedule"] = ("serial" if args.serial else
+                           " -> ".join("(" + " | ".join(st) + ")" if len(st) > 1 else st[0] for st in stages))
+    gemm_call = next((n for n in ("sq_linear", "sq_forward", "sq_linear_weight_only") if n in per_call), None)
     line = {
         "metric": metric_for(args.path), "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": step_ms, "ms_per_step_median": step_median_ms,
         "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "int8", "data": "synthetic",
-        "config": dict(workload_config(wl, args.path),
-                       schedule="serial" if args.serial else
-                       " -> ".join("(" + " | ".join(st) + ")" if len(st) > 1 else st[0] for st in stages)),
+        "config": cfg,
         "tops_per_step": 2.0 * wl.M * wl.N * wl.K * world / (step_ms * 1e-3) / 1e12,
-        "gemm_tops": 2 * wl.M * wl.N * wl.K / (per_call.get("sq_linear", per_call.get("sq_linear_weight_only"))
-                                                * 1e-3) / 1e12,
+        "gemm_tops": 2 * wl.M * wl.N * wl.K / (per_call[gemm_call] * 1e-3) / 1e12 if gemm_call else None,
         "roofline": roof, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
-        "gpu_launches": args.steps * sum(launches_per_call.values()),  # the timed step replays
+        "gpu_launches": args.steps * sum(launches_per_call.values()),  # the timed steps
         "clocks": clocks, "wall_s_timed": wall,
     }
     print(json.dumps(line), flush=True)

@@ -306,6 +306,9 @@ SQ_API sq_status sq_gemm_s32(const int8_t* Xq, const int8_t* Wq, int64_t M, int6
  * quantisation kernels) timed out; the results of that call are undefined.
  * Synchronises the device.  Returns SQ_ERR_TIMEOUT if any bit is set.
  * Clearing a set status also re-zeroes the scratch of sq_calibrate_noalloc.
+ * Both the read and the clear apply to the CURRENT device only: a timed-out
+ * call on another device stays flagged (and its no-allocation scratch dirty)
+ * until that device is made current and its status cleared.
  */
 SQ_API sq_status sq_device_status(uint32_t* flags, int clear);
 

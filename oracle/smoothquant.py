@@ -13,7 +13,7 @@ alpha APRENDIVEL (V5)" (module docstring "Algoritmo", functions
 methods ``SmoothQuantW8A8.calibrate`` / ``freeze_quantization`` / ``forward``
 / ``quantization_error``).
 
-Precision, per step (the readings are listed in the design doc as well):
+Precision, per step:
 
 * Inputs are bf16 bit patterns, widened exactly.
 * Max-abs reductions are exact (a max of exactly representable values).

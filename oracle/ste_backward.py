@@ -35,7 +35,7 @@ where raw_j = mx_j^alpha / mw_j^(1-alpha) before the clamp, mx and mw
 clamped at 1e-8 (the clamp's gradient passes where its input is at or above
 the floor).
 
-Readings (listed in DESIGN.md as well):
+Readings:
 
 * The forward values are those of the inference path: s, (Wq, w_scale) and
   (Xq, x_scale) come from ``oracle.smoothquant`` (the page's fp32 steps), so

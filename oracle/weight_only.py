@@ -11,7 +11,7 @@ is taken against the int8 weight codes and then multiplied by the
 per-output-channel weight scale, and the bias is added:
 ``y[m][n] = (sum_k x[m][k] * Wq[n][k]) * w_scale[n] + bias[n]``.
 
-Readings (listed in DESIGN.md as well):
+Readings:
 
 * The weight is quantised per output channel, symmetric to +-127, by the
   SmoothQuant page's ``quantize_per_channel_symmetric`` (``sq_prepare_weight``

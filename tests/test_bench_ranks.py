@@ -56,7 +56,7 @@ def test_reference_arm_runs_on_rank_zero_only(capsys):
     assert capsys.readouterr().out == ""
 
 
-@pytest.mark.parametrize("path", ["smoothquant", "per-tensor", "ste-train", "weight-only"])
+@pytest.mark.parametrize("path", ["smoothquant", "forward", "per-tensor", "ste-train", "weight-only"])
 def test_reference_arm_line_on_rank_zero(capsys, path):
     """The reference arm (the CPU oracle) prints one JSON line per run with
     the keys the driver reads, for every bench path."""

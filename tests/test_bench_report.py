@@ -62,12 +62,15 @@ def test_other_paths_take_their_own_peaks():
     assert k["bound"] == "tensor" and k["operands"] == "bf16"
     assert abs(k["int8_peak_tops"] - bf16) < 1e-9
     assert abs(k["achieved_tops"] - 4 * 2048 * 11008 * 4096 / 300e-6 / 1e12) < 1e-6
-    # at proj size the backward's bytes take (slightly) longer than its products
+    # at proj size the backward's bytes and products take about as long: the
+    # bound is whichever roofline is the longer at the peaks in use
     wl = workloads.get("proj")
     kernels, roof = bench.kernel_report(wl, names, {"sq_linear": 0.0125, "sq_ste_backward": 0.1},
                                         {"sq_linear": 0.0125, "sq_ste_backward": 0.1},
                                         {"sq_linear": 1, "sq_ste_backward": 7})
-    assert roof["kernel"] == "sq_ste_backward" and roof["bound"] == "hbm"
+    nb, ops, _ = bench.algorithmic_work(wl)["sq_ste_backward"]
+    want = "hbm" if nb / (hbm * 1e9) >= ops / (bf16 * 1e12) else "tensor"
+    assert roof["kernel"] == "sq_ste_backward" and roof["bound"] == want
     wl = workloads.get("decode")
     names = ["sq_prepare_weight", "sq_linear_weight_only"]
     per = {"sq_prepare_weight": 0.0115, "sq_linear_weight_only": 0.054}
@@ -75,3 +78,45 @@ def test_other_paths_take_their_own_peaks():
     assert roof["bound"] == "alu" and roof["kernel"] == "sq_linear_weight_only"
     assert abs(roof["peak"] - 148 * 128 * 2 * 1.965e9 / 1e12) < 1e-9
     assert abs(roof["frac"] - 2 * 8 * 8192 * 8192 / 54e-6 / 1e12 / roof["peak"]) < 1e-9
+
+
+def test_headline_defaults():
+    """With no flags the bench times the largest layer (prefill) on the whole
+    path; the decode layer defaults to the per-call forward on prepared,
+    rotated weights."""
+    a = bench.parse_args([])
+    assert a.workload == "prefill" and a.path == "smoothquant" and a.warmup >= 3
+    assert bench.parse_args(["--workload", "decode"]).path == "forward"
+    assert bench.parse_args(["--workload", "decode", "--path", "smoothquant"]).path == "smoothquant"
+    wl = workloads.get("decode")
+    r = bench.forward_rotation(wl)
+    assert r >= 4 and r * wl.N * wl.K >= 256 << 20
+
+
+def test_rotation_makes_inputs_exceed_l2():
+    assert bench.rotation_count(600 << 20) == 1
+    assert bench.rotation_count(128 << 20) == 2
+    assert bench.rotation_count(36 << 20) * (36 << 20) >= 256 << 20
+    assert bench.rotation_count(1) == bench.MAX_ROTATION
+
+
+def test_oracle_sample_plan():
+    """Smaller layers run whole oracle steps; the prefill layer is sampled
+    (and the sample text says how it is extrapolated)."""
+    for name in ("tiny", "proj", "mlp", "decode"):
+        wl = workloads.get(name)
+        assert bench.sample_plan(wl, "smoothquant") == (wl.M, wl.N)
+        assert "whole" in bench.oracle_sample_text(wl, "smoothquant")
+    wl = workloads.get("prefill")
+    mx, mw = bench.sample_plan(wl, "smoothquant")
+    assert mx < wl.M and mw < wl.N
+    assert "extrapolated" in bench.oracle_sample_text(wl, "smoothquant")
+
+
+def test_forward_work_counts_the_weight_stream():
+    wl = workloads.get("decode")
+    nb, ops, typ = bench.algorithmic_work(wl)["sq_forward"]
+    assert nb >= wl.N * wl.K and ops == 2 * wl.M * wl.N * wl.K and typ == "int8"
+    kernels, roof = bench.kernel_report(wl, ["sq_forward"], {"sq_forward": 0.012}, {"sq_forward": 0.018},
+                                        {"sq_forward": 1})
+    assert roof["bound"] == "hbm" and roof["kernel"] == "sq_forward"

@@ -15,6 +15,7 @@ import pytest
 import torch
 
 import workloads
+from oracle import smoothquant as O
 from tests.helpers import assert_scales_close, dev_bf16, host
 
 pytestmark = pytest.mark.gpu
@@ -46,27 +47,35 @@ def test_noalloc_matches_workspace_calibration_on_consecutive_calls(sq):
     C1, W = dev_bf16(inp["C"]), dev_bf16(inp["W"])
     # second batch: same shape, no outlier channels, so every column max is
     # smaller than in the first -- stale maxima from call 1 would show up in s
-    C2 = dev_bf16(workloads.random_bf16((wl.R, wl.K), seed=777))
+    C2_bits = workloads.random_bf16((wl.R, wl.K), seed=777)
+    C2 = dev_bf16(C2_bits)
     K = wl.K
-    for C in (C1, C2):                                   # two calls in a row
+    for C, C_bits in ((C1, inp["C"]), (C2, C2_bits)):   # two calls in a row
         s_ref = sq.sq_calibrate(C, W, wl.alpha_f32)      # existing entry point (workspace)
         s = torch.empty(K, dtype=torch.float32, device="cuda")
         assert _noalloc(sq, C, W, wl.alpha_f32, s) == SQ_OK, sq.lib.sq_last_error()
         torch.cuda.synchronize()
         assert_scales_close(host(s), host(s_ref), "sq_calibrate_noalloc vs sq_calibrate")
+        # and against the CPU oracle on the same bf16 inputs
+        s_o, _ = O.calibrate(C_bits, inp["W"], wl.alpha_f32)
+        assert_scales_close(host(s), s_o, "sq_calibrate_noalloc vs the oracle")
     # with the running max, twice more (tiny layer, different K)
     wt = workloads.get("tiny")
     it = workloads.make_inputs(wt, ("C", "W"))
     Ct, Wt = dev_bf16(it["C"]), dev_bf16(it["W"])
     mx_a = torch.zeros(wt.K, dtype=torch.float32, device="cuda")
     mx_b = torch.zeros(wt.K, dtype=torch.float32, device="cuda")
-    for half in (Ct[:32], Ct[32:]):
+    mx_o = None
+    for half, lo, hi in ((Ct[:32], 0, 32), (Ct[32:], 32, None)):
         s_ref = sq.sq_calibrate(half, Wt, wt.alpha_f32, mx_inout=mx_a)
         s = torch.empty(wt.K, dtype=torch.float32, device="cuda")
         assert _noalloc(sq, half, Wt, wt.alpha_f32, s, mx_b) == SQ_OK, sq.lib.sq_last_error()
         torch.cuda.synchronize()
         assert_scales_close(host(s), host(s_ref), "noalloc with running max")
         assert np.array_equal(host(mx_a), host(mx_b))
+        s_o, mx_o = O.calibrate(it["C"][lo:hi], it["W"], wt.alpha_f32, mx_prev=mx_o)
+        assert_scales_close(host(s), s_o, "noalloc with running max vs the oracle")
+        assert np.array_equal(host(mx_b), mx_o)
 
 
 def test_noalloc_rejects_k_beyond_its_scratch(sq):
