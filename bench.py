@@ -792,54 +792,48 @@ def run_ours(args, wl, rank, world, local_rank):
     assert sq.sq_device_status() == 0, "device-side timeout flagged"
 
     # ------------------------------------------------------------- e2e leg
-    stream = torch.cuda.current_stream()
+    # Through the Python binding, every step's inputs copied in from pinned
+    # host memory and its Y (and d eta) copied out.  Two device buffer sets
+    # and three streams pipeline the steps: the copy-in of step i+1 and the
+    # copy-out of step i-1 overlap the kernels of step i (the copy engines and
+    # the SMs work side by side, as a serving loop would run them).
     e2e = None
     if not args.no_e2e:
         def pinned(bits):
             return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).pin_memory()
 
         hX = pinned(inp["X"])
-        hY = torch.empty(M, N, dtype=torch.bfloat16).pin_memory()
-        D = dict(T)
-        D["X"] = torch.empty_like(T["X"])
-        ins = [hX]
-        if not forward_path:
-            hW = pinned(inp["W"])
-            D["W"] = torch.empty_like(T["W"])
-            ins.append(hW)
-        if args.path == "smoothquant":
-            hC = pinned(inp["C"])
-            D["C"] = torch.empty_like(T["C"])
-            ins.append(hC)
-        hb = None
-        if T["b"] is not None and not forward_path:
-            hb = pinned(inp["bias"])
-            D["b"] = torch.empty_like(T["b"])
-            ins.append(hb)
-        outs = [hY]
-        if args.path == "ste-train":
-            hG = pinned(train_gradient(wl))
-            hmx = T["mx"].cpu().pin_memory()
-            h_eta = torch.empty(1, dtype=torch.float32).pin_memory()
-            D["G"], D["mx"] = torch.empty_like(T["G"]), torch.empty_like(T["mx"])
-            ins += [hG, hmx]
-            outs.append(h_eta)
-        e2e_count = [0]
+        hW = pinned(inp["W"]) if not forward_path else None
+        hC = pinned(inp["C"]) if args.path == "smoothquant" else None
+        hb = pinned(inp["bias"]) if (T["b"] is not None and not forward_path) else None
+        hG = pinned(train_gradient(wl)) if args.path == "ste-train" else None
+        hmx = T["mx"].cpu().pin_memory() if args.path == "ste-train" else None
+        host_in = {"X": hX, "W": hW, "C": hC, "b": hb, "G": hG, "mx": hmx}
+        host_in = {k: v for k, v in host_in.items() if v is not None}
+        bufs, h_out = [], []
+        for _ in range(2):
+            D = dict(T)
+            for k in host_in:
+                D[k] = torch.empty_like(T[k])
+            D["Y"] = torch.empty_like(T["Y"])
+            if args.path == "ste-train":
+                D["d_eta"] = torch.empty_like(T["d_eta"])
+            bufs.append(D)
+            h_out.append({"Y": torch.empty(M, N, dtype=torch.bfloat16).pin_memory(),
+                          "d_eta": torch.empty(1, dtype=torch.float32).pin_memory()})
+        s_in, s_comp, s_out = (torch.cuda.Stream(device=dev) for _ in range(3))
+        ev_in = [torch.cuda.Event() for _ in range(2)]
+        ev_comp = [torch.cuda.Event() for _ in range(2)]
+        ev_out = [torch.cuda.Event() for _ in range(2)]
+        for b_ in range(2):  # nothing pending on either buffer set at the start
+            ev_comp[b_].record(s_comp)
+            ev_out[b_].record(s_out)
 
-        def e2e_step():
-            D["X"].copy_(hX, non_blocking=True)
-            if not forward_path:
-                D["W"].copy_(hW, non_blocking=True)
-            if args.path == "smoothquant":
-                D["C"].copy_(hC, non_blocking=True)
-            if hb is not None:
-                D["b"].copy_(hb, non_blocking=True)
+        def compute(D, i):
             if args.path == "weight-only":
                 sq.sq_prepare_weight(D["W"], D["ones"], Wq=D["Wq"], w_scale=D["w_scale"])
                 sq.sq_linear_weight_only(D["X"], D["Wq"], D["w_scale"], D["b"], Y=D["Y"])
             elif args.path == "ste-train":
-                D["G"].copy_(hG, non_blocking=True)
-                D["mx"].copy_(hmx, non_blocking=True)
                 sq.sq_calibrate(None, D["W"], a, s=D["s"], mx_inout=D["mx"], workspace=D["ws_cal"])
                 sq.sq_prepare_weight(D["W"], D["s"], Wq=D["Wq"], w_scale=D["w_scale"])
                 sq.sq_quantize_act(D["X"], D["s"], Xq=D["Xq"], x_scale=D["x_scale"])
@@ -847,42 +841,67 @@ def run_ours(args, wl, rank, world, local_rank):
                 sq.sq_ste_backward(D["G"], D["X"], D["W"], D["s"], D["mx"], a, D["Xq"], D["x_scale"], D["Wq"],
                                    D["w_scale"], with_db=D["b"] is not None, dX=D["dXg"], dW=D["dWg"], db=D["dbg"],
                                    ds=D["dsg"], d_eta=D["d_eta"], workspace=D["ws_bwd"])
-                h_eta.copy_(D["d_eta"], non_blocking=True)
             elif args.path == "per-tensor":
                 sq.sq_quantize_per_tensor(D["W"], Aq=D["Wq"], scale_rows=D["w_scale"], workspace=D["ws_pt"])
                 sq.sq_quantize_per_tensor(D["X"], Aq=D["Xq"], scale_rows=D["x_scale"], workspace=D["ws_pt2"])
                 sq.sq_linear(D["Xq"], D["x_scale"], D["Wq"], D["w_scale"], D["b"], Y=D["Y"], workspace=D["ws_lin"])
             elif forward_path:
-                F = sets["sq_forward"][e2e_count[0] % len(sets["sq_forward"])]
+                F = sets["sq_forward"][i % len(sets["sq_forward"])]
                 sq.sq_forward(D["X"], F["s"], F["Wq"], F["w_scale"], F["b"], Y=D["Y"], workspace=D["ws_fwd"])
             else:
                 sq.sq_calibrate(D["C"], D["W"], a, s=D["s"], workspace=D["ws_cal"])
                 sq.sq_prepare_weight(D["W"], D["s"], Wq=D["Wq"], w_scale=D["w_scale"])
                 sq.sq_forward(D["X"], D["s"], D["Wq"], D["w_scale"], D["b"], Y=D["Y"], workspace=D["ws_fwd"])
-            hY.copy_(D["Y"], non_blocking=True)
-            e2e_count[0] += 1
 
-        for _ in range(3):
-            e2e_step()
+        def e2e_step(i):
+            b_ = i % 2
+            D, H = bufs[b_], h_out[b_]
+            with torch.cuda.stream(s_in):
+                s_in.wait_event(ev_comp[b_])      # step i-2 has finished reading these inputs
+                for k, h in host_in.items():
+                    D[k].copy_(h, non_blocking=True)
+                ev_in[b_].record(s_in)
+            with torch.cuda.stream(s_comp):
+                s_comp.wait_event(ev_in[b_])
+                s_comp.wait_event(ev_out[b_])     # step i-2's Y has been copied out
+                compute(D, i)
+                ev_comp[b_].record(s_comp)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_comp[b_])
+                H["Y"].copy_(D["Y"], non_blocking=True)
+                if args.path == "ste-train":
+                    H["d_eta"].copy_(D["d_eta"], non_blocking=True)
+                ev_out[b_].record(s_out)
+
+        for i in range(3):
+            e2e_step(i)
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(args.e2e_steps):
-            e2e_step()
-        e1.record(stream)
+        e0.record(s_in)
+        for i in range(args.e2e_steps):
+            e2e_step(3 + i)
+        for b_ in range(2):
+            s_out.wait_event(ev_out[b_])
+        e1.record(s_out)
         torch.cuda.synchronize()
         e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, world, dev)
+        # the copies of the last step agree with the device result
+        assert torch.equal(h_out[(2 + args.e2e_steps) % 2]["Y"].view(torch.int16),
+                           bufs[(2 + args.e2e_steps) % 2]["Y"].cpu().view(torch.int16))
         call = {"ste-train": "sq_calibrate(mx) + sq_prepare_weight + sq_quantize_act + sq_linear + "
                              "sq_ste_backward, Y and d eta read back",
                 "weight-only": "sq_prepare_weight (s = 1) + sq_linear_weight_only",
                 "per-tensor": "sq_quantize_per_tensor(W) + sq_quantize_per_tensor(X) + sq_linear",
                 "forward": "sq_forward on a prepared weight (X in, Y out)",
                 "smoothquant": "sq_calibrate + sq_prepare_weight + sq_forward"}[args.path]
+        outs = [h_out[0]["Y"]] + ([h_out[0]["d_eta"]] if args.path == "ste-train" else [])
         e2e = {"value": whole_job_rate(wl.M, world, e2e_ms), "unit": UNIT,
-               "h2d_bytes_per_step": sum(nbytes(t) for t in ins),
-               "d2h_bytes_per_step": sum(nbytes(t) for t in outs), "ms_per_step": e2e_ms, "call": call}
+               "h2d_bytes_per_step": sum(nbytes(t) for t in host_in.values()),
+               "d2h_bytes_per_step": sum(nbytes(t) for t in outs), "ms_per_step": e2e_ms, "call": call,
+               "pipelined": "two buffer sets, three streams: copy-in of step i+1 and copy-out of step i-1 "
+                            "overlap the kernels of step i"}
 
     if rank != 0:
         return

@@ -103,6 +103,8 @@ def test_workload_stage_parity(sq, name):
     (33, 256, 512, True),       # just above the few-token path
     (40, 96, 16384, False),     # largest K: eight warps per row in the row quantisers
     (3, 64, 16384, True),       # largest K on the few-token path
+    (2056, 8200, 4112, True),   # 256 x 256 tiles on CTA pairs: ragged M, N and K blocks
+    (200, 19004, 1024, False),  # CTA pairs with one m-block (the odd CTA's rows partly past M), scalar stores
 ])
 def test_ragged_shapes(sq, M, N, K, with_bias):
     rng = np.random.default_rng(M * 7919 + N * 31 + K)
@@ -132,7 +134,8 @@ def test_zero_rows_and_floor(sq):
     assert np.array_equal(host(Xq), Xq_o) and np.array_equal(host(xs), xs_o)
 
 
-def test_tiny_values_and_subnormal_quotients(sq):
+@pytest.mark.parametrize("K", [256, 4096])  # both row quantisers: register prefetch and bulk-copy ring
+def test_tiny_values_and_subnormal_quotients(sq, K):
     """Values near the bottom of the fp32 range: X / s and W * s below 2^-126
     (subnormal quotients and products), rows whose maximum sits on the 1e-8
     floor, and rows mixing normal values with subnormal quotients.  The
@@ -141,7 +144,7 @@ def test_tiny_values_and_subnormal_quotients(sq):
     quotient is below the smallest scale fl(1e-8 / 127) by more than 2^80, so
     its code is 0 whatever its last bit, and a row maximum on the floor is
     1e-8 exactly.  Codes and scales must equal the oracle's."""
-    K, M = 256, 8
+    M = 8
     rng = np.random.default_rng(99)
     s = np.ones(K, np.float32)
     s[:64] = np.float32(2.0 ** 40)          # X / s of moderate X lands near 2^-126

@@ -73,3 +73,29 @@ def test_split_k_wait_timeout_is_reported_and_the_context_survives(sq):
     torch.cuda.synchronize()
     assert_y_close(host_bf16_bits(Y), O.int8_gemm(Xq, Wq), xs, ws, None, "split-K after a timeout")
     assert sq.sq_device_status() == 0
+
+
+def test_cta_pair_wait_timeout_is_reported_and_the_context_survives(sq):
+    """The same failure in the CTA-pair GEMM (256 x 256 tiles shared by the two
+    CTAs of a cluster): both producers skip their first stage, every wait of
+    both CTAs gives up, and the pair meets at its closing cluster barrier."""
+    rng = np.random.default_rng(97)
+    M, N, K = 2048, 9472, 1024  # 8 x 37 pair tiles: more than one per pair
+    Xq = rng.integers(-127, 128, (M, K), dtype=np.int64).astype(np.int8)
+    Wq = rng.integers(-127, 128, (N, K), dtype=np.int64).astype(np.int8)
+    Xq_d, Wq_d = dev(Xq), dev(Wq)
+    assert sq.sq_device_status(clear=True) == 0
+    try:
+        sq.sq_debug_pipeline_stall(True, 50_000_000)
+        t0 = time.perf_counter()
+        sq.sq_gemm_s32(Xq_d, Wq_d)
+        torch.cuda.synchronize()
+        elapsed = time.perf_counter() - t0
+    finally:
+        sq.sq_debug_pipeline_stall(False)
+    flags = sq.sq_device_status(clear=True)
+    assert flags & 1, "the stalled pair pipeline was not reported"
+    assert elapsed < 5.0
+    acc = host(sq.sq_gemm_s32(Xq_d, Wq_d))
+    assert np.array_equal(acc.astype(np.int64), O.int8_gemm(Xq, Wq))
+    assert sq.sq_device_status() == 0

@@ -62,6 +62,9 @@ constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // 2 s per wait
 #ifndef SQ_GEMM_SPLITK  // 1: split K over a CTA pair when 128 x 256 tiles fill at most half the SMs
 #define SQ_GEMM_SPLITK 1
 #endif
+#ifndef SQ_GEMM_PAIR  // 1: 256 x 256 tiles on CTA pairs (cta_group::2) when they fill every pair
+#define SQ_GEMM_PAIR 0
+#endif
 #ifndef SQ_GEMM_CHAINS128  // accumulator chains for 128-wide tiles (1 or 2)
 #define SQ_GEMM_CHAINS128 2
 #endif
@@ -80,11 +83,27 @@ __device__ __forceinline__ int k_start(int m_blk, int n_blk, int nk) {
 #endif
 }
 
+// Output tile `tile` of a persistent GEMM -> (m block, n block).  Tiles run
+// in groups of `group_m` m-blocks: within a group the m-blocks turn fastest
+// and the group sweeps every n-block before the next group starts, so the
+// tiles in flight at any moment share a few Wq slices and the group's Xq rows
+// (group_m * BM * K bytes, sized to stay in L2) are fetched from DRAM once.
+__device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int group_m, int& m_blk, int& n_blk) {
+  const int per_group = group_m * num_n;
+  const int g = tile / per_group;
+  const int first_m = g * group_m;
+  const int gm = min(group_m, num_m - first_m);  // the last group may be narrower
+  const int r = tile - g * per_group;
+  m_blk = first_m + r % gm;
+  n_blk = r / gm;
+}
+
 struct KParams {
   unsigned long long timeout_ns;  // limit of every mbarrier wait
   int skip_first_load;            // test hook: the producer never loads the first stage
   int M, N, K;
   int num_m_blocks, num_n_blocks, num_k_blocks;
+  int group_m;                    // m-blocks per tile group (tile_coords)
   const float* x_scale;
   const float* w_scale;
   const uint16_t* bias;
@@ -209,7 +228,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto prefetch_upto = [&](int64_t limit) {
         for (; pf < limit && pf < total; ++pf) {
           const int t = static_cast<int>(blockIdx.x) + static_cast<int>(pf / nk) * static_cast<int>(gridDim.x);
-          const int mb = t % p.num_m_blocks, nb = t / p.num_m_blocks;
+          int mb, nb;
+          tile_coords(t, p.num_m_blocks, p.num_n_blocks, p.group_m, mb, nb);
           int k = static_cast<int>(pf % nk) + k_start(mb, nb, nk);
           if (k >= nk) k -= nk;
           if (SQ_GEMM_PF_A) tma_prefetch_l2_2d(&tmA, k * kBK, mb * kBM);
@@ -219,8 +239,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (kPrefetchAhead > 0) prefetch_upto(kPrefetchAhead);
       int64_t seq = 0;
       for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
-        const int m_blk = tile % p.num_m_blocks;
-        const int n_blk = tile / p.num_m_blocks;
+        int m_blk, n_blk;
+        tile_coords(tile, p.num_m_blocks, p.num_n_blocks, p.group_m, m_blk, n_blk);
         const int k0 = k_start(m_blk, n_blk, nk);
         for (int kb = 0; kb < nk; ++kb, ++seq) {
           if (kPrefetchAhead > 0) prefetch_upto(seq + 1 + kPrefetchAhead);
@@ -318,8 +338,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
       const int acc = it & 1;
       const uint32_t acc_phase = (it >> 1) & 1;
-      const int m_blk = tile % p.num_m_blocks;
-      const int n_blk = tile / p.num_m_blocks;
+      int m_blk, n_blk;
+      tile_coords(tile, p.num_m_blocks, p.num_n_blocks, p.group_m, m_blk, n_blk);
       const int row = m_blk * kBM + quarter * 32 + lane;
       const bool row_ok = row < p.M;
       float xs = 0.0f;
@@ -432,6 +452,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 namespace sq {
 namespace {
+#include "sq_gemm_pair.cuh"
+}  // namespace
+}  // namespace sq
+
+namespace sq {
+namespace {
 
 // ----------------------------------------------------------- host helpers
 // test hook state (sq_debug_pipeline_stall)
@@ -470,6 +496,18 @@ bool make_tmap_i8(CUtensorMap* map, const int8_t* base, int64_t rows, int64_t K,
   return r == CUDA_SUCCESS;
 }
 
+// m-blocks per tile group: the group's Xq rows (group_m * bm * K bytes) are
+// kept near SQ_GEMM_GROUP_BYTES so that they stay in L2 while the group sweeps
+// every Wq slice.
+#ifndef SQ_GEMM_GROUP_BYTES  // build-time knob
+#define SQ_GEMM_GROUP_BYTES (32ll << 20)
+#endif
+int tile_group_m(int bm, int64_t K, int num_m_blocks) {
+  const int64_t per_block = static_cast<int64_t>(bm) * K;
+  const int64_t g = std::max<int64_t>(1, SQ_GEMM_GROUP_BYTES / per_block);
+  return static_cast<int>(std::min<int64_t>(g, num_m_blocks));
+}
+
 template <int BN, int STAGES, int EPI, int CHAINS>
 cudaError_t run_gemm(const GemmArgs& a, cudaStream_t st, const DeviceInfo& dev, const char** why) {
   using L = SmemLayout<BN, STAGES>;
@@ -487,6 +525,7 @@ cudaError_t run_gemm(const GemmArgs& a, cudaStream_t st, const DeviceInfo& dev, 
   p.num_m_blocks = static_cast<int>((a.M + kBM - 1) / kBM);
   p.num_n_blocks = static_cast<int>((a.N + BN - 1) / BN);
   p.num_k_blocks = static_cast<int>((a.K + kBK - 1) / kBK);
+  p.group_m = tile_group_m(kBM, a.K, p.num_m_blocks);
   p.x_scale = a.x_scale;
   p.w_scale = a.w_scale;
   p.bias = a.bias;
@@ -572,6 +611,75 @@ cudaError_t run_small(const SmallArgs& a, cudaStream_t st, const DeviceInfo& dev
   return e;
 }
 
+// Clusters of two CTAs that can run at once with the pair kernel's shared
+// memory (cached per device): the pair kernel's persistent grid.
+int pair_clusters(const DeviceInfo& dev) {
+  static std::mutex mu;
+  static int cached[64] = {};
+  std::lock_guard<std::mutex> lk(mu);
+  if (dev.device < 0 || dev.device >= 64) return 0;
+  if (cached[dev.device] != 0) return cached[dev.device];
+  int n = 0;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * static_cast<unsigned>(dev.sm_count / 2));
+  cfg.blockDim = dim3(kPairThreads);
+  cfg.dynamicSmemBytes = kPairAlloc;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  auto kern = gemm_i8_pair_kernel<0>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kPairAlloc) != cudaSuccess ||
+      cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess)
+    n = 0;
+  cached[dev.device] = n > 0 ? n : -1;
+  return cached[dev.device];
+}
+
+template <int EPI>
+cudaError_t run_pair(const GemmArgs& a, cudaStream_t st, const DeviceInfo& dev, int clusters, const char** why) {
+  CUtensorMap tmA, tmB;
+  if (!make_tmap_i8(&tmA, a.A, a.M, a.K, kPairHalf) || !make_tmap_i8(&tmB, a.B, a.N, a.K, kPairHalf)) {
+    *why = "cuTensorMapEncodeTiled failed or unavailable";
+    return cudaErrorInvalidValue;
+  }
+  PairParams p;
+  p.timeout_ns = g_debug_stall.load() ? g_debug_timeout_ns.load() : kWaitTimeoutNs;
+  p.skip_first_load = g_debug_stall.load() ? 1 : 0;
+  p.M = static_cast<int>(a.M);
+  p.N = static_cast<int>(a.N);
+  p.K = static_cast<int>(a.K);
+  p.num_m_blocks = static_cast<int>((a.M + kPairBM - 1) / kPairBM);
+  p.num_n_blocks = static_cast<int>((a.N + kPairBN - 1) / kPairBN);
+  p.num_k_blocks = static_cast<int>((a.K + kBK - 1) / kBK);
+  p.group_m = tile_group_m(kPairBM, a.K, p.num_m_blocks);
+  p.x_scale = a.x_scale;
+  p.w_scale = a.w_scale;
+  p.bias = a.bias;
+  p.out = a.out;
+  const int elem = (EPI == 0) ? 2 : 4;
+  p.vec_ok = ((a.N * elem) % 16 == 0) && (reinterpret_cast<uintptr_t>(a.out) % 16 == 0) &&
+             (reinterpret_cast<uintptr_t>(a.w_scale) % 16 == 0 || EPI != 0) &&
+             (a.bias == nullptr || reinterpret_cast<uintptr_t>(a.bias) % 16 == 0);
+  auto kern = gemm_i8_pair_kernel<EPI>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kPairAlloc);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, kCarveoutMaxShared);
+  if (e != cudaSuccess) {
+    *why = "cudaFuncSetAttribute failed";
+    return e;
+  }
+  const int tiles = p.num_m_blocks * p.num_n_blocks;
+  const int pairs = std::min(tiles, clusters);
+  e = launch_pdl_cluster(kern, dim3(2u * static_cast<unsigned>(pairs)), dim3(kPairThreads),
+                         static_cast<size_t>(kPairAlloc), st, 2u, tmA, tmB, p);
+  if (e != cudaSuccess) *why = "cluster launch of the CTA-pair GEMM failed";
+  return e;
+}
+
 // K split over a CTA pair (cluster of 2); the pair exchanges partial sums
 // through `a.ws` (at least splitk_workspace_bytes).
 cudaError_t run_splitk(const GemmArgs& a, cudaStream_t st, const char** why) {
@@ -650,6 +758,16 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t st, const DeviceInfo& de
   if (a.epi == Epilogue::kBf16Dequant && a.ws != nullptr) {
     const size_t need = gemm_workspace_bytes(a.M, a.N, a.K, dev.sm_count);
     if (need > 0 && a.ws_bytes >= need) return run_splitk(a, st, why);
+  }
+  // Output tiles of 256 x 256 on CTA pairs whenever they fill every pair at
+  // least once: each CTA then reads a third less operand data per MMA than
+  // with 128 x 256 tiles of its own.
+  if (SQ_GEMM_PAIR && SQ_GEMM_BN == 0) {
+    const int64_t pair_tiles = ((a.M + kPairBM - 1) / kPairBM) * ((a.N + kPairBN - 1) / kPairBN);
+    const int clusters = pair_clusters(dev);
+    if (clusters > 0 && pair_tiles >= clusters)
+      return a.epi == Epilogue::kBf16Dequant ? run_pair<0>(a, st, dev, clusters, why)
+                                             : run_pair<1>(a, st, dev, clusters, why);
   }
   const bool wide = SQ_GEMM_BN == 256 || (SQ_GEMM_BN == 0 && 2 * tiles256 > dev.sm_count);
   if (a.epi == Epilogue::kBf16Dequant) {
