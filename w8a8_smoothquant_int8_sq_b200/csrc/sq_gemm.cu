@@ -63,7 +63,7 @@ constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // 2 s per wait
 #define SQ_GEMM_SPLITK 1
 #endif
 #ifndef SQ_GEMM_PAIR  // 1: 256 x 256 tiles on CTA pairs (cta_group::2) when they fill every pair
-#define SQ_GEMM_PAIR 0
+#define SQ_GEMM_PAIR 1
 #endif
 #ifndef SQ_GEMM_CHAINS128  // accumulator chains for 128-wide tiles (1 or 2)
 #define SQ_GEMM_CHAINS128 2

@@ -575,14 +575,18 @@ static cudaError_t launch_rq(const uint16_t* src, int64_t rows, int K, const flo
 // by the ring (about 128 KB), not by registers.  Sixteen consumer warps form
 // G = 16 / WPG groups of WPG warps; group g takes every G-th row of the block
 // and owns SPG stages of the ring, so G rows are reduced at once.  Lane l of
-// the w-th warp of a group reads the 16-byte vectors i*(32*WPG) + 32*w + l
-// (i < 4) of the row from shared memory (each warp read one contiguous 512-byte
-// run, free of bank conflicts), releases the stage as soon as the smoothed
-// values are in registers, and writes its codes as 8-byte stores (one 256-byte
-// run per warp instruction).  The arithmetic -- t = fl(w*s) or fl(x/s), the row
-// maximum, scale = fl(max(m,1e-8)/127), q = rne(fl(t/scale)) -- is the same
-// sequence of correctly rounded fp32 operations as row_quant_kernel, so the
-// codes and scales are bit-identical.
+// the w-th warp of a group owns the 16-byte vectors i*(32*WPG) + 32*w + l
+// (i < 4) of every row, so the per-column factors it needs are the same for
+// all rows: s (weights) or -s (activations) sits in the lane's registers for
+// the whole kernel, and only RN(1/s) of the activation path is read per row,
+// from a shared-memory table of float4 in vector order (consecutive lanes,
+// consecutive 16 bytes: no bank conflicts).  Each warp reads one contiguous
+// 512-byte run of the row per instruction, releases the stage as soon as the
+// smoothed values are in registers, and writes its codes as 8-byte stores (one
+// 256-byte run per warp instruction).  The arithmetic -- t = fl(w*s) or
+// fl(x/s), the row maximum, scale = fl(max(m,1e-8)/127), q = rne(fl(t/scale))
+// -- is the same sequence of correctly rounded fp32 operations as
+// row_quant_kernel, so the codes and scales are bit-identical.
 // A wait that runs out of time is voted on beside the row maximum: every warp
 // of the group reads the same votes after the group barrier and leaves the row
 // loop together (no barrier is left waiting); the producer waits for the
@@ -605,12 +609,10 @@ __global__ void __launch_bounds__(kRqRingThreads, 1)
   const int nvec = K >> 3;
   const int nstages = G * spg;
   uint8_t* ring = smem;
-  float4* tab = reinterpret_cast<float4*>(ring + static_cast<size_t>(nstages) * row_stride);
-  float4* sA = tab;
-  float4* sB = tab + nvec;
-  float4* rA = tab + 2 * nvec;
-  float4* rB = tab + 3 * nvec;
-  uint64_t* full = reinterpret_cast<uint64_t*>(tab + (kMul ? 2 : 4) * nvec);
+  // activations: RN(1/s) of the 8 columns of vector v at rA[v], rB[v]
+  float4* rA = reinterpret_cast<float4*>(ring + static_cast<size_t>(nstages) * row_stride);
+  float4* rB = rA + nvec;
+  uint64_t* full = reinterpret_cast<uint64_t*>(rA + (kMul ? 0 : 2 * nvec));
   uint64_t* empty = full + nstages;
   float* red = reinterpret_cast<float*>(empty + nstages);  // [G][2][WPG] warp maxima
   int* vote = reinterpret_cast<int*>(red + G * 2 * WPG);     // [G][2][WPG] 1: the warp's wait ran out
@@ -640,17 +642,10 @@ __global__ void __launch_bounds__(kRqRingThreads, 1)
   griddep_wait();
   griddep_launch_dependents();
 
-  // table of s (weights) or of -s and RN(1/s) (activations), one float4 pair
-  // per 16-byte vector of 8 columns
   const float4* s4 = reinterpret_cast<const float4*>(s);
-  for (int v = tid; v < nvec; v += kRqRingThreads) {
-    const float4 a = __ldg(s4 + 2 * v), b = __ldg(s4 + 2 * v + 1);
-    if (kMul) {
-      sA[v] = a;
-      sB[v] = b;
-    } else {
-      sA[v] = make_float4(-a.x, -a.y, -a.z, -a.w);
-      sB[v] = make_float4(-b.x, -b.y, -b.z, -b.w);
+  if (!kMul) {
+    for (int v = tid; v < nvec; v += kRqRingThreads) {
+      const float4 a = __ldg(s4 + 2 * v), b = __ldg(s4 + 2 * v + 1);
       rA[v] = make_float4(__frcp_rn(a.x), __frcp_rn(a.y), __frcp_rn(a.z), __frcp_rn(a.w));
       rB[v] = make_float4(__frcp_rn(b.x), __frcp_rn(b.y), __frcp_rn(b.z), __frcp_rn(b.w));
     }
@@ -688,10 +683,23 @@ __global__ void __launch_bounds__(kRqRingThreads, 1)
 
   // -------------------------------------------------------------- consumers
   const int g = warp / WPG, w = warp % WPG;
-  const f2x* sA2 = reinterpret_cast<const f2x*>(sA);
-  const f2x* sB2 = reinterpret_cast<const f2x*>(sB);
-  const f2x* rA2 = reinterpret_cast<const f2x*>(rA);
-  const f2x* rB2 = reinterpret_cast<const f2x*>(rB);
+  // this lane's columns: s (weights) or -s (activations), as fp32 pairs
+  f2x sv[kRqRingVpl][4];
+#pragma unroll
+  for (int i = 0; i < kRqRingVpl; ++i) {
+    const int v = i * (32 * WPG) + w * 32 + lane;
+    float4 a = make_float4(1.f, 1.f, 1.f, 1.f), b = a;
+    if (v < nvec) {
+      a = __ldg(s4 + 2 * v);
+      b = __ldg(s4 + 2 * v + 1);
+    }
+    const float sg = kMul ? 1.0f : -1.0f;
+    sv[i][0] = f2_pack(sg * a.x, sg * a.y);
+    sv[i][1] = f2_pack(sg * a.z, sg * a.w);
+    sv[i][2] = f2_pack(sg * b.x, sg * b.y);
+    sv[i][3] = f2_pack(sg * b.z, sg * b.w);
+  }
+  const float r127 = __frcp_rn(kQmax);  // RN(1/127), for the correctly rounded max / 127
   for (int64_t jg = 0;; ++jg) {
     const int64_t j = jg * G + g;
     if (j >= my_rows) break;
@@ -709,14 +717,14 @@ __global__ void __launch_bounds__(kRqRingThreads, 1)
           const uint4 xw = *reinterpret_cast<const uint4*>(rowp + static_cast<size_t>(v) * 16);
           const f2x x[4] = {f2_from_bf16x2(xw.x), f2_from_bf16x2(xw.y), f2_from_bf16x2(xw.z),
                             f2_from_bf16x2(xw.w)};
-          const f2x sv[4] = {sA2[2 * v], sA2[2 * v + 1], sB2[2 * v], sB2[2 * v + 1]};
           if (kMul) {
 #pragma unroll
-            for (int e = 0; e < 4; ++e) t[i][e] = f2_mul(x[e], sv[e]);
+            for (int e = 0; e < 4; ++e) t[i][e] = f2_mul(x[e], sv[i][e]);
           } else {
-            const f2x rv[4] = {rA2[2 * v], rA2[2 * v + 1], rB2[2 * v], rB2[2 * v + 1]};
+            const float4 ra = rA[v], rb = rB[v];
+            const f2x rv[4] = {f2_pack(ra.x, ra.y), f2_pack(ra.z, ra.w), f2_pack(rb.x, rb.y), f2_pack(rb.z, rb.w)};
 #pragma unroll
-            for (int e = 0; e < 4; ++e) t[i][e] = f2_div_rn(x[e], sv[e], rv[e]);
+            for (int e = 0; e < 4; ++e) t[i][e] = f2_div_rn(x[e], sv[i][e], rv[e]);
           }
 #pragma unroll
           for (int e = 0; e < 4; ++e) m = f2_absmax(m, t[i][e]);
@@ -749,7 +757,10 @@ __global__ void __launch_bounds__(kRqRingThreads, 1)
       }
     }
     if (give_up) break;
-    const float sc = __fdiv_rn(fmaxf(m, kClampFloor), kQmax);
+    // fl(max / 127) by Markstein's correction of the product with RN(1/127):
+    // equal to the IEEE quotient for every fp32 from 1e-8 up (checked
+    // exhaustively on the CPU), and a few cycles instead of a division
+    const float sc = div_rn(fmaxf(m, kClampFloor), kQmax, r127);
     const float rsc = __frcp_rn(sc);
     const f2x nsc2 = f2_pack(-sc, -sc), rsc2 = f2_pack(rsc, rsc);
     int8_t* qr = q + row * static_cast<int64_t>(K);
@@ -773,7 +784,7 @@ static cudaError_t launch_rq_ring(const uint16_t* src, int64_t rows, int K, cons
   constexpr int G = kRqConsumerWarps / WPG;
   const int nvec = K / 8;
   const int row_stride = (K * 2 + 127) / 128 * 128;
-  const int tab_bytes = nvec * 16 * (kMul ? 2 : 4);
+  const int tab_bytes = kMul ? 0 : nvec * 16 * 2;  // RN(1/s) for the activation path
   const int fixed = tab_bytes + 128 /* alignment */ + 64 /* flag, slack */ + G * 2 * WPG * 8;
   // stages per group: as many as fit (at most kRqRingMaxSpg), at least 2
   int spg = kRqRingMaxSpg;
