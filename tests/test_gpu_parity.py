@@ -134,7 +134,7 @@ def test_zero_rows_and_floor(sq):
     assert np.array_equal(host(Xq), Xq_o) and np.array_equal(host(xs), xs_o)
 
 
-@pytest.mark.parametrize("K", [256, 4096])  # both row quantisers: register prefetch and bulk-copy ring
+@pytest.mark.parametrize("K", [256, 4096])  # one and four warps per row in the row quantiser
 def test_tiny_values_and_subnormal_quotients(sq, K):
     """Values near the bottom of the fp32 range: X / s and W * s below 2^-126
     (subnormal quotients and products), rows whose maximum sits on the 1e-8

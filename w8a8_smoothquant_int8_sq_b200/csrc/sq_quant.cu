@@ -475,10 +475,7 @@ __global__ void __launch_bounds__(kRowThreads) row_quant_kernel(const uint16_t* 
   }
   __syncthreads();
   SQ_BLOCK_MARK(3);
-  const f2x* sA2 = reinterpret_cast<const f2x*>(sA);
-  const f2x* sB2 = reinterpret_cast<const f2x*>(sB);
-  const f2x* rA2 = reinterpret_cast<const f2x*>(rA);
-  const f2x* rB2 = reinterpret_cast<const f2x*>(rB);
+  const float r127 = __frcp_rn(kQmax);  // RN(1/127), for the correctly rounded max / 127
 
   for (int it = 0; row < rows; ++it) {
     f2x t[VPL][4];  // smoothed values, pairs of columns
@@ -489,12 +486,16 @@ __global__ void __launch_bounds__(kRowThreads) row_quant_kernel(const uint16_t* 
       if (v < nvec) {
         const uint4 w = xv[i];
         const f2x x[4] = {f2_from_bf16x2(w.x), f2_from_bf16x2(w.y), f2_from_bf16x2(w.z), f2_from_bf16x2(w.w)};
-        const f2x sv[4] = {sA2[2 * v], sA2[2 * v + 1], sB2[2 * v], sB2[2 * v + 1]};
+        // one 16-byte table read per float4: consecutive lanes, consecutive
+        // 16 bytes (no bank conflicts)
+        const float4 sa = sA[v], sb = sB[v];
+        const f2x sv[4] = {f2_pack(sa.x, sa.y), f2_pack(sa.z, sa.w), f2_pack(sb.x, sb.y), f2_pack(sb.z, sb.w)};
         if (kMul) {
 #pragma unroll
           for (int e = 0; e < 4; ++e) t[i][e] = f2_mul(x[e], sv[e]);
         } else {
-          const f2x rv[4] = {rA2[2 * v], rA2[2 * v + 1], rB2[2 * v], rB2[2 * v + 1]};
+          const float4 ra = rA[v], rb = rB[v];
+          const f2x rv[4] = {f2_pack(ra.x, ra.y), f2_pack(ra.z, ra.w), f2_pack(rb.x, rb.y), f2_pack(rb.z, rb.w)};
 #pragma unroll
           for (int e = 0; e < 4; ++e) t[i][e] = f2_div_rn(x[e], sv[e], rv[e]);
         }
@@ -523,7 +524,10 @@ __global__ void __launch_bounds__(kRowThreads) row_quant_kernel(const uint16_t* 
 #pragma unroll
       for (int w = 0; w < WPR; ++w) m = fmaxf(m, red[it & 1][slot * WPR + w]);
     }
-    const float sc = __fdiv_rn(fmaxf(m, kClampFloor), kQmax);
+    // fl(max / 127): Markstein's correction of the product with RN(1/127),
+    // equal to the IEEE quotient for every fp32 from 1e-8 up (checked
+    // exhaustively on the CPU)
+    const float sc = div_rn(fmaxf(m, kClampFloor), kQmax, r127);
     const float rsc = __frcp_rn(sc);
     const f2x nsc2 = f2_pack(-sc, -sc), rsc2 = f2_pack(rsc, rsc);
     int8_t* qr = q + row * static_cast<int64_t>(K);
@@ -567,257 +571,9 @@ static cudaError_t launch_rq(const uint16_t* src, int64_t rows, int K, const flo
 #define SQ_RQ_VPL 4
 #endif
 
-// ------------------------------------- row quantiser with a bulk-copy row ring
-// For rows of at least kRqRingMinK columns.  One block per SM, persistent
-// over rows (block b takes rows b, b + grid, b + 2 grid, ...).  A producer
-// warp streams whole rows by 1-D bulk copies (cp.async.bulk, one copy of 2K
-// bytes per row) into a shared-memory ring; the bytes in flight per SM are set
-// by the ring (about 128 KB), not by registers.  Sixteen consumer warps form
-// G = 16 / WPG groups of WPG warps; group g takes every G-th row of the block
-// and owns SPG stages of the ring, so G rows are reduced at once.  Lane l of
-// the w-th warp of a group owns the 16-byte vectors i*(32*WPG) + 32*w + l
-// (i < 4) of every row, so the per-column factors it needs are the same for
-// all rows: s (weights) or -s (activations) sits in the lane's registers for
-// the whole kernel, and only RN(1/s) of the activation path is read per row,
-// from a shared-memory table of float4 in vector order (consecutive lanes,
-// consecutive 16 bytes: no bank conflicts).  Each warp reads one contiguous
-// 512-byte run of the row per instruction, releases the stage as soon as the
-// smoothed values are in registers, and writes its codes as 8-byte stores (one
-// 256-byte run per warp instruction).  The arithmetic -- t = fl(w*s) or
-// fl(x/s), the row maximum, scale = fl(max(m,1e-8)/127), q = rne(fl(t/scale))
-// -- is the same sequence of correctly rounded fp32 operations as
-// row_quant_kernel, so the codes and scales are bit-identical.
-// A wait that runs out of time is voted on beside the row maximum: every warp
-// of the group reads the same votes after the group barrier and leaves the row
-// loop together (no barrier is left waiting); the producer waits for the
-// copies it issued before the block exits.
-constexpr int kRqConsumerWarps = 16;
-constexpr int kRqRingThreads = 32 * (kRqConsumerWarps + 1);
-constexpr int kRqRingVpl = 4;              // 16-byte vectors per lane per row
-constexpr int64_t kRqRingMinK = 1024;      // rows of at least 2 KB
-constexpr int kRqRingMaxSpg = 4;           // ring stages per group at most
-constexpr int kRqRingSmemBudget = 220 * 1024;
-
-template <bool kMul, int WPG>
-__global__ void __launch_bounds__(kRqRingThreads, 1)
-    row_quant_ring_kernel(const uint16_t* __restrict__ src, int64_t rows, int K, const float* __restrict__ s,
-                          int8_t* __restrict__ q, float* __restrict__ scale, int spg, int row_stride,
-                          unsigned long long timeout_ns) {
-  constexpr int G = kRqConsumerWarps / WPG;  // row groups
-  extern __shared__ __align__(128) uint8_t rq_smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(rq_smem_raw) + 127) & ~uintptr_t(127));
-  const int nvec = K >> 3;
-  const int nstages = G * spg;
-  uint8_t* ring = smem;
-  // activations: RN(1/s) of the 8 columns of vector v at rA[v], rB[v]
-  float4* rA = reinterpret_cast<float4*>(ring + static_cast<size_t>(nstages) * row_stride);
-  float4* rB = rA + nvec;
-  uint64_t* full = reinterpret_cast<uint64_t*>(rA + (kMul ? 0 : 2 * nvec));
-  uint64_t* empty = full + nstages;
-  float* red = reinterpret_cast<float*>(empty + nstages);  // [G][2][WPG] warp maxima
-  int* vote = reinterpret_cast<int*>(red + G * 2 * WPG);     // [G][2][WPG] 1: the warp's wait ran out
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(vote + G * 2 * WPG);
-
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int64_t grid = gridDim.x;
-  const int64_t my_rows = rows > static_cast<int64_t>(blockIdx.x)
-                              ? (rows - static_cast<int64_t>(blockIdx.x) + grid - 1) / grid
-                              : 0;
-  const uint32_t row_bytes = static_cast<uint32_t>(K) * 2u;
-
-  if (tid == 0) {
-    for (int i = 0; i < nstages; ++i) {
-      mbar_init(&full[i], 1);
-      mbar_init(&empty[i], WPG);
-    }
-    *abort_flag = 0;
-    fence_mbar_init();
-  }
-  // While the previous kernel is still running, pull this block's first rows
-  // into L2 (a hint: the copies into shared memory come after the wait).
-  if (warp == kRqConsumerWarps && lane == 0) {
-    for (int64_t j = 0; j < my_rows && j < nstages; ++j)
-      bulk_prefetch_l2(src + (blockIdx.x + j * grid) * static_cast<int64_t>(K), row_bytes);
-  }
-  griddep_wait();
-  griddep_launch_dependents();
-
-  const float4* s4 = reinterpret_cast<const float4*>(s);
-  if (!kMul) {
-    for (int v = tid; v < nvec; v += kRqRingThreads) {
-      const float4 a = __ldg(s4 + 2 * v), b = __ldg(s4 + 2 * v + 1);
-      rA[v] = make_float4(__frcp_rn(a.x), __frcp_rn(a.y), __frcp_rn(a.z), __frcp_rn(a.w));
-      rB[v] = make_float4(__frcp_rn(b.x), __frcp_rn(b.y), __frcp_rn(b.z), __frcp_rn(b.w));
-    }
-  }
-  __syncthreads();
-
-  if (warp == kRqConsumerWarps) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      int64_t j = 0;
-      for (; j < my_rows; ++j) {
-        const int g = static_cast<int>(j % G);
-        const int64_t jg = j / G;
-        const int st = g * spg + static_cast<int>(jg % spg);
-        if (jg >= spg && (*abort_flag || !mbar_wait_bounded(&empty[st], static_cast<uint32_t>(((jg / spg) - 1) & 1),
-                                                            timeout_ns))) {
-          *abort_flag = 1;
-          break;
-        }
-        mbar_arrive_expect_tx(&full[st], row_bytes);
-        bulk_load(ring + static_cast<size_t>(st) * row_stride, src + (blockIdx.x + j * grid) * static_cast<int64_t>(K),
-                  row_bytes, &full[st]);
-      }
-      // every copy issued must land before the block exits (a no-op wait for
-      // the copies the consumers have taken already)
-      for (int64_t i = j > nstages ? j - nstages : 0; i < j; ++i) {
-        const int g = static_cast<int>(i % G);
-        const int64_t ig = i / G;
-        (void)mbar_wait_bounded(&full[g * spg + static_cast<int>(ig % spg)], static_cast<uint32_t>((ig / spg) & 1),
-                                timeout_ns);
-      }
-    }
-    return;
-  }
-
-  // -------------------------------------------------------------- consumers
-  const int g = warp / WPG, w = warp % WPG;
-  // this lane's columns: s (weights) or -s (activations), as fp32 pairs
-  f2x sv[kRqRingVpl][4];
-#pragma unroll
-  for (int i = 0; i < kRqRingVpl; ++i) {
-    const int v = i * (32 * WPG) + w * 32 + lane;
-    float4 a = make_float4(1.f, 1.f, 1.f, 1.f), b = a;
-    if (v < nvec) {
-      a = __ldg(s4 + 2 * v);
-      b = __ldg(s4 + 2 * v + 1);
-    }
-    const float sg = kMul ? 1.0f : -1.0f;
-    sv[i][0] = f2_pack(sg * a.x, sg * a.y);
-    sv[i][1] = f2_pack(sg * a.z, sg * a.w);
-    sv[i][2] = f2_pack(sg * b.x, sg * b.y);
-    sv[i][3] = f2_pack(sg * b.z, sg * b.w);
-  }
-  const float r127 = __frcp_rn(kQmax);  // RN(1/127), for the correctly rounded max / 127
-  for (int64_t jg = 0;; ++jg) {
-    const int64_t j = jg * G + g;
-    if (j >= my_rows) break;
-    const int64_t row = blockIdx.x + j * grid;
-    const int st = g * spg + static_cast<int>(jg % spg);
-    const bool ok = !*abort_flag && mbar_wait_bounded(&full[st], static_cast<uint32_t>((jg / spg) & 1), timeout_ns);
-    f2x t[kRqRingVpl][4];
-    float m = 0.0f;
-    if (ok) {
-      const uint8_t* rowp = ring + static_cast<size_t>(st) * row_stride;
-#pragma unroll
-      for (int i = 0; i < kRqRingVpl; ++i) {
-        const int v = i * (32 * WPG) + w * 32 + lane;
-        if (v < nvec) {
-          const uint4 xw = *reinterpret_cast<const uint4*>(rowp + static_cast<size_t>(v) * 16);
-          const f2x x[4] = {f2_from_bf16x2(xw.x), f2_from_bf16x2(xw.y), f2_from_bf16x2(xw.z),
-                            f2_from_bf16x2(xw.w)};
-          if (kMul) {
-#pragma unroll
-            for (int e = 0; e < 4; ++e) t[i][e] = f2_mul(x[e], sv[i][e]);
-          } else {
-            const float4 ra = rA[v], rb = rB[v];
-            const f2x rv[4] = {f2_pack(ra.x, ra.y), f2_pack(ra.z, ra.w), f2_pack(rb.x, rb.y), f2_pack(rb.z, rb.w)};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) t[i][e] = f2_div_rn(x[e], sv[i][e], rv[e]);
-          }
-#pragma unroll
-          for (int e = 0; e < 4; ++e) m = f2_absmax(m, t[i][e]);
-        } else {
-#pragma unroll
-          for (int e = 0; e < 4; ++e) t[i][e] = 0ull;
-        }
-      }
-    } else if (lane == 0 && !*abort_flag) {
-      *abort_flag = 1;
-      atomicOr(&g_sq_quant_status, 1u);
-    }
-    // the smoothed values are in registers: the stage may be refilled
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[st]);
-    m = warp_max(m);
-    bool give_up = !ok;
-    if (WPG > 1) {
-      const int slot = (g * 2 + static_cast<int>(jg & 1)) * WPG;
-      if (lane == 0) {
-        red[slot + w] = m;
-        vote[slot + w] = ok ? 0 : 1;
-      }
-      named_bar_sync(1 + g, 32 * WPG);
-      // every warp of the group reads the same votes: they leave together
-#pragma unroll
-      for (int k = 0; k < WPG; ++k) {
-        m = fmaxf(m, red[slot + k]);
-        give_up = give_up || vote[slot + k] != 0;
-      }
-    }
-    if (give_up) break;
-    // fl(max / 127) by Markstein's correction of the product with RN(1/127):
-    // equal to the IEEE quotient for every fp32 from 1e-8 up (checked
-    // exhaustively on the CPU), and a few cycles instead of a division
-    const float sc = div_rn(fmaxf(m, kClampFloor), kQmax, r127);
-    const float rsc = __frcp_rn(sc);
-    const f2x nsc2 = f2_pack(-sc, -sc), rsc2 = f2_pack(rsc, rsc);
-    int8_t* qr = q + row * static_cast<int64_t>(K);
-#pragma unroll
-    for (int i = 0; i < kRqRingVpl; ++i) {
-      const int v = i * (32 * WPG) + w * 32 + lane;
-      if (v < nvec) {
-        f2x c[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) c[e] = f2_round_codes(f2_div_rn(t[i][e], nsc2, rsc2));
-        *reinterpret_cast<uint2*>(qr + static_cast<int64_t>(v) * 8) = pack8_codes(c[0], c[1], c[2], c[3]);
-      }
-    }
-    if (w == 0 && lane == 0) scale[row] = sc;
-  }
-}
-
-template <bool kMul, int WPG>
-static cudaError_t launch_rq_ring(const uint16_t* src, int64_t rows, int K, const float* s, int8_t* q, float* scale,
-                                  cudaStream_t st, const DeviceInfo& dev) {
-  constexpr int G = kRqConsumerWarps / WPG;
-  const int nvec = K / 8;
-  const int row_stride = (K * 2 + 127) / 128 * 128;
-  const int tab_bytes = kMul ? 0 : nvec * 16 * 2;  // RN(1/s) for the activation path
-  const int fixed = tab_bytes + 128 /* alignment */ + 64 /* flag, slack */ + G * 2 * WPG * 8;
-  // stages per group: as many as fit (at most kRqRingMaxSpg), at least 2
-  int spg = kRqRingMaxSpg;
-  while (spg > 2 && fixed + G * spg * (row_stride + 16) > kRqRingSmemBudget) --spg;
-  const int smem = fixed + G * spg * (row_stride + 16);
-  if (smem > static_cast<int>(dev.max_smem_optin)) return cudaErrorNotSupported;
-  auto kern = row_quant_ring_kernel<kMul, WPG>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e == cudaSuccess) e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, kCarveoutMaxShared);
-  if (e != cudaSuccess) return e;
-  const int64_t grid = std::min<int64_t>(rows, dev.sm_count);
-  return launch_pdl(kern, dim3(static_cast<unsigned>(grid)), dim3(kRqRingThreads), static_cast<size_t>(smem), st, src,
-                    rows, K, s, q, scale, spg, row_stride, kQuantWaitTimeoutNs);
-}
-
-#ifndef SQ_RQ_RING  // build-time knob: 0 keeps every row width on the register-prefetch kernel
-#define SQ_RQ_RING 0
-#endif
-
 template <bool kMul>
 static cudaError_t dispatch_rq(const uint16_t* src, int64_t rows, int K, const float* s, int8_t* q, float* scale,
                                cudaStream_t st, const DeviceInfo& dev) {
-  if (SQ_RQ_RING && K >= kRqRingMinK) {
-    // warps per row: enough for four 16-byte vectors per lane
-    const int nvec = K / 8;
-    cudaError_t e;
-    if (nvec <= 128) e = launch_rq_ring<kMul, 1>(src, rows, K, s, q, scale, st, dev);
-    else if (nvec <= 256) e = launch_rq_ring<kMul, 2>(src, rows, K, s, q, scale, st, dev);
-    else if (nvec <= 512) e = launch_rq_ring<kMul, 4>(src, rows, K, s, q, scale, st, dev);
-    else if (nvec <= 1024) e = launch_rq_ring<kMul, 8>(src, rows, K, s, q, scale, st, dev);
-    else e = launch_rq_ring<kMul, 16>(src, rows, K, s, q, scale, st, dev);
-    if (e != cudaErrorNotSupported) return e;
-  }
   // vectors per lane (up to SQ_RQ_VPL), then warps per row (up to 8) to cover K
   constexpr int V = SQ_RQ_VPL;
   static_assert(V == 4 || V == 8, "SQ_RQ_VPL must be 4 or 8");
