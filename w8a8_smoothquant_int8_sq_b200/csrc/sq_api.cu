@@ -33,8 +33,6 @@ cudaError_t current_device_info(DeviceInfo* out) {
   int smem = 0;
   if ((e = cudaDeviceGetAttribute(&smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess) return e;
   d.max_smem_optin = static_cast<size_t>(smem);
-  if ((e = cudaDeviceGetAttribute(&smem, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev)) != cudaSuccess) return e;
-  d.max_smem_per_sm = static_cast<size_t>(smem);
   if (static_cast<int>(cache.size()) <= dev) cache.resize(dev + 1);
   cache[dev] = d;
   *out = d;
@@ -406,8 +404,6 @@ sq_status sq_forward(const sq_bf16* X, const float* s, const int8_t* Wq, const f
   SQ_TRY(prologue(&dev));
   if (M <= sq::kSmallFusedMaxM) {  // few tokens: quantisation fused into the weight-streaming kernel
     sq::SmallArgs a{X, s, nullptr, nullptr, Wq, w_scale, bias, M, N, K, Y};
-    // the per-token scales of the fused path go where the unfused path keeps x_scale
-    a.xs_scratch = reinterpret_cast<float*>(static_cast<char*>(workspace) + forward_xq_bytes(M, K));
     const char* why = "fused small-M kernel";
     cudaError_t e = sq::launch_small_m(a, static_cast<cudaStream_t>(stream), dev, &why);
     if (e != cudaErrorNotSupported) return cuda_status(e, why);

@@ -62,12 +62,6 @@ constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // 2 s per wait
 #ifndef SQ_GEMM_SPLITK  // 1: split K over a CTA pair when 128 x 256 tiles fill at most half the SMs
 #define SQ_GEMM_SPLITK 1
 #endif
-#ifndef SQ_DECODE_NT  // 1: few-token GEMM with the tokens on the MMA's M side (gemm_decode_kernel)
-#define SQ_DECODE_NT 0
-#endif
-#ifndef SQ_DEC_TWO_PER_SM  // 1: the decode kernel runs two CTAs per SM when the row blocks allow it
-#define SQ_DEC_TWO_PER_SM 1
-#endif
 #ifndef SQ_GEMM_PAIR  // 1: 256 x 256 tiles on CTA pairs (cta_group::2) when they fill every pair
 #define SQ_GEMM_PAIR 1
 #endif
@@ -459,7 +453,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 namespace sq {
 namespace {
 #include "sq_gemm_pair.cuh"
-#include "sq_gemm_decode.cuh"
 }  // namespace
 }  // namespace sq
 
@@ -731,99 +724,9 @@ cudaError_t run_splitk(const GemmArgs& a, cudaStream_t st, const char** why) {
 
 }  // namespace
 
-// The weight-streaming decode GEMM (tokens on the MMA's M side, 256 Wq rows
-// on its N side).  Cluster size and ring depth: two CTAs per SM (a cluster of
-// 8 over K) when the row blocks allow it -- two CTAs per SM keep more weight
-// boxes in flight than one -- else one CTA per SM with up to 8 splits.
-template <bool kFused>
-cudaError_t run_decode(const SmallArgs& a, cudaStream_t st, const DeviceInfo& dev, const char** why) {
-  const int nrb = static_cast<int>((a.N + kDecRows - 1) / kDecRows);
-  const int nk = static_cast<int>((a.K + kBK - 1) / kBK);
-  const int a_atoms = static_cast<int>((a.M + 7) / 8);
-  const int mp = static_cast<int>((a.M + 3) / 4 * 4);
-  const bool two = SQ_DEC_TWO_PER_SM && nrb * 8 <= 2 * dev.sm_count && nk >= 16;
-  int S = 1;
-  if (two) {
-    S = 8;
-  } else {
-    while (S < 8 && static_cast<int64_t>(nrb) * S * 2 <= dev.sm_count && (nk + 2 * S - 1) / (2 * S) >= 2) S *= 2;
-  }
-  // fused: each of the 256 code threads takes one 16-byte vector of the slice
-  while (kFused && S < 8 && (nk + S - 1) / S > 16) S *= 2;
-  const int kps = (nk + S - 1) / S;
-  if (kFused && kps > 16) {
-    *why = "decode kernel: K too large for the fused codes";
-    return cudaErrorNotSupported;
-  }
-  // the token atoms, then the ring: the MMA of the last k-blocks reads its
-  // unused rows (16 atoms from each k-block's first) from the ring's start
-  const int a_bytes = kps * a_atoms * 1024;
-  const int part_bytes = kDecRows * mp * 4;
-  const int budget = two ? static_cast<int>(dev.max_smem_per_sm / 2) - 1024 : static_cast<int>(dev.max_smem_optin);
-  const int fixed = a_bytes + part_bytes + 256 + 16 + 1024;
-  int stages = std::min(kDecMaxStages, (budget - fixed) / kDecStageBytes);
-  if (stages < 2 || kDecRows * mp * 4 > stages * kDecStageBytes) {
-    *why = "decode kernel: shape does not fit shared memory";
-    return cudaErrorNotSupported;
-  }
-  DecParams p{};
-  p.M = static_cast<int>(a.M);
-  p.N = static_cast<int>(a.N);
-  p.K = static_cast<int>(a.K);
-  p.nk = nk;
-  p.kb_per_split = kps;
-  p.stages = stages;
-  p.a_atoms = a_atoms;
-  p.mp = mp;
-  p.X = a.X;
-  p.s = a.s;
-  p.x_scale = kFused ? a.xs_scratch : a.x_scale;
-  p.w_scale = a.w_scale;
-  p.bias = a.bias;
-  p.Y = a.Y;
-  p.ring_off = a_bytes;
-  p.part_off = p.ring_off + stages * kDecStageBytes;
-  p.bar_off = p.part_off + part_bytes;
-  p.misc_off = p.bar_off + 256;
-  p.timeout_ns = kWaitTimeoutNs;
-  const int alloc = p.misc_off + 16 + 1024;
-  CUtensorMap tmW, tmX;
-  if (!make_tmap_i8(&tmW, a.Wq, a.N, a.K, kDecRows) || (!kFused && !make_tmap_i8(&tmX, a.Xq, a.M, a.K, 8 * a_atoms))) {
-    *why = "cuTensorMapEncodeTiled failed or unavailable";
-    return cudaErrorInvalidValue;
-  }
-  if (kFused) tmX = tmW;  // unused
-  auto kern = gemm_decode_kernel<kFused>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, alloc);
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, kCarveoutMaxShared);
-  if (e != cudaSuccess) {
-    *why = "cudaFuncSetAttribute failed";
-    return e;
-  }
-  if (kFused) {
-    // the per-token scales first; the GEMM launches as soon as this kernel
-    // starts and streams its weight meanwhile
-    e = launch_pdl(row_scale_kernel, dim3(static_cast<unsigned>(a.M)), dim3(256), 0, st, a.X, p.K, a.s,
-                   a.xs_scratch);
-    if (e != cudaSuccess) {
-      *why = "launch of the per-token scale pre-pass failed";
-      return e;
-    }
-  }
-  e = launch_pdl_cluster(kern, dim3(static_cast<unsigned>(S), static_cast<unsigned>(nrb), 1), dim3(kDecThreads),
-                         static_cast<size_t>(alloc), st, static_cast<unsigned>(S), tmW, tmX, p);
-  if (e != cudaSuccess) *why = "cluster launch of the decode kernel failed";
-  return e;
-}
-
 cudaError_t launch_small_m(const SmallArgs& a, cudaStream_t st, const DeviceInfo& dev, const char** why) {
   if (a.M < 1 || a.M > kSmallMaxM) return cudaErrorNotSupported;
   const bool fused = a.X != nullptr;
-  if (SQ_DECODE_NT && (!fused || a.xs_scratch != nullptr)) {
-    const cudaError_t e = fused ? run_decode<true>(a, st, dev, why) : run_decode<false>(a, st, dev, why);
-    if (e != cudaErrorNotSupported) return e;
-  }
   if (a.M <= 16) return fused ? run_small<16, true>(a, st, dev, why) : run_small<16, false>(a, st, dev, why);
   return fused ? run_small<32, true>(a, st, dev, why) : run_small<32, false>(a, st, dev, why);
 }
@@ -885,9 +788,6 @@ extern "C" __attribute__((visibility("default"))) int sq_trace_read_big(unsigned
                  cudaSuccess
              ? 0
              : 1;
-}
-extern "C" __attribute__((visibility("default"))) int sq_trace_read_dec(unsigned long long* host) {
-  return cudaMemcpyFromSymbol(host, g_dec_trace, sizeof(g_dec_trace)) == cudaSuccess ? 0 : 1;
 }
 extern "C" __attribute__((visibility("default"))) int sq_trace_read(unsigned long long* host, int n) {
   return cudaMemcpyFromSymbol(host, g_small_trace, sizeof(unsigned long long) * 12 * static_cast<size_t>(n)) ==

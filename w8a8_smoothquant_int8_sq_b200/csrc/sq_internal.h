@@ -55,7 +55,6 @@ struct DeviceInfo {
   int sm_count = 0;
   int major = 0, minor = 0;
   size_t max_smem_optin = 0;
-  size_t max_smem_per_sm = 0;
 };
 
 // Cached properties of the current device.
@@ -158,7 +157,6 @@ struct SmallArgs {
   const uint16_t* bias;   // [N] or null
   int64_t M, N, K;
   uint16_t* Y;            // [M][N]
-  float* xs_scratch = nullptr;  // fused: [M] floats the per-token scale pre-pass writes
 };
 cudaError_t launch_small_m(const SmallArgs& a, cudaStream_t st, const DeviceInfo& dev, const char** why);
 
