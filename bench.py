@@ -1,7 +1,8 @@
 """Benchmark of the SmoothQuant W8A8 int8 linear layer on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload prefill]
-                    [--path smoothquant|forward|per-tensor|ste-train|weight-only] [--serial]
+                    [--path smoothquant|forward|forward-prologue|per-tensor|ste-train|weight-only]
+                    [--serial]
                     [--impl ours|reference] [--no-e2e] [--no-cpu-baseline]
 
 A step is one pass of the whole path over one batch of seeded synthetic input:
@@ -19,6 +20,10 @@ Paths (`--path`):
                pre-quantised weights (default for decode: every call streams
                the 64 MiB of int8 W from HBM -- the calls rotate over enough
                prepared weight copies, >= 256 MiB, that L2 cannot serve them);
+  forward-prologue
+               the same per-call forward through sq_forward_prologue, whose
+               GEMM quantises X itself (codes written straight into the
+               tensor core's shared-memory operand after a scale pre-pass);
   per-tensor   one scale per tensor for W and X, then the int8 GEMM;
   ste-train    s from the running max, the forward, and the straight-through
                backward to X, W, bias and eta_alpha of a seeded dL/dY;
@@ -83,7 +88,9 @@ FALLBACK_BF16_TFLOPS = 1590.0
 INT8_OVER_BF16 = 2.0  # nominal dense int8 / bf16 ratio (4.5 / 2.25 PFLOP/s)
 # fp32 multiply-add peak of the CUDA cores: 148 SMs x 128 lanes x 2 flops x 1.965 GHz
 FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
-PATHS = ["smoothquant", "forward", "per-tensor", "ste-train", "weight-only"]
+PATHS = ["smoothquant", "forward", "forward-prologue", "per-tensor", "ste-train", "weight-only"]
+# the per-call forward paths and the call each one times
+FORWARD_CALLS = {"forward": "sq_forward", "forward-prologue": "sq_forward_prologue"}
 # sq_forward fuses the activation quantisation into the weight-streaming
 # kernel up to this many tokens (one launch), else runs the quantiser first
 FORWARD_FUSED_MAX_M = 8
@@ -98,7 +105,8 @@ def parse_args(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--path", default=None, choices=PATHS,
                     help="smoothquant: the whole path (default); forward: sq_forward on prepared weights "
-                         "(default for decode); per-tensor: the baseline W8A8 path (one scale per tensor); "
+                         "(default for decode); forward-prologue: sq_forward_prologue (the GEMM quantises "
+                         "X itself) on prepared weights; per-tensor: the baseline W8A8 path (one scale per tensor); "
                          "ste-train: a learnable-alpha training step (s from the running max, forward, "
                          "straight-through backward); weight-only: the int8 weight-only comparison")
     ap.add_argument("--serial", action="store_true",
@@ -143,9 +151,11 @@ def workload_config(wl, path="smoothquant"):
     elif path == "ste-train":
         c["workload"] = ("learnable-alpha training step (s from the running max of the calibration batch, "
                          "forward, straight-through backward of a seeded bf16 dL/dY), " + c["workload"])
-    elif path == "forward":
-        c["workload"] = ("per-call forward on pre-quantised weights (sq_forward: activation quantisation + "
-                         "int8 GEMM + epilogue; calibration and weight prep done once, untimed), " + c["workload"])
+    elif path in FORWARD_CALLS:
+        what = ("sq_forward: activation quantisation + int8 GEMM + epilogue" if path == "forward" else
+                "sq_forward_prologue: scale pre-pass + int8 GEMM that quantises X in its prologue + epilogue")
+        c["workload"] = (f"per-call forward on pre-quantised weights ({what}; calibration and weight prep done "
+                         "once, untimed), " + c["workload"])
         c["l2"] = (f"calls rotate over {forward_rotation(wl)} prepared weight copies "
                    f"({forward_rotation(wl) * wl.N * wl.K / 2**20:.0f} MiB of int8 W), so every call streams "
                    f"its weight from HBM")
@@ -177,6 +187,7 @@ def algorithmic_work(wl):
         # X in (bf16), s, the codes and scales of W in, Y out; the codes of X
         # need not leave the chip
         "sq_forward": (2 * M * K + 4 * K + N * K + 4 * N + 2 * M * N, 2 * M * N * K),
+        "sq_forward_prologue": (2 * M * K + 4 * K + N * K + 4 * N + 2 * M * N, 2 * M * N * K),
         # one scale per tensor: the data once in, the codes and the scale row out
         "sq_quantize_per_tensor(W)": (3 * N * K + 4 * N, 0),
         "sq_quantize_per_tensor(X)": (3 * M * K + 4 * M, 0),
@@ -324,8 +335,10 @@ SAMPLE_W_ROWS = 4096
 
 def sample_plan(wl, path):
     """(rows of X, rows of W) the oracle's step runs on: all of them for the
-    smaller layers, a seeded-input prefix for the prefill layer."""
-    if path != "smoothquant" or (wl.M * wl.N * wl.K <= WHOLE_STEP_MAX_MNK and wl.N * wl.K <= WHOLE_STEP_MAX_NK):
+    smaller layers, a seeded-input prefix for the prefill layer (whole path
+    and per-call forward)."""
+    if (path != "smoothquant" and path not in FORWARD_CALLS) or (wl.M * wl.N * wl.K <= WHOLE_STEP_MAX_MNK and
+                                                                   wl.N * wl.K <= WHOLE_STEP_MAX_NK):
         return wl.M, wl.N
     return min(wl.M, SAMPLE_X_ROWS), min(wl.N, SAMPLE_W_ROWS)
 
@@ -336,12 +349,13 @@ def oracle_inputs(wl, path, inp=None):
     inp = dict(workloads.make_inputs(wl) if inp is None else inp)
     if path == "ste-train":
         inp["G"] = train_gradient(wl)
-    if path == "forward":
+    if path in FORWARD_CALLS:
         # the weight is prepared once, outside the timed calls (as on the GPU)
         from oracle import smoothquant as O
         s, _ = O.calibrate(inp["C"], inp["W"], wl.alpha_f32)
         inp["s"] = s
-        inp["Wq"], inp["ws"] = O.fold_and_quantize_weight(inp["W"], s)
+        # the rows of W the (possibly sampled) forward multiplies by
+        inp["Wq"], inp["ws"] = O.fold_and_quantize_weight(inp["W"][:sample_plan(wl, path)[1]], s)
     return inp
 
 
@@ -376,10 +390,18 @@ def oracle_step_seconds(inp, wl, path="smoothquant"):
         t0 = pc()
         PT.linear_per_tensor(inp["X"], inp["W"], inp["bias"])
         return pc() - t0
-    if path == "forward":
+    if path in FORWARD_CALLS:
+        # quantisation of X, then product + epilogue (on the sampled block for
+        # the prefill layer, each phase scaled by what it covers)
+        mx_rows, mw_rows = sample_plan(wl, path)
+        b = inp["bias"]
         t0 = pc()
-        O.forward(inp["X"], inp["s"], inp["Wq"], inp["ws"], inp["bias"])
-        return pc() - t0
+        Xq, xs = O.quantize_activation(inp["X"][:mx_rows], inp["s"])
+        t1 = pc()
+        acc = O.int8_gemm(Xq, inp["Wq"][:mw_rows])
+        O.dequant_epilogue(acc, xs, inp["ws"][:mw_rows], None if b is None else b[:mw_rows])
+        t2 = pc()
+        return (t1 - t0) * wl.M / mx_rows + (t2 - t1) * (wl.M * wl.N) / (mx_rows * mw_rows)
     mx_rows, mw_rows = sample_plan(wl, path)
     b = inp["bias"]
     t0 = pc()
@@ -402,9 +424,14 @@ def oracle_sample_text(wl, path):
             "weight-only": "quantise W per output channel, bf16 x int8 product",
             "ste-train": "s from the running max, fold+quantise W, forward, straight-through backward",
             "forward": "forward on the prepared weight: quantise X, int8 product, epilogue",
+            "forward-prologue": "forward on the prepared weight: quantise X, int8 product, epilogue",
             "smoothquant": "calibrate, fold+quantise W, quantise X, int8 product, epilogue"}[path]
     if (mx_rows, mw_rows) == (wl.M, wl.N):
         return f"whole {wl.name} steps ({what})"
+    if path in FORWARD_CALLS:
+        return (f"{wl.name} calls ({what}) timed on a sample and extrapolated per phase: activation quantisation "
+                f"on {mx_rows} of {wl.M} X rows, product + epilogue on the {mx_rows}x{mw_rows} block (each phase "
+                f"scaled by the rows it covers)")
     return (f"{wl.name} steps ({what}) timed on a sample and extrapolated per phase: calibration in full, "
             f"weight prep on {mw_rows} of {wl.N} W rows, activation quantisation on {mx_rows} of {wl.M} X rows, "
             f"product + epilogue on the {mx_rows}x{mw_rows} block (each phase scaled by the rows it covers)")
@@ -556,6 +583,8 @@ def run_ours(args, wl, rank, world, local_rank):
          "Y": torch.empty(M, N, dtype=torch.bfloat16, device=dev),
          "ws_cal": torch.empty(sq.sq_calibrate_workspace_bytes(K), dtype=torch.uint8, device=dev),
          "ws_fwd": torch.empty(max(sq.sq_forward_workspace_bytes(M, N, K), 16), dtype=torch.uint8, device=dev),
+         "ws_pro": torch.empty(max(sq.sq_forward_prologue_workspace_bytes(M, K), 16), dtype=torch.uint8,
+                               device=dev),
          "ws_lin": torch.empty(max(sq.sq_workspace_bytes(M, N, K), 16), dtype=torch.uint8, device=dev)}
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     flush_read = torch.ones(FLUSH_READ_BYTES // 4, dtype=torch.int32, device=dev)
@@ -625,6 +654,15 @@ def run_ours(args, wl, rank, world, local_rank):
                                                        workspace=T["ws_fwd"]), ["Wq", "w_scale"], fwd_launches),
         }
         stages = [["sq_forward"]]
+    elif args.path == "forward-prologue":
+        sq.sq_calibrate(T["C"], T["W"], a, s=T["s"], workspace=T["ws_cal"])
+        sq.sq_prepare_weight(T["W"], T["s"], Wq=T["Wq"], w_scale=T["w_scale"])
+        calls = {  # the scale pre-pass and the GEMM
+            "sq_forward_prologue": Call(lambda T: sq.sq_forward_prologue(T["X"], T["s"], T["Wq"], T["w_scale"],
+                                                                         T["b"], Y=T["Y"], workspace=T["ws_pro"]),
+                                        ["Wq", "w_scale"], 2),
+        }
+        stages = [["sq_forward_prologue"]]
     else:
         calls = {
             "sq_calibrate": Call(lambda T: sq.sq_calibrate(T["C"], T["W"], a, s=T["s"], workspace=T["ws_cal"]),
@@ -682,21 +720,22 @@ def run_ours(args, wl, rank, world, local_rank):
         rotations[n] = (r, r * foot >= ROTATE_BYTES)
     torch.cuda.synchronize()
 
-    forward_path = args.path == "forward"
+    forward_path = args.path in FORWARD_CALLS
+    fwd_call = FORWARD_CALLS.get(args.path)
     step_evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)]
     g_step = torch.cuda.CUDAGraph()
     if forward_path:
         # the K timed calls in one graph, each on the next prepared weight copy
-        fsets = sets["sq_forward"]
+        fsets = sets[fwd_call]
         with torch.cuda.graph(g_step):
             step_evs[0].record()
             for k in range(args.steps):
-                calls["sq_forward"].fn(fsets[k % len(fsets)])
+                calls[fwd_call].fn(fsets[k % len(fsets)])
             step_evs[1].record()
         g_warm = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g_warm):
             for k in range(max(args.warmup, 1)):
-                calls["sq_forward"].fn(fsets[k % len(fsets)])
+                calls[fwd_call].fn(fsets[k % len(fsets)])
     else:
         with torch.cuda.graph(g_step):
             step_evs[0].record()
@@ -845,9 +884,13 @@ def run_ours(args, wl, rank, world, local_rank):
                 sq.sq_quantize_per_tensor(D["W"], Aq=D["Wq"], scale_rows=D["w_scale"], workspace=D["ws_pt"])
                 sq.sq_quantize_per_tensor(D["X"], Aq=D["Xq"], scale_rows=D["x_scale"], workspace=D["ws_pt2"])
                 sq.sq_linear(D["Xq"], D["x_scale"], D["Wq"], D["w_scale"], D["b"], Y=D["Y"], workspace=D["ws_lin"])
-            elif forward_path:
+            elif args.path == "forward":
                 F = sets["sq_forward"][i % len(sets["sq_forward"])]
                 sq.sq_forward(D["X"], F["s"], F["Wq"], F["w_scale"], F["b"], Y=D["Y"], workspace=D["ws_fwd"])
+            elif args.path == "forward-prologue":
+                F = sets["sq_forward_prologue"][i % len(sets["sq_forward_prologue"])]
+                sq.sq_forward_prologue(D["X"], F["s"], F["Wq"], F["w_scale"], F["b"], Y=D["Y"],
+                                       workspace=D["ws_pro"])
             else:
                 sq.sq_calibrate(D["C"], D["W"], a, s=D["s"], workspace=D["ws_cal"])
                 sq.sq_prepare_weight(D["W"], D["s"], Wq=D["Wq"], w_scale=D["w_scale"])
@@ -895,6 +938,7 @@ def run_ours(args, wl, rank, world, local_rank):
                 "weight-only": "sq_prepare_weight (s = 1) + sq_linear_weight_only",
                 "per-tensor": "sq_quantize_per_tensor(W) + sq_quantize_per_tensor(X) + sq_linear",
                 "forward": "sq_forward on a prepared weight (X in, Y out)",
+                "forward-prologue": "sq_forward_prologue on a prepared weight (X in, Y out)",
                 "smoothquant": "sq_calibrate + sq_prepare_weight + sq_forward"}[args.path]
         outs = [h_out[0]["Y"]] + ([h_out[0]["d_eta"]] if args.path == "ste-train" else [])
         e2e = {"value": whole_job_rate(wl.M, world, e2e_ms), "unit": UNIT,
@@ -919,7 +963,8 @@ def run_ours(args, wl, rank, world, local_rank):
     if not forward_path:
         cfg["schedule"] = ("serial" if args.serial else
                            " -> ".join("(" + " | ".join(st) + ")" if len(st) > 1 else st[0] for st in stages))
-    gemm_call = next((n for n in ("sq_linear", "sq_forward", "sq_linear_weight_only") if n in per_call), None)
+    gemm_call = next((n for n in ("sq_linear", "sq_forward", "sq_forward_prologue", "sq_linear_weight_only")
+                      if n in per_call), None)
     line = {
         "metric": metric_for(args.path), "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": step_ms, "ms_per_step_median": step_median_ms,

@@ -292,6 +292,31 @@ SQ_API sq_status sq_forward(const sq_bf16* X, const float* s, const int8_t* Wq,
                      int64_t M, int64_t N, int64_t K, sq_bf16* Y,
                      void* workspace, size_t workspace_bytes, void* stream);
 
+/* -------------------------------------- forward, quantisation in the GEMM
+ * sq_forward_prologue -- the same Y as sq_forward, with the per-token
+ * quantisation of X / s done inside the GEMM instead of by a separate pass
+ * that writes Xq to global memory.  Page: forward of SmoothQuantW8A8 once
+ * frozen (X / s, quantize_per_token_symmetric, the int8 product, the
+ * dequantisation and bias).
+ *
+ *   X[M][K] bf16, s[K], Wq[N][K], w_scale[N], bias[N] or NULL -> Y[M][N] bf16
+ *   workspace  at least sq_forward_prologue_workspace_bytes(M, K) bytes; it
+ *              receives x_scale[M] (at offset 0) and RN(1/s_j)[K]; contents on
+ *              entry are ignored.
+ * Two kernels: a pre-pass that reads X once and writes only the per-token
+ * scales (the scales of sq_quantize_act, bit for bit), then a CTA-pair GEMM
+ * (tiles of 256 x 512) whose converter warps read X in bf16 and write the int8
+ * codes straight into the tensor core's shared-memory operand.  The codes, and
+ * so Y, are identical to those of sq_quantize_act followed by sq_linear.
+ * Meant for many tokens (prefill); any M >= 1 is accepted.  K % 16 == 0,
+ * 16 <= K <= 16384; pointers 16-byte aligned (bias may be NULL).
+ */
+SQ_API size_t sq_forward_prologue_workspace_bytes(int64_t M, int64_t K);
+SQ_API sq_status sq_forward_prologue(const sq_bf16* X, const float* s, const int8_t* Wq,
+                              const float* w_scale, const sq_bf16* bias,
+                              int64_t M, int64_t N, int64_t K, sq_bf16* Y,
+                              void* workspace, size_t workspace_bytes, void* stream);
+
 /* ------------------------------------------------------------- test hook
  * sq_gemm_s32 -- the same tcgen05 GEMM main loop with a raw int32 epilogue:
  * acc[M][N] = Xq Wq^T, exposing the accumulator for bit-exact checks.
@@ -321,7 +346,7 @@ SQ_API void sq_debug_fail_after(int n);
 
 /* sq_debug_pipeline_stall -- device-side failure test: while enabled
  * (enable != 0), the GEMM kernels used by sq_linear / sq_forward / sq_gemm_s32
- * for M > 32 never load their first pipeline stage and every pipeline wait gives
+ * for M > 32, and by sq_forward_prologue, never load their first pipeline stage and every pipeline wait gives
  * up after timeout_ns (<= 0: the normal 2 s).  The kernel then sets bit 0 of
  * the device status word, drains its copies in flight, frees its tensor memory
  * and returns: the call's output is invalid, the CUDA context stays usable and

@@ -69,6 +69,9 @@ def test_validation_before_device(sq):
     assert lib.sq_linear(a, a, a, a, mis, 4, 8, 64, a, None, 0, None) == 3
     assert lib.sq_linear(a, a, a, a, None, 4, 8, 200000, a, None, 0, None) == 2
     assert lib.sq_forward(a, a, a, a, None, 4, 8, 64, a, a, 16, None) == 8
+    assert lib.sq_forward_prologue(a, a, a, a, None, 4, 8, 64, a, a, 16, None) == 8      # workspace too small
+    assert lib.sq_forward_prologue(a, mis, a, a, None, 4, 8, 64, a, a, 512, None) == 3   # s misaligned
+    assert lib.sq_forward_prologue(a, a, a, a, None, 4, 8, 16400, a, a, 1 << 20, None) == 2  # K above 16384
     assert lib.sq_gemm_s32(a, a, 4, 0, 64, a, None) == 2
     ws = lib.sq_quantize_per_tensor_workspace_bytes()
     assert ws >= 4

@@ -120,3 +120,21 @@ def test_forward_work_counts_the_weight_stream():
     kernels, roof = bench.kernel_report(wl, ["sq_forward"], {"sq_forward": 0.012}, {"sq_forward": 0.018},
                                         {"sq_forward": 1})
     assert roof["bound"] == "hbm" and roof["kernel"] == "sq_forward"
+
+
+def test_forward_paths_sample_the_prefill_oracle():
+    """The per-call forward paths time the oracle's forward whole on the
+    smaller layers and on a sampled block at prefill size; the sampled form
+    runs through the same phases (checked on the tiny layer, whole)."""
+    wl = workloads.get("prefill")
+    for path in ("forward", "forward-prologue"):
+        mx, mw = bench.sample_plan(wl, path)
+        assert mx < wl.M and mw < wl.N
+        assert "extrapolated" in bench.oracle_sample_text(wl, path)
+    tiny = workloads.get("tiny")
+    assert bench.sample_plan(tiny, "forward-prologue") == (tiny.M, tiny.N)
+    inp = bench.oracle_inputs(tiny, "forward-prologue")
+    assert inp["Wq"].shape == (tiny.N, tiny.K)
+    assert bench.oracle_step_seconds(inp, tiny, "forward-prologue") > 0
+    nb, ops, typ = bench.algorithmic_work(wl)["sq_forward_prologue"]
+    assert nb == bench.algorithmic_work(wl)["sq_forward"][0] and ops == 2 * wl.M * wl.N * wl.K

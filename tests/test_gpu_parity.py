@@ -59,6 +59,14 @@ def _stages(sq, C, W, X, bias, alpha, label, report):
     # fused forward = the two kernels above, bit for bit
     Y_f = sq.sq_forward(Xd, s_g, Wq_g, ws_g, bd)
     assert torch.equal(Y_f.view(torch.int16), Y_g.view(torch.int16)), f"{label}: sq_forward != sq_linear(quantize_act)"
+    # quantisation inside the GEMM: the same codes, so the same Y bit for bit,
+    # and the pre-pass's x_scale (workspace offset 0) equal to sq_quantize_act's
+    M = X.shape[0]
+    wsp = torch.full((sq.sq_forward_prologue_workspace_bytes(M, K),), 0x7F, dtype=torch.uint8, device="cuda")
+    Y_p = sq.sq_forward_prologue(Xd, s_g, Wq_g, ws_g, bd, workspace=wsp)
+    assert torch.equal(Y_p.view(torch.int16), Y_g.view(torch.int16)), \
+        f"{label}: sq_forward_prologue != sq_linear(quantize_act)"
+    assert torch.equal(wsp[:4 * M].view(torch.float32), xs_g), f"{label}: pre-pass x_scale != sq_quantize_act's"
     torch.cuda.synchronize()
     return dict(s=s_g, Wq=Wq_g, ws=ws_g, Xq=Xq_g, xs=xs_g, Y=Y_g, Yf=Y_f)
 
@@ -176,6 +184,11 @@ def test_tiny_values_and_subnormal_quotients(sq, K):
     assert_codes(host(Wq), Wq_o, vw, "tiny W: codes")
     floor_scale = np.float32(np.float32(1e-8) / np.float32(127))
     assert host(xs)[0] == floor_scale and host(xs)[6] == floor_scale
+    # the GEMM that quantises X itself makes the same codes in this range:
+    # its Y equals sq_linear on the row quantiser's codes, bit for bit
+    Y_l = sq.sq_linear(Xq, xs, Wq, ws)
+    Y_p = sq.sq_forward_prologue(dev_bf16(X), sd, Wq, ws)
+    assert torch.equal(Y_p.view(torch.int16), Y_l.view(torch.int16))
 
 
 def test_accumulator_extremes(sq):
@@ -276,6 +289,11 @@ def test_status_codes(sq):
     assert lib.sq_forward(p(X), p(s), p(Wq), p(w_scale), None, 4, 8, 64, p(Y), p(ws), 16, None) == 8
     with pytest.raises(ValueError):
         sq.sq_forward(X, s, Wq, w_scale, workspace=ws)
+    assert sq.sq_forward_prologue_workspace_bytes(4, 64) == 512
+    assert lib.sq_forward_prologue(p(X), p(s), p(Wq), p(w_scale), None, 4, 8, 64, p(Y), p(ws), 16, None) == 8
+    big = torch.empty(512, dtype=torch.uint8, device="cuda")
+    assert lib.sq_forward_prologue(p(X), p(s, 4), p(Wq), p(w_scale), None, 4, 8, 64, p(Y), p(big), 512, None) == 3
+    assert lib.sq_forward_prologue(p(X), p(s), p(Wq), p(w_scale), None, 4, 8, 40, p(Y), p(big), 512, None) == 3
 
 
 def test_fault_injection(sq):
@@ -306,6 +324,10 @@ def test_prefill_full_size_sampled(sq):
     s_g = sq.sq_calibrate(Cd, Wd, wl.alpha_f32)
     Wq_g, ws_g = sq.sq_prepare_weight(Wd, s_g)
     Y_g = sq.sq_forward(Xd, s_g, Wq_g, ws_g)
+    # activation quantisation inside the GEMM: every element equal
+    Y_p = sq.sq_forward_prologue(Xd, s_g, Wq_g, ws_g)
+    assert torch.equal(Y_p.view(torch.int16), Y_g.view(torch.int16)), "prefill: sq_forward_prologue != sq_forward"
+    del Y_p
     torch.cuda.synchronize()
     s_o, _ = O.calibrate(inp["C"], inp["W"], wl.alpha_f32)
     assert_scales_close(host(s_g), s_o, "prefill: s")

@@ -99,3 +99,34 @@ def test_cta_pair_wait_timeout_is_reported_and_the_context_survives(sq):
     acc = host(sq.sq_gemm_s32(Xq_d, Wq_d))
     assert np.array_equal(acc.astype(np.int64), O.int8_gemm(Xq, Wq))
     assert sq.sq_device_status() == 0
+
+
+def test_fused_prologue_wait_timeout_is_reported_and_the_context_survives(sq):
+    """The same failure in the GEMM that quantises X itself (CTA pairs, 256 x
+    512 tiles, converter warps feeding the A operand): the Wq producers skip
+    their first stage, so the MMA's first wait gives up; every other wait of
+    both CTAs (converters, X producer, epilogue) gives up in turn."""
+    rng = np.random.default_rng(96)
+    M, N, K = 1024, 4096, 1024  # 4 x 8 pair tiles, 8 k-blocks: more than the ring holds
+    X = torch.randn(M, K, device="cuda").to(torch.bfloat16)
+    s = (torch.rand(K, device="cuda") + 0.5).float()
+    Wq = dev(rng.integers(-127, 128, (N, K), dtype=np.int64).astype(np.int8))
+    ws = dev((rng.random(N, dtype=np.float32) * 1e-3 + 1e-4).astype(np.float32))
+    assert sq.sq_device_status(clear=True) == 0
+    try:
+        sq.sq_debug_pipeline_stall(True, 50_000_000)
+        t0 = time.perf_counter()
+        sq.sq_forward_prologue(X, s, Wq, ws)
+        torch.cuda.synchronize()
+        elapsed = time.perf_counter() - t0
+    finally:
+        sq.sq_debug_pipeline_stall(False)
+    flags = sq.sq_device_status(clear=True)
+    assert flags & 1, "the stalled fused-prologue pipeline was not reported"
+    assert elapsed < 5.0
+    Y = sq.sq_forward_prologue(X, s, Wq, ws)
+    Xq, xs = sq.sq_quantize_act(X, s)
+    Y_l = sq.sq_linear(Xq, xs, Wq, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(Y.view(torch.int16), Y_l.view(torch.int16))
+    assert sq.sq_device_status() == 0

@@ -24,7 +24,7 @@ __all__ = [
     "sq_version", "sq_calibrate", "sq_calibrate_workspace_bytes", "sq_calibrate_noalloc", "sq_prepare_weight",
     "sq_quantize_act", "sq_quantize_per_tensor", "sq_quantize_per_tensor_workspace_bytes", "sq_linear_weight_only", "sq_ste_backward",
     "sq_ste_backward_workspace_bytes", "sq_linear", "sq_workspace_bytes", "sq_forward",
-    "sq_forward_workspace_bytes", "sq_gemm_s32", "sq_device_status", "sq_debug_fail_after",
+    "sq_forward_workspace_bytes", "sq_forward_prologue", "sq_forward_prologue_workspace_bytes", "sq_gemm_s32", "sq_device_status", "sq_debug_fail_after",
     "sq_debug_pipeline_stall",
     "STATUS",
 ]
@@ -61,6 +61,8 @@ _SIGNATURES = [
     ("sq_linear", ctypes.c_int, (_P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _SZ, _P)),
     ("sq_forward_workspace_bytes", _SZ, (_I64, _I64, _I64)),
     ("sq_forward", ctypes.c_int, (_P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _SZ, _P)),
+    ("sq_forward_prologue_workspace_bytes", _SZ, (_I64, _I64)),
+    ("sq_forward_prologue", ctypes.c_int, (_P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _SZ, _P)),
     ("sq_gemm_s32", ctypes.c_int, (_P, _P, _I64, _I64, _I64, _P, _P)),
     ("sq_device_status", ctypes.c_int, (ctypes.POINTER(ctypes.c_uint32), ctypes.c_int)),
     ("sq_debug_fail_after", None, (ctypes.c_int,)),
@@ -368,6 +370,36 @@ def sq_forward(X: torch.Tensor, s: torch.Tensor, Wq: torch.Tensor, w_scale: torc
     ws = _workspace(workspace, sq_forward_workspace_bytes(M, N, K), X.device)
     _check(_load().sq_forward(_ptr(X), _ptr(s), _ptr(Wq), _ptr(w_scale), _ptr(bias), M, N, K, _ptr(Y), _ptr(ws),
                           ws.numel(), _stream(stream)))
+    return Y
+
+
+def sq_forward_prologue_workspace_bytes(M: int, K: int) -> int:
+    return int(_load().sq_forward_prologue_workspace_bytes(M, K))
+
+
+def sq_forward_prologue(X: torch.Tensor, s: torch.Tensor, Wq: torch.Tensor, w_scale: torch.Tensor,
+                        bias: Optional[torch.Tensor] = None, Y: Optional[torch.Tensor] = None,
+                        workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Y[M,N] bf16 from X[M,K] bf16 like ``sq_forward``, with the per-token
+    quantisation done inside the GEMM (a scale pre-pass, then converter warps
+    that write the codes into the tensor core's shared-memory operand).  The
+    workspace receives x_scale[M] at offset 0."""
+    _want(X, "X", torch.bfloat16, 2)
+    _want(s, "s", torch.float32, 1)
+    _want(Wq, "Wq", torch.int8, 2)
+    _want(w_scale, "w_scale", torch.float32, 1)
+    M, K = X.shape
+    N = Wq.shape[0]
+    if Wq.shape[1] != K or s.shape[0] != K or w_scale.shape[0] != N:
+        raise ValueError("inconsistent shapes")
+    if bias is not None:
+        _want(bias, "bias", torch.bfloat16, 1)
+        if bias.shape[0] != N:
+            raise ValueError("bias must have N entries")
+    Y = _out(Y, (M, N), torch.bfloat16, X.device, "Y")
+    ws = _workspace(workspace, sq_forward_prologue_workspace_bytes(M, K), X.device)
+    _check(_load().sq_forward_prologue(_ptr(X), _ptr(s), _ptr(Wq), _ptr(w_scale), _ptr(bias), M, N, K, _ptr(Y),
+                                   _ptr(ws), ws.numel(), _stream(stream)))
     return Y
 
 

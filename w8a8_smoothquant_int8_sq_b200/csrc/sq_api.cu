@@ -425,6 +425,38 @@ sq_status sq_forward(const sq_bf16* X, const float* s, const int8_t* Wq, const f
                      static_cast<char*>(workspace) + gemm_off, workspace_bytes - gemm_off);
 }
 
+// ------------------------------------- forward, quantisation in the GEMM
+size_t sq_forward_prologue_workspace_bytes(int64_t M, int64_t K) {
+  if (M <= 0 || K <= 0) return 0;
+  return round_up(static_cast<size_t>(M) * sizeof(float), 256) + round_up(static_cast<size_t>(K) * sizeof(float), 256);
+}
+
+sq_status sq_forward_prologue(const sq_bf16* X, const float* s, const int8_t* Wq, const float* w_scale,
+                              const sq_bf16* bias, int64_t M, int64_t N, int64_t K, sq_bf16* Y, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+  SQ_TRY(check_k(K, sq::kMaxQuantK));
+  SQ_TRY(check_rows(M, "M"));
+  SQ_TRY(check_rows(N, "N"));
+  SQ_NONNULL(X);
+  SQ_NONNULL(s);
+  SQ_NONNULL(Wq);
+  SQ_NONNULL(w_scale);
+  SQ_NONNULL(Y);
+  if (bias != nullptr && !aligned16(bias)) return fail(SQ_ERR_ALIGN, "bias is not 16-byte aligned");
+  if (workspace == nullptr || workspace_bytes < sq_forward_prologue_workspace_bytes(M, K))
+    return fail(SQ_ERR_WORKSPACE, "workspace must hold sq_forward_prologue_workspace_bytes(M, K) = " +
+                                      std::to_string(sq_forward_prologue_workspace_bytes(M, K)) + " bytes");
+  if (!aligned16(workspace)) return fail(SQ_ERR_ALIGN, "workspace is not 16-byte aligned");
+  sq::DeviceInfo dev;
+  SQ_TRY(prologue(&dev));
+  float* xs = static_cast<float*>(workspace);
+  float* rs = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                       round_up(static_cast<size_t>(M) * sizeof(float), 256));
+  sq::PrologueArgs a{X, s, Wq, w_scale, bias, M, N, K, Y, xs, rs};
+  const char* why = "fused-prologue forward";
+  return cuda_status(sq::launch_forward_prologue(a, static_cast<cudaStream_t>(stream), dev, &why), why);
+}
+
 // ---------------------------------------------------------------- test hook
 sq_status sq_gemm_s32(const int8_t* Xq, const int8_t* Wq, int64_t M, int64_t N, int64_t K, int32_t* acc,
                       void* stream) {

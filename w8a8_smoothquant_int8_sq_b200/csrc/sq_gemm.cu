@@ -453,6 +453,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 namespace sq {
 namespace {
 #include "sq_gemm_pair.cuh"
+#include "sq_gemm_prologue.cuh"
 }  // namespace
 }  // namespace sq
 
@@ -611,19 +612,19 @@ cudaError_t run_small(const SmallArgs& a, cudaStream_t st, const DeviceInfo& dev
   return e;
 }
 
-// Clusters of two CTAs that can run at once with the pair kernel's shared
-// memory (cached per device): the pair kernel's persistent grid.
-int pair_clusters(const DeviceInfo& dev) {
+// Clusters of two CTAs of `kern` (threads, smem bytes) that can run at once:
+// the persistent grid of a CTA-pair kernel.  Cached per device in `cache`.
+template <typename Kern>
+int max_pair_clusters(Kern kern, int threads, int smem, const DeviceInfo& dev, int (&cache)[64]) {
   static std::mutex mu;
-  static int cached[64] = {};
   std::lock_guard<std::mutex> lk(mu);
   if (dev.device < 0 || dev.device >= 64) return 0;
-  if (cached[dev.device] != 0) return cached[dev.device];
+  if (cache[dev.device] != 0) return cache[dev.device];
   int n = 0;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * static_cast<unsigned>(dev.sm_count / 2));
-  cfg.blockDim = dim3(kPairThreads);
-  cfg.dynamicSmemBytes = kPairAlloc;
+  cfg.blockDim = dim3(static_cast<unsigned>(threads));
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
@@ -631,12 +632,21 @@ int pair_clusters(const DeviceInfo& dev) {
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  auto kern = gemm_i8_pair_kernel<0>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kPairAlloc) != cudaSuccess ||
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
       cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess)
     n = 0;
-  cached[dev.device] = n > 0 ? n : -1;
-  return cached[dev.device];
+  cache[dev.device] = n > 0 ? n : -1;
+  return cache[dev.device];
+}
+
+int pair_clusters(const DeviceInfo& dev) {
+  static int cache[64] = {};
+  return max_pair_clusters(gemm_i8_pair_kernel<0>, kPairThreads, kPairAlloc, dev, cache);
+}
+
+int prologue_clusters(const DeviceInfo& dev) {
+  static int cache[64] = {};
+  return max_pair_clusters(gemm_i8_prologue_kernel, kFThreads, kFAlloc, dev, cache);
 }
 
 template <int EPI>
@@ -776,6 +786,58 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t st, const DeviceInfo& de
   return wide ? run_gemm<256, 4, 1, 1>(a, st, dev, why) : run_gemm<128, 6, 1, SQ_GEMM_CHAINS128>(a, st, dev, why);
 }
 
+cudaError_t launch_forward_prologue(const PrologueArgs& a, cudaStream_t st, const DeviceInfo& dev, const char** why) {
+  // pre-pass: x_scale[M] and RN(1/s)[K]
+  cudaError_t e = launch_act_scales(a.X, a.M, a.K, a.s, a.x_scale, a.rs, st, dev);
+  if (e != cudaSuccess) {
+    *why = "scale pre-pass launch";
+    return e;
+  }
+  const int clusters = prologue_clusters(dev);
+  if (clusters <= 0) {
+    *why = "the fused-prologue GEMM cannot be resident on this device";
+    return cudaErrorNotSupported;
+  }
+  CUtensorMap tmX, tmB;
+  if (!make_tmap_2d(&tmX, a.X, a.M, a.K, 2, kFXCols, kFHalf) || !make_tmap_i8(&tmB, a.Wq, a.N, a.K, kFHalf)) {
+    *why = "cuTensorMapEncodeTiled failed or unavailable";
+    return cudaErrorInvalidValue;
+  }
+  PrologueParams p;
+  p.timeout_ns = g_debug_stall.load() ? g_debug_timeout_ns.load() : kWaitTimeoutNs;
+  p.skip_first_load = g_debug_stall.load() ? 1 : 0;
+  p.M = static_cast<int>(a.M);
+  p.N = static_cast<int>(a.N);
+  p.K = static_cast<int>(a.K);
+  p.num_m_blocks = static_cast<int>((a.M + kFBM - 1) / kFBM);
+  p.num_n_blocks = static_cast<int>((a.N + kFBN - 1) / kFBN);
+  p.num_k_blocks = static_cast<int>((a.K + kBK - 1) / kBK);
+  p.group_m = tile_group_m(kFBM, 2 * a.K, p.num_m_blocks);  // groups of bf16 X rows
+  p.s = a.s;
+  p.rs = a.rs;
+  p.x_scale = a.x_scale;
+  p.w_scale = a.w_scale;
+  p.bias = a.bias;
+  p.out = a.Y;
+  p.vec_ok = (a.N % 8 == 0) && (reinterpret_cast<uintptr_t>(a.Y) % 16 == 0) &&
+             (reinterpret_cast<uintptr_t>(a.w_scale) % 16 == 0) &&
+             (a.bias == nullptr || reinterpret_cast<uintptr_t>(a.bias) % 16 == 0);
+  auto kern = gemm_i8_prologue_kernel;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kFAlloc);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, kCarveoutMaxShared);
+  if (e != cudaSuccess) {
+    *why = "cudaFuncSetAttribute failed";
+    return e;
+  }
+  const int tiles = p.num_m_blocks * p.num_n_blocks;
+  const int pairs = std::min(tiles, clusters);
+  e = launch_pdl_cluster(kern, dim3(2u * static_cast<unsigned>(pairs)), dim3(kFThreads), static_cast<size_t>(kFAlloc),
+                         st, 2u, tmX, tmB, p);
+  if (e != cudaSuccess) *why = "cluster launch of the fused-prologue GEMM failed";
+  return e;
+}
+
 #ifdef SQ_TRACE
 extern "C" __attribute__((visibility("default"))) int sq_trace_read_sk(unsigned long long* host, int n) {
   return cudaMemcpyFromSymbol(host, g_sk_trace, sizeof(unsigned long long) * 8 * static_cast<size_t>(n)) ==
@@ -786,6 +848,13 @@ extern "C" __attribute__((visibility("default"))) int sq_trace_read_sk(unsigned 
 extern "C" __attribute__((visibility("default"))) int sq_trace_read_big(unsigned long long* host, int n) {
   return cudaMemcpyFromSymbol(host, g_big_trace, sizeof(unsigned long long) * 5 * static_cast<size_t>(n)) ==
                  cudaSuccess
+             ? 0
+             : 1;
+}
+extern "C" __attribute__((visibility("default"))) int sq_trace_read_prologue(unsigned long long* conv,
+                                                                             unsigned long long* x) {
+  return cudaMemcpyFromSymbol(conv, sq::g_pro_trace, sizeof(sq::g_pro_trace)) == cudaSuccess &&
+                 cudaMemcpyFromSymbol(x, sq::g_pro_xtrace, sizeof(sq::g_pro_xtrace)) == cudaSuccess
              ? 0
              : 1;
 }

@@ -96,6 +96,12 @@ cudaError_t launch_calibrate_noalloc(const uint16_t* C, int64_t R, int64_t K, co
 cudaError_t launch_row_quant(bool multiply, const uint16_t* src, int64_t rows, int64_t K, const float* s,
                              int8_t* q, float* scale, cudaStream_t st, const DeviceInfo& dev);
 
+// Activation scales only (the pre-pass of launch_forward_prologue):
+// scale[m] exactly as launch_row_quant(false, ...) computes it, no codes, and
+// RN(1/s_j) into recip[K] (16-byte aligned).
+cudaError_t launch_act_scales(const uint16_t* X, int64_t rows, int64_t K, const float* s, float* scale, float* recip,
+                              cudaStream_t st, const DeviceInfo& dev);
+
 // ---- per-tensor quantisation, the baseline beside SmoothQuant (sq_quant.cu)
 // Workspace: one partial maximum per pass-1 block.
 size_t per_tensor_workspace_bytes();
@@ -159,6 +165,23 @@ struct SmallArgs {
   uint16_t* Y;            // [M][N]
 };
 cudaError_t launch_small_m(const SmallArgs& a, cudaStream_t st, const DeviceInfo& dev, const char** why);
+
+// Many tokens, activation quantisation fused into the GEMM: a pre-pass writes
+// x_scale[M] and RN(1/s)[K] (caller scratch, 16-byte aligned), then a CTA-pair
+// GEMM converts bf16 X to codes in shared memory as it goes (codes, scales and
+// Y identical to launch_row_quant followed by launch_gemm).  Needs K % 16 == 0.
+struct PrologueArgs {
+  const uint16_t* X;      // [M][K] bf16
+  const float* s;         // [K]
+  const int8_t* Wq;       // [N][K]
+  const float* w_scale;   // [N]
+  const uint16_t* bias;   // [N] or null
+  int64_t M, N, K;
+  uint16_t* Y;            // [M][N]
+  float* x_scale;         // scratch [M]
+  float* rs;              // scratch [K]
+};
+cudaError_t launch_forward_prologue(const PrologueArgs& a, cudaStream_t st, const DeviceInfo& dev, const char** why);
 
 // Test hook: while enabled, the general GEMM's producer skips its first stage
 // and every wait gives up after timeout_ns (the kernel then reports bit 0).

@@ -421,10 +421,14 @@ __device__ __forceinline__ void load_row_vectors(uint4 (&xv)[VPL], const uint16_
   }
 }
 
-template <bool kMul, int WPR, int VPL>
+// kCodes == false (activations only): the scales alone, no codes (q unused);
+// block 0 also writes RN(1/s_j) to recip[K] when recip is not null.  This is
+// the pre-pass of the GEMM that quantises its A operand itself.
+template <bool kMul, int WPR, int VPL, bool kCodes = true>
 __global__ void __launch_bounds__(kRowThreads) row_quant_kernel(const uint16_t* __restrict__ src, int64_t rows, int K,
                                                                 const float* __restrict__ s, int8_t* __restrict__ q,
-                                                                float* __restrict__ scale) {
+                                                                float* __restrict__ scale,
+                                                                float* __restrict__ recip) {
   constexpr int RPC = 8 / WPR;  // rows per block in flight
   // Table, one float4 pair per 16-byte vector of 8 columns:
   //   weights:     sA = s[8v..8v+3], sB = s[8v+4..8v+7]
@@ -469,8 +473,14 @@ __global__ void __launch_bounds__(kRowThreads) row_quant_kernel(const uint16_t* 
     } else {
       sA[v] = make_float4(-a.x, -a.y, -a.z, -a.w);
       sB[v] = make_float4(-b.x, -b.y, -b.z, -b.w);
-      rA[v] = make_float4(__frcp_rn(a.x), __frcp_rn(a.y), __frcp_rn(a.z), __frcp_rn(a.w));
-      rB[v] = make_float4(__frcp_rn(b.x), __frcp_rn(b.y), __frcp_rn(b.z), __frcp_rn(b.w));
+      const float4 ra = make_float4(__frcp_rn(a.x), __frcp_rn(a.y), __frcp_rn(a.z), __frcp_rn(a.w));
+      const float4 rb = make_float4(__frcp_rn(b.x), __frcp_rn(b.y), __frcp_rn(b.z), __frcp_rn(b.w));
+      rA[v] = ra;
+      rB[v] = rb;
+      if (!kCodes && recip != nullptr && blockIdx.x == 0) {
+        reinterpret_cast<float4*>(recip)[2 * v] = ra;
+        reinterpret_cast<float4*>(recip)[2 * v + 1] = rb;
+      }
     }
   }
   __syncthreads();
@@ -528,17 +538,19 @@ __global__ void __launch_bounds__(kRowThreads) row_quant_kernel(const uint16_t* 
     // equal to the IEEE quotient for every fp32 from 1e-8 up (checked
     // exhaustively on the CPU)
     const float sc = div_rn(fmaxf(m, kClampFloor), kQmax, r127);
-    const float rsc = __frcp_rn(sc);
-    const f2x nsc2 = f2_pack(-sc, -sc), rsc2 = f2_pack(rsc, rsc);
-    int8_t* qr = q + row * static_cast<int64_t>(K);
+    if (kCodes) {
+      const float rsc = __frcp_rn(sc);
+      const f2x nsc2 = f2_pack(-sc, -sc), rsc2 = f2_pack(rsc, rsc);
+      int8_t* qr = q + row * static_cast<int64_t>(K);
 #pragma unroll
-    for (int i = 0; i < VPL; ++i) {
-      const int v = i * (32 * WPR) + wsub * 32 + lane;
-      if (v < nvec) {
-        f2x c[4];
+      for (int i = 0; i < VPL; ++i) {
+        const int v = i * (32 * WPR) + wsub * 32 + lane;
+        if (v < nvec) {
+          f2x c[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) c[e] = f2_round_codes(f2_div_rn(t[i][e], nsc2, rsc2));
-        *reinterpret_cast<uint2*>(qr + static_cast<int64_t>(v) * 8) = pack8_codes(c[0], c[1], c[2], c[3]);
+          for (int e = 0; e < 4; ++e) c[e] = f2_round_codes(f2_div_rn(t[i][e], nsc2, rsc2));
+          *reinterpret_cast<uint2*>(qr + static_cast<int64_t>(v) * 8) = pack8_codes(c[0], c[1], c[2], c[3]);
+        }
       }
     }
     if (wsub == 0 && lane == 0) scale[row] = sc;
@@ -546,11 +558,11 @@ __global__ void __launch_bounds__(kRowThreads) row_quant_kernel(const uint16_t* 
   }
 }
 
-template <bool kMul, int WPR, int VPL>
+template <bool kMul, int WPR, int VPL, bool kCodes>
 static cudaError_t launch_rq(const uint16_t* src, int64_t rows, int K, const float* s, int8_t* q, float* scale,
-                             cudaStream_t st, const DeviceInfo& dev) {
+                             float* recip, cudaStream_t st, const DeviceInfo& dev) {
   const size_t smem = static_cast<size_t>(K / 8) * sizeof(float4) * (kMul ? 2 : 4);
-  auto kern = row_quant_kernel<kMul, WPR, VPL>;
+  auto kern = row_quant_kernel<kMul, WPR, VPL, kCodes>;
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
@@ -564,28 +576,29 @@ static cudaError_t launch_rq(const uint16_t* src, int64_t rows, int K, const flo
   constexpr int RPC = 8 / WPR;
   const int64_t groups = (rows + RPC - 1) / RPC;
   const int64_t grid = std::min<int64_t>(groups, static_cast<int64_t>(dev.sm_count) * per_sm);
-  return launch_pdl(kern, dim3(static_cast<unsigned>(grid)), dim3(kRowThreads), smem, st, src, rows, K, s, q, scale);
+  return launch_pdl(kern, dim3(static_cast<unsigned>(grid)), dim3(kRowThreads), smem, st, src, rows, K, s, q, scale,
+                    recip);
 }
 
 #ifndef SQ_RQ_VPL  // build-time tuning knob: most 16-byte vectors a lane holds (4 or 8)
 #define SQ_RQ_VPL 4
 #endif
 
-template <bool kMul>
+template <bool kMul, bool kCodes = true>
 static cudaError_t dispatch_rq(const uint16_t* src, int64_t rows, int K, const float* s, int8_t* q, float* scale,
-                               cudaStream_t st, const DeviceInfo& dev) {
+                               cudaStream_t st, const DeviceInfo& dev, float* recip = nullptr) {
   // vectors per lane (up to SQ_RQ_VPL), then warps per row (up to 8) to cover K
   constexpr int V = SQ_RQ_VPL;
   static_assert(V == 4 || V == 8, "SQ_RQ_VPL must be 4 or 8");
   const int nvec = K / 8;
-  if (nvec <= 32) return launch_rq<kMul, 1, 1>(src, rows, K, s, q, scale, st, dev);
-  if (nvec <= 64) return launch_rq<kMul, 1, 2>(src, rows, K, s, q, scale, st, dev);
-  if (nvec <= 128) return launch_rq<kMul, 1, 4>(src, rows, K, s, q, scale, st, dev);
-  if (nvec <= 32 * V) return launch_rq<kMul, 1, V>(src, rows, K, s, q, scale, st, dev);
-  if (nvec <= 64 * V) return launch_rq<kMul, 2, V>(src, rows, K, s, q, scale, st, dev);
-  if (nvec <= 128 * V) return launch_rq<kMul, 4, V>(src, rows, K, s, q, scale, st, dev);
-  if (nvec <= 256 * V) return launch_rq<kMul, 8, V>(src, rows, K, s, q, scale, st, dev);
-  return launch_rq<kMul, 8, 8>(src, rows, K, s, q, scale, st, dev);  // K up to 16384
+  if (nvec <= 32) return launch_rq<kMul, 1, 1, kCodes>(src, rows, K, s, q, scale, recip, st, dev);
+  if (nvec <= 64) return launch_rq<kMul, 1, 2, kCodes>(src, rows, K, s, q, scale, recip, st, dev);
+  if (nvec <= 128) return launch_rq<kMul, 1, 4, kCodes>(src, rows, K, s, q, scale, recip, st, dev);
+  if (nvec <= 32 * V) return launch_rq<kMul, 1, V, kCodes>(src, rows, K, s, q, scale, recip, st, dev);
+  if (nvec <= 64 * V) return launch_rq<kMul, 2, V, kCodes>(src, rows, K, s, q, scale, recip, st, dev);
+  if (nvec <= 128 * V) return launch_rq<kMul, 4, V, kCodes>(src, rows, K, s, q, scale, recip, st, dev);
+  if (nvec <= 256 * V) return launch_rq<kMul, 8, V, kCodes>(src, rows, K, s, q, scale, recip, st, dev);
+  return launch_rq<kMul, 8, 8, kCodes>(src, rows, K, s, q, scale, recip, st, dev);  // K up to 16384
 }
 
 // ============================================ per-tensor quantisation (baseline)
@@ -703,6 +716,11 @@ cudaError_t launch_row_quant(bool multiply, const uint16_t* src, int64_t rows, i
   const int Ki = static_cast<int>(K);
   return multiply ? dispatch_rq<true>(src, rows, Ki, s, q, scale, st, dev)
                   : dispatch_rq<false>(src, rows, Ki, s, q, scale, st, dev);
+}
+
+cudaError_t launch_act_scales(const uint16_t* X, int64_t rows, int64_t K, const float* s, float* scale, float* recip,
+                              cudaStream_t st, const DeviceInfo& dev) {
+  return dispatch_rq<false, false>(X, rows, static_cast<int>(K), s, nullptr, scale, st, dev, recip);
 }
 
 }  // namespace sq
