@@ -80,9 +80,12 @@ __device__ __forceinline__ f2x f2_add(f2x a, f2x b) {
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
 }
-// the two bf16 values of a 32-bit word, widened exactly to an fp32 pair
+// the two bf16 values of a 32-bit word, widened exactly to an fp32 pair (two
+// 32-bit operations into the halves of a register pair)
 __device__ __forceinline__ f2x f2_from_bf16x2(uint32_t w) {
-  return (static_cast<f2x>(w & 0xFFFF0000u) << 32) | static_cast<f2x>(w << 16);
+  f2x d;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "r"(w << 16), "r"(w & 0xFFFF0000u));
+  return d;
 }
 // a / b per lane, correctly rounded, given nb = -b and rb = RN(1/b) (div_rn)
 __device__ __forceinline__ f2x f2_div_rn(f2x a, f2x nb, f2x rb) {

@@ -408,7 +408,9 @@ constexpr int kRowThreads = 256;
 #define SQ_RQ_EARLY_L2 4
 #endif
 
-template <int VPL, int WPR>
+// kExact: the row fills the WPR warps' VPL vectors exactly (K == 256 VPL WPR),
+// so no vector index needs a bounds check.
+template <int VPL, int WPR, bool kExact>
 __device__ __forceinline__ void load_row_vectors(uint4 (&xv)[VPL], const uint16_t* __restrict__ src, int64_t row,
                                                  int64_t rows, int K, int nvec, int wsub, int lane) {
   if (row < rows) {
@@ -416,15 +418,16 @@ __device__ __forceinline__ void load_row_vectors(uint4 (&xv)[VPL], const uint16_
 #pragma unroll
     for (int i = 0; i < VPL; ++i) {
       const int v = i * (32 * WPR) + wsub * 32 + lane;
-      xv[i] = (v < nvec) ? __ldcs(xr + v) : make_uint4(0u, 0u, 0u, 0u);
+      xv[i] = (kExact || v < nvec) ? __ldcs(xr + v) : make_uint4(0u, 0u, 0u, 0u);
     }
   }
 }
 
+// kExact: K == 256 * VPL * WPR (every vector index in range; no bounds checks).
 // kCodes == false (activations only): the scales alone, no codes (q unused);
 // block 0 also writes RN(1/s_j) to recip[K] when recip is not null.  This is
 // the pre-pass of the GEMM that quantises its A operand itself.
-template <bool kMul, int WPR, int VPL, bool kCodes = true>
+template <bool kMul, int WPR, int VPL, bool kCodes, bool kExact>
 __global__ void __launch_bounds__(kRowThreads) row_quant_kernel(const uint16_t* __restrict__ src, int64_t rows, int K,
                                                                 const float* __restrict__ s, int8_t* __restrict__ q,
                                                                 float* __restrict__ scale,
@@ -462,7 +465,7 @@ __global__ void __launch_bounds__(kRowThreads) row_quant_kernel(const uint16_t* 
   SQ_BLOCK_MARK(1);
   griddep_launch_dependents();
   uint4 xv[VPL];
-  load_row_vectors<VPL, WPR>(xv, src, row, rows, K, nvec, wsub, lane);  // in flight during the table build
+  load_row_vectors<VPL, WPR, kExact>(xv, src, row, rows, K, nvec, wsub, lane);  // in flight during the table build
 
   const float4* s4 = reinterpret_cast<const float4*>(s);
   for (int v = tid; v < nvec; v += kRowThreads) {
@@ -493,7 +496,7 @@ __global__ void __launch_bounds__(kRowThreads) row_quant_kernel(const uint16_t* 
 #pragma unroll
     for (int i = 0; i < VPL; ++i) {
       const int v = i * (32 * WPR) + wsub * 32 + lane;
-      if (v < nvec) {
+      if (kExact || v < nvec) {
         const uint4 w = xv[i];
         const f2x x[4] = {f2_from_bf16x2(w.x), f2_from_bf16x2(w.y), f2_from_bf16x2(w.z), f2_from_bf16x2(w.w)};
         // one 16-byte table read per float4: consecutive lanes, consecutive
@@ -517,7 +520,7 @@ __global__ void __launch_bounds__(kRowThreads) row_quant_kernel(const uint16_t* 
       }
     }
     const int64_t next = row + row_step;
-    load_row_vectors<VPL, WPR>(xv, src, next, rows, K, nvec, wsub, lane);  // prefetch
+    load_row_vectors<VPL, WPR, kExact>(xv, src, next, rows, K, nvec, wsub, lane);  // prefetch
 #if SQ_RQ_L2_AHEAD
     {
       // and the row after that into L2, so the register prefetch above finds
@@ -545,7 +548,7 @@ __global__ void __launch_bounds__(kRowThreads) row_quant_kernel(const uint16_t* 
 #pragma unroll
       for (int i = 0; i < VPL; ++i) {
         const int v = i * (32 * WPR) + wsub * 32 + lane;
-        if (v < nvec) {
+        if (kExact || v < nvec) {
           f2x c[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) c[e] = f2_round_codes(f2_div_rn(t[i][e], nsc2, rsc2));
@@ -562,7 +565,9 @@ template <bool kMul, int WPR, int VPL, bool kCodes>
 static cudaError_t launch_rq(const uint16_t* src, int64_t rows, int K, const float* s, int8_t* q, float* scale,
                              float* recip, cudaStream_t st, const DeviceInfo& dev) {
   const size_t smem = static_cast<size_t>(K / 8) * sizeof(float4) * (kMul ? 2 : 4);
-  auto kern = row_quant_kernel<kMul, WPR, VPL, kCodes>;
+  // rows that fill the warps' vectors exactly take the kernel without bounds checks
+  auto kern = (K == 256 * VPL * WPR) ? row_quant_kernel<kMul, WPR, VPL, kCodes, true>
+                                     : row_quant_kernel<kMul, WPR, VPL, kCodes, false>;
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
