@@ -405,7 +405,7 @@ constexpr int kRowThreads = 256;
 #define SQ_RQ_L2_AHEAD 1
 #endif
 #ifndef SQ_RQ_EARLY_L2  // build-time tuning knob: rows per row group prefetched into L2 before the wait
-#define SQ_RQ_EARLY_L2 4
+#define SQ_RQ_EARLY_L2 2
 #endif
 
 // kExact: the row fills the WPR warps' VPL vectors exactly (K == 256 VPL WPR),
@@ -464,28 +464,51 @@ __global__ void __launch_bounds__(kRowThreads) row_quant_kernel(const uint16_t* 
   griddep_wait();
   SQ_BLOCK_MARK(1);
   griddep_launch_dependents();
+  // The table, kTabChunk vectors per thread at a time: all of a chunk's loads
+  // of s are issued before any of them is used (one memory round trip per
+  // chunk instead of one per vector), and the first chunk's before the loads
+  // of the first row, so that s does not queue behind a row per block (and
+  // the rows prefetched above) in the memory system.
   uint4 xv[VPL];
-  load_row_vectors<VPL, WPR, kExact>(xv, src, row, rows, K, nvec, wsub, lane);  // in flight during the table build
-
+  bool row_issued = false;
   const float4* s4 = reinterpret_cast<const float4*>(s);
-  for (int v = tid; v < nvec; v += kRowThreads) {
-    const float4 a = __ldg(s4 + 2 * v), b = __ldg(s4 + 2 * v + 1);
-    if (kMul) {
-      sA[v] = a;
-      sB[v] = b;
-    } else {
-      sA[v] = make_float4(-a.x, -a.y, -a.z, -a.w);
-      sB[v] = make_float4(-b.x, -b.y, -b.z, -b.w);
-      const float4 ra = make_float4(__frcp_rn(a.x), __frcp_rn(a.y), __frcp_rn(a.z), __frcp_rn(a.w));
-      const float4 rb = make_float4(__frcp_rn(b.x), __frcp_rn(b.y), __frcp_rn(b.z), __frcp_rn(b.w));
-      rA[v] = ra;
-      rB[v] = rb;
-      if (!kCodes && recip != nullptr && blockIdx.x == 0) {
-        reinterpret_cast<float4*>(recip)[2 * v] = ra;
-        reinterpret_cast<float4*>(recip)[2 * v + 1] = rb;
+  constexpr int kTabChunk = 4;
+  for (int v0 = tid; v0 < nvec; v0 += kTabChunk * kRowThreads) {
+    float4 a[kTabChunk], b[kTabChunk];
+#pragma unroll
+    for (int j = 0; j < kTabChunk; ++j) {
+      const int v = v0 + j * kRowThreads;
+      if (v < nvec) {
+        a[j] = __ldg(s4 + 2 * v);
+        b[j] = __ldg(s4 + 2 * v + 1);
+      }
+    }
+    if (!row_issued) {  // the first row, in flight during the table build
+      load_row_vectors<VPL, WPR, kExact>(xv, src, row, rows, K, nvec, wsub, lane);
+      row_issued = true;
+    }
+#pragma unroll
+    for (int j = 0; j < kTabChunk; ++j) {
+      const int v = v0 + j * kRowThreads;
+      if (v >= nvec) break;
+      if (kMul) {
+        sA[v] = a[j];
+        sB[v] = b[j];
+      } else {
+        sA[v] = make_float4(-a[j].x, -a[j].y, -a[j].z, -a[j].w);
+        sB[v] = make_float4(-b[j].x, -b[j].y, -b[j].z, -b[j].w);
+        const float4 ra = make_float4(__frcp_rn(a[j].x), __frcp_rn(a[j].y), __frcp_rn(a[j].z), __frcp_rn(a[j].w));
+        const float4 rb = make_float4(__frcp_rn(b[j].x), __frcp_rn(b[j].y), __frcp_rn(b[j].z), __frcp_rn(b[j].w));
+        rA[v] = ra;
+        rB[v] = rb;
+        if (!kCodes && recip != nullptr && blockIdx.x == 0) {
+          reinterpret_cast<float4*>(recip)[2 * v] = ra;
+          reinterpret_cast<float4*>(recip)[2 * v + 1] = rb;
+        }
       }
     }
   }
+  if (!row_issued) load_row_vectors<VPL, WPR, kExact>(xv, src, row, rows, K, nvec, wsub, lane);
   __syncthreads();
   SQ_BLOCK_MARK(3);
   const float r127 = __frcp_rn(kQmax);  // RN(1/127), for the correctly rounded max / 127
