@@ -555,7 +555,7 @@ cudaError_t run_small(const SmallArgs& a, cudaStream_t st, const DeviceInfo& dev
   const int smem_cap = static_cast<int>(dev.max_smem_optin) - 1024;
   const int part_bytes = kSmallRows * NT * 4;
   const int stage_bytes = kSmallABytes + (kFused ? 0 : NT * kBK);
-  const int fixed = part_bytes + 128 + 10 * NT * 4 + 2 * kSmallRows * 4 + 256 + 16;
+  const int fixed = part_bytes + 128 + 18 * NT * 4 + 2 * kSmallRows * 4 + 256 + 16;
   // split K over a cluster of S CTAs: as many splits as keep one wave of CTAs
   // (S <= 8, at least two k-blocks each), more if the fused codes would not fit
   int S = 1;
@@ -587,7 +587,7 @@ cudaError_t run_small(const SmallArgs& a, cudaStream_t st, const DeviceInfo& dev
   p.part_off = p.b_off + b_bytes;
   p.xs_off = p.part_off + part_bytes;
   p.red_off = p.xs_off + 128;
-  p.wsb_off = p.red_off + 10 * NT * 4;
+  p.wsb_off = p.red_off + 18 * NT * 4;
   p.bar_off = p.wsb_off + 2 * kSmallRows * 4;
   p.misc_off = p.bar_off + 256;
   const int alloc = p.misc_off + 16 + 1024;

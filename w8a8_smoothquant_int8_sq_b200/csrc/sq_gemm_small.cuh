@@ -28,8 +28,11 @@
 //     this CTA's K-slice of X / s (correctly rounded fp32 division, as
 //     sq_quantize_act), holding their X vectors in registers between the two
 //     passes.  The per-token maxima over the whole row are assembled from the
-//     S ranks' slice maxima through distributed shared memory at a mid-kernel
-//     cluster barrier; the codes then go straight into the shared-memory B
+//     S ranks' slice maxima: every rank stores its maxima into every rank's
+//     shared memory with st.async, which counts the bytes on the receiver's
+//     own mbarrier (no cluster barrier, no cluster-scope release: under the
+//     weight stream a cluster barrier here took ~5 us, the asynchronous
+//     stores ~0.4 us); the codes then go straight into the shared-memory B
 //     operand in the 128-byte-swizzled K-major layout the tensor core reads.
 //     The MMAs cannot start before the codes exist, and past that point the
 //     kernel runs at the weight-stream rate, so the fused path is only about
@@ -47,6 +50,12 @@ namespace {
 // scales are known, 3 once the codes are written).
 #ifndef SQ_SMALL_GATE
 #define SQ_SMALL_GATE 0
+#endif
+// Build-time knob: 1 = the fused kernel's ranks exchange their slice maxima by
+// asynchronous remote stores that complete bytes on the receiver's own
+// mbarrier (st.async), 0 = plain remote loads after a cluster barrier.
+#ifndef SQ_SMALL_XCHG_ASYNC
+#define SQ_SMALL_XCHG_ASYNC 1
 #endif
 
 constexpr int kSmallThreads = 320;
@@ -83,6 +92,14 @@ __device__ __forceinline__ void cluster_arrive_relaxed() {
   asm volatile("barrier.cluster.arrive.relaxed;" ::: "memory");
 }
 __device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire;" ::: "memory"); }
+// 4-byte store into a cluster peer's shared memory whose completion is
+// counted (in bytes) on the peer's mbarrier at remote_bar; no fence, no
+// release: the receiver sees the value once that barrier's phase completes.
+__device__ __forceinline__ void st_async_f32(uint32_t remote_addr, float v, uint32_t remote_bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(remote_addr),
+               "r"(__float_as_uint(v)), "r"(remote_bar)
+               : "memory");
+}
 __device__ __forceinline__ uint32_t map_cluster_rank(uint32_t smem_addr, uint32_t rank) {
   uint32_t d;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(d) : "r"(smem_addr), "r"(rank));
@@ -241,6 +258,7 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
   float* red = reinterpret_cast<float*>(smem + p.red_off);  // [8 warps][NT], then the slice maxima [NT]
   float* cmax = red + 8 * NT;
   float* rxs_s = red + 9 * NT;  // fused: RN(1 / x_scale) per token
+  float* recv = red + 10 * NT;  // fused: [rank][NT] slice maxima received from every rank
   float* wsb = reinterpret_cast<float*>(smem + p.wsb_off);  // w_scale[256], bias[256] of this row block
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + p.bar_off);
   uint64_t* full = bars;
@@ -249,6 +267,7 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
   uint64_t* acc_full = b_ready + 1;
   uint64_t* drain = b_ready + 2;
   uint64_t* x_in = b_ready + 3;  // fused: every quantisation warp holds its slice of X
+  uint64_t* xchg = b_ready + 4;  // fused: the slice maxima of every rank have landed in recv
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + p.misc_off);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + p.misc_off + 4);
 
@@ -275,10 +294,18 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
     mbar_init(acc_full, 1);
     mbar_init(drain, 1);
     mbar_init(x_in, kSmallQuantThreads / 32);
+    if (kFused && SQ_SMALL_XCHG_ASYNC) {
+      mbar_init(xchg, 1);
+      mbar_arrive_expect_tx(xchg, static_cast<uint32_t>(S * NT * 4));
+    }
     *abort_flag = 0;
     fence_mbar_init();
     fence_proxy_async_smem();
   }
+  // fused, asynchronous exchange: a cluster phase that says every rank's
+  // exchange barrier is initialised; arrived now, waited for just before the
+  // first remote store (warps 0 and 1 wait for it at the end)
+  if (kFused && SQ_SMALL_XCHG_ASYNC) cluster_arrive_relaxed();
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmW);
     if (!kFused) tma_prefetch_desc(&tmX);
@@ -297,7 +324,7 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
   if (threadIdx.x == 0) SQ_TRACE_MARK(0);
   // fused: warps 0 and 1 take no part in the mid-kernel exchange of row maxima;
   // they arrive now and complete that phase at the end
-  if (kFused && warp < 2) cluster_arrive_relaxed();
+  if (kFused && !SQ_SMALL_XCHG_ASYNC && warp < 2) cluster_arrive_relaxed();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -457,10 +484,29 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
         cmax[qt] = mx;
       }
       if (warp == 2 && lane == 0) SQ_TRACE_MARK(8);
-      // exchange of the slice maxima across the cluster (warps 0, 1 arrived early)
-      asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+      // exchange of the slice maxima across the cluster
+      if (SQ_SMALL_XCHG_ASYNC) {
+        cluster_wait();  // every rank's exchange barrier is initialised
+        if (qt < NT) {
+          const uint32_t slot = smem_u32(recv + static_cast<int>(rank) * NT + qt);
+          const uint32_t bar = smem_u32(xchg);
+          for (int r = 0; r < S; ++r)
+            st_async_f32(map_cluster_rank(slot, static_cast<uint32_t>(r)), cmax[qt],
+                         map_cluster_rank(bar, static_cast<uint32_t>(r)));
+        }
+        if (!mbar_wait_bounded(xchg, 0, kWaitTimeoutNs) && lane == 0) flag_timeout(abort_flag);
+      } else {  // warps 0, 1 arrived early
+        asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+      }
       if (warp == 2 && lane == 0) SQ_TRACE_MARK(9);
-      if (qt < NT) {
+      if (SQ_SMALL_XCHG_ASYNC && qt < NT) {
+        float mx = 0.0f;
+        for (int r = 0; r < S; ++r) mx = fmaxf(mx, recv[r * NT + qt]);
+        const float sc = __fdiv_rn(fmaxf(mx, kClampFloor), kQmax);
+        xs_s[qt] = sc;
+        rxs_s[qt] = __frcp_rn(sc);
+      }
+      if (!SQ_SMALL_XCHG_ASYNC && qt < NT) {
         // all S remote loads are issued before the first use of any of them
         const uint32_t a = smem_u32(cmax + qt);
         float part_max[8];
