@@ -131,7 +131,8 @@ def default_path(workload_name):
 
 def metric_for(path):
     if path == "ste-train":
-        return "learnable-alpha W8A8 training step (forward + straight-through backward) tokens/s at 1 B200"
+        return ("learnable-alpha W8A8 training step (forward + relative-MSE auxiliary loss + straight-through "
+                "backward) tokens/s at 1 B200")
     return METRIC
 
 
@@ -150,7 +151,9 @@ def workload_config(wl, path="smoothquant"):
                          "bf16), " + c["workload"])
     elif path == "ste-train":
         c["workload"] = ("learnable-alpha training step (s from the running max of the calibration batch, "
-                         "forward, straight-through backward of a seeded bf16 dL/dY), " + c["workload"])
+                         "forward, relative-MSE auxiliary loss against the unquantised output with weight "
+                         f"{AUX_WEIGHT:g} folded into a seeded bf16 dL/dY, straight-through backward), "
+                         + c["workload"])
     elif path in FORWARD_CALLS:
         what = ("sq_forward: activation quantisation + int8 GEMM + epilogue" if path == "forward" else
                 "sq_forward_prologue: scale pre-pass + int8 GEMM that quantises X in its prologue + epilogue")
@@ -196,6 +199,8 @@ def algorithmic_work(wl):
         # G, X, W, Xq, Wq and the scales in; dX, dW (fp32), db, ds out; two
         # contractions of 2MNK each (counted once, whatever the kernel's split)
         "sq_ste_backward": (2 * M * N + 7 * M * K + 7 * N * K + 8 * M + 12 * N + 12 * K, 4 * M * N * K),
+        # two passes: Y_fp and Y_q for the sums, then Y_fp, Y_q and G in, G out
+        "sq_rel_mse": (12 * M * N + 8, 0),
         # X (bf16) and the codes in, Y out; 2MNK multiply-add operations on the fp32 CUDA cores
         "sq_linear_weight_only": (2 * M * K + N * K + 4 * N + 2 * M * N, 2 * M * N * K),
     }
@@ -349,6 +354,7 @@ def oracle_inputs(wl, path, inp=None):
     inp = dict(workloads.make_inputs(wl) if inp is None else inp)
     if path == "ste-train":
         inp["G"] = train_gradient(wl)
+        inp["Yfp"] = unquantised_output(wl, inp)
     if path in FORWARD_CALLS:
         # the weight is prepared once, outside the timed calls (as on the GPU)
         from oracle import smoothquant as O
@@ -376,8 +382,11 @@ def oracle_step_seconds(inp, wl, path="smoothquant"):
         mx = O.column_max_abs(O.widen_bf16(inp["C"]))
         s, _ = O.calibrate(inp["C"][:0], inp["W"], wl.alpha_f32, mx_prev=mx)
         Wq, ws = O.fold_and_quantize_weight(inp["W"], s)
-        O.forward(inp["X"], s, Wq, ws, inp["bias"])
-        STE.ste_backward(inp["G"], inp["X"], inp["W"], mx, wl.alpha_f32)
+        Yq = O.forward(inp["X"], s, Wq, ws, inp["bias"])[0]
+        from oracle import aux_loss as AUX
+        AUX.rel_mse(inp["Yfp"], Yq)
+        Gt = AUX.add_aux_grad(inp["G"], inp["Yfp"], Yq, AUX_WEIGHT)
+        STE.ste_backward(Gt, inp["X"], inp["W"], mx, wl.alpha_f32)
         return pc() - t0
     if path == "weight-only":
         from oracle import weight_only as WO
@@ -422,7 +431,7 @@ def oracle_sample_text(wl, path):
     mx_rows, mw_rows = sample_plan(wl, path)
     what = {"per-tensor": "quantise W and X per tensor, product",
             "weight-only": "quantise W per output channel, bf16 x int8 product",
-            "ste-train": "s from the running max, fold+quantise W, forward, straight-through backward",
+            "ste-train": "s from the running max, fold+quantise W, forward, auxiliary loss, straight-through backward",
             "forward": "forward on the prepared weight: quantise X, int8 product, epilogue",
             "forward-prologue": "forward on the prepared weight: quantise X, int8 product, epilogue",
             "smoothquant": "calibrate, fold+quantise W, quantise X, int8 product, epilogue"}[path]
@@ -451,6 +460,17 @@ def cpu_threads():
 def train_gradient(wl):
     """Seeded synthetic dL/dY [M, N] (bf16 bits) for the training step."""
     return workloads.random_bf16((wl.M, wl.N), seed=1000 * wl.index + 9, scale=1e-3)
+
+
+# weight of the relative-MSE auxiliary loss in the training step's total loss
+AUX_WEIGHT = 1.0
+
+
+def unquantised_output(wl, inp):
+    """Y_fp = X W^T + b of the unquantised layer (bf16 bits, one rounding from
+    float64): the reference output the auxiliary loss compares with."""
+    from oracle import smoothquant as O
+    return O.bf16_round(O.reference_linear_f64(inp["X"], inp["W"], inp["bias"]))
 
 
 def cpu_oracle_rate(wl, seconds, path="smoothquant", inp=None):
@@ -604,8 +624,15 @@ def run_ours(args, wl, rank, world, local_rank):
     elif args.path == "ste-train":
         # the training step of the learnable-alpha layer: s recomputed from the
         # running activation max (taken once from the calibration batch) and
-        # the weight, the forward, and the straight-through backward
+        # the weight, the forward, the relative-MSE auxiliary loss against the
+        # unquantised output folded into dL/dY, and the straight-through
+        # backward.  Y_fp (the unquantised layer, an input of the step like G)
+        # is formed once by the set-up.
         T["G"] = d(train_gradient(wl))
+        T["Yfp"] = d(unquantised_output(wl, inp))
+        T["Gt"] = torch.empty_like(T["G"])
+        T["aux_loss"] = torch.empty(1, dtype=torch.float64, device=dev)
+        T["ws_aux"] = torch.empty(sq.sq_rel_mse_workspace_bytes(), dtype=torch.uint8, device=dev)
         T["mx"] = torch.zeros(K, dtype=torch.float32, device=dev)
         sq.sq_calibrate(T["C"], T["W"], a, s=T["s"], mx_inout=T["mx"], workspace=T["ws_cal"])
         T.update(dXg=torch.empty(M, K, dtype=torch.float32, device=dev),
@@ -616,7 +643,7 @@ def run_ours(args, wl, rank, world, local_rank):
                  ws_bwd=torch.empty(sq.sq_ste_backward_workspace_bytes(M, N, K), dtype=torch.uint8, device=dev))
 
         def bwd(T):
-            sq.sq_ste_backward(T["G"], T["X"], T["W"], T["s"], T["mx"], a, T["Xq"], T["x_scale"], T["Wq"],
+            sq.sq_ste_backward(T["Gt"], T["X"], T["W"], T["s"], T["mx"], a, T["Xq"], T["x_scale"], T["Wq"],
                                T["w_scale"], with_db=T["b"] is not None, dX=T["dXg"], dW=T["dWg"], db=T["dbg"],
                                ds=T["dsg"], d_eta=T["d_eta"], workspace=T["ws_bwd"])
         calls = {
@@ -628,9 +655,12 @@ def run_ours(args, wl, rank, world, local_rank):
                                     ["X"], 1),
             "sq_linear": Call(lambda T: sq.sq_linear(T["Xq"], T["x_scale"], T["Wq"], T["w_scale"], T["b"], Y=T["Y"],
                                                      workspace=T["ws_lin"]), ["Xq", "Wq", "x_scale", "w_scale"], 1),
-            "sq_ste_backward": Call(bwd, ["G", "X", "W", "Xq", "Wq"], 7),
+            "sq_rel_mse": Call(lambda T: sq.sq_rel_mse(T["Yfp"], T["Y"], AUX_WEIGHT, G_in=T["G"], G_out=T["Gt"],
+                                                       loss=T["aux_loss"], workspace=T["ws_aux"]),
+                               ["Yfp", "Y", "G"], 2),
+            "sq_ste_backward": Call(bwd, ["Gt", "X", "W", "Xq", "Wq"], 7),
         }
-        stages = [["sq_calibrate(mx)"], ["sq_prepare_weight", "sq_quantize_act"], ["sq_linear"],
+        stages = [["sq_calibrate(mx)"], ["sq_prepare_weight", "sq_quantize_act"], ["sq_linear"], ["sq_rel_mse"],
                   ["sq_ste_backward"]]
     elif args.path == "per-tensor":
         T["ws_pt"] = torch.empty(sq.sq_quantize_per_tensor_workspace_bytes(), dtype=torch.uint8, device=dev)
@@ -846,8 +876,9 @@ def run_ours(args, wl, rank, world, local_rank):
         hC = pinned(inp["C"]) if args.path == "smoothquant" else None
         hb = pinned(inp["bias"]) if (T["b"] is not None and not forward_path) else None
         hG = pinned(train_gradient(wl)) if args.path == "ste-train" else None
+        hYfp = pinned(unquantised_output(wl, inp)) if args.path == "ste-train" else None
         hmx = T["mx"].cpu().pin_memory() if args.path == "ste-train" else None
-        host_in = {"X": hX, "W": hW, "C": hC, "b": hb, "G": hG, "mx": hmx}
+        host_in = {"X": hX, "W": hW, "C": hC, "b": hb, "G": hG, "Yfp": hYfp, "mx": hmx}
         host_in = {k: v for k, v in host_in.items() if v is not None}
         bufs, h_out = [], []
         for _ in range(2):
@@ -857,6 +888,8 @@ def run_ours(args, wl, rank, world, local_rank):
             D["Y"] = torch.empty_like(T["Y"])
             if args.path == "ste-train":
                 D["d_eta"] = torch.empty_like(T["d_eta"])
+                D["Gt"] = torch.empty_like(T["Gt"])
+                D["aux_loss"] = torch.empty_like(T["aux_loss"])
             bufs.append(D)
             h_out.append({"Y": torch.empty(M, N, dtype=torch.bfloat16).pin_memory(),
                           "d_eta": torch.empty(1, dtype=torch.float32).pin_memory()})
@@ -877,7 +910,9 @@ def run_ours(args, wl, rank, world, local_rank):
                 sq.sq_prepare_weight(D["W"], D["s"], Wq=D["Wq"], w_scale=D["w_scale"])
                 sq.sq_quantize_act(D["X"], D["s"], Xq=D["Xq"], x_scale=D["x_scale"])
                 sq.sq_linear(D["Xq"], D["x_scale"], D["Wq"], D["w_scale"], D["b"], Y=D["Y"], workspace=D["ws_lin"])
-                sq.sq_ste_backward(D["G"], D["X"], D["W"], D["s"], D["mx"], a, D["Xq"], D["x_scale"], D["Wq"],
+                sq.sq_rel_mse(D["Yfp"], D["Y"], AUX_WEIGHT, G_in=D["G"], G_out=D["Gt"], loss=D["aux_loss"],
+                              workspace=D["ws_aux"])
+                sq.sq_ste_backward(D["Gt"], D["X"], D["W"], D["s"], D["mx"], a, D["Xq"], D["x_scale"], D["Wq"],
                                    D["w_scale"], with_db=D["b"] is not None, dX=D["dXg"], dW=D["dWg"], db=D["dbg"],
                                    ds=D["dsg"], d_eta=D["d_eta"], workspace=D["ws_bwd"])
             elif args.path == "per-tensor":
@@ -933,7 +968,7 @@ def run_ours(args, wl, rank, world, local_rank):
         # the copies of the last step agree with the device result
         assert torch.equal(h_out[(2 + args.e2e_steps) % 2]["Y"].view(torch.int16),
                            bufs[(2 + args.e2e_steps) % 2]["Y"].cpu().view(torch.int16))
-        call = {"ste-train": "sq_calibrate(mx) + sq_prepare_weight + sq_quantize_act + sq_linear + "
+        call = {"ste-train": "sq_calibrate(mx) + sq_prepare_weight + sq_quantize_act + sq_linear + sq_rel_mse + "
                              "sq_ste_backward, Y and d eta read back",
                 "weight-only": "sq_prepare_weight (s = 1) + sq_linear_weight_only",
                 "per-tensor": "sq_quantize_per_tensor(W) + sq_quantize_per_tensor(X) + sq_linear",

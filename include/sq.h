@@ -274,6 +274,31 @@ SQ_API sq_status sq_linear(const int8_t* Xq, const float* x_scale, const int8_t*
                     int64_t M, int64_t N, int64_t K, sq_bf16* Y,
                     void* workspace, size_t workspace_bytes, void* stream);
 
+/* ------------------------------------------------ auxiliary loss (learnable alpha)
+ * sq_rel_mse -- the relative-MSE auxiliary loss that trains alpha, and its
+ * gradient folded into the gradient of the quantised output.  Page: module
+ * docstring of "w8a8_smoothquant.py" (V5): ||Y_fp - Y_q||_F^2 / ||Y_fp||_F^2
+ * added to the total loss so that its gradient reaches eta_alpha;
+ * SmoothQuantW8A8.quantization_error (the unsquared ratio, norm floored at
+ * 1e-12).
+ *
+ *   Y_fp[M][N], Y_q[M][N] bf16 (the unquantised and the W8A8 layer outputs)
+ *   loss_out   one double (device): sum (Y_fp - Y_q)^2 / max(sum Y_fp^2, 1e-24),
+ *              accumulated in float64
+ *   G_in, G_out  [M][N] bf16 or both NULL; when given,
+ *              G_out = bf16(G_in + lambda * 2 (Y_q - Y_fp) / max(sum Y_fp^2, 1e-24)),
+ *              evaluated in float64 and rounded once (nearest, ties to even):
+ *              the G of sq_ste_backward for a total loss L + lambda * aux.
+ *              G_in == G_out is allowed (in place).  Y_fp carries no gradient
+ *              (it does not depend on alpha).
+ *   workspace  at least sq_rel_mse_workspace_bytes() bytes, 16-byte aligned.
+ * Pointers 16-byte aligned (loss_out 8-byte); lambda finite.  Two kernels.
+ */
+SQ_API size_t sq_rel_mse_workspace_bytes(void);
+SQ_API sq_status sq_rel_mse(const sq_bf16* Y_fp, const sq_bf16* Y_q, int64_t M, int64_t N, double lambda,
+                     const sq_bf16* G_in, sq_bf16* G_out, double* loss_out,
+                     void* workspace, size_t workspace_bytes, void* stream);
+
 /* --------------------------------------------------------- fused forward
  * sq_forward -- the per-batch path: sq_quantize_act followed by sq_linear,
  * Y from bf16 X.  Page: forward of SmoothQuantW8A8 once frozen.

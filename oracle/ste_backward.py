@@ -47,8 +47,8 @@ Readings:
 * The dequantised operands are the exact products q * scale (the page
   rounds them to fp32; the difference is below 2^-24 relative).
 * Everything after the codes and scales is evaluated in float64.
-* The auxiliary relative-MSE loss of the page is composed by the caller: its
-  gradient with respect to Y enters through G.
+* The auxiliary relative-MSE loss of the page enters through G: its gradient
+  with respect to Y_q is folded into G by ``oracle.aux_loss.add_aux_grad``.
 """
 from __future__ import annotations
 

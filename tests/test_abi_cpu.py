@@ -70,6 +70,15 @@ def test_validation_before_device(sq):
     assert lib.sq_linear(a, a, a, a, None, 4, 8, 200000, a, None, 0, None) == 2
     assert lib.sq_forward(a, a, a, a, None, 4, 8, 64, a, a, 16, None) == 8
     assert lib.sq_forward_prologue(a, a, a, a, None, 4, 8, 64, a, a, 16, None) == 8      # workspace too small
+    wsb = sq.sq_rel_mse_workspace_bytes()
+    assert wsb >= 2 * 8 * 148 * 8
+    d = ctypes.c_double
+    assert lib.sq_rel_mse(a, a, 4, 8, d(0.5), a, None, a, a, wsb, None) == 4           # G_in without G_out
+    assert lib.sq_rel_mse(a, a, 4, 8, d(0.5), None, None, None, a, wsb, None) == 1     # no loss_out
+    assert lib.sq_rel_mse(a, mis, 4, 8, d(0.5), None, None, a, a, wsb, None) == 3      # Y_q misaligned
+    assert lib.sq_rel_mse(a, a, 4, 8, d(0.5), None, None, a, a, 16, None) == 8         # workspace too small
+    assert lib.sq_rel_mse(a, a, 0, 8, d(0.5), None, None, a, a, wsb, None) == 2        # M = 0
+    assert lib.sq_rel_mse(a, a, 4, 8, d(float("nan")), None, None, a, a, wsb, None) == 4
     assert lib.sq_forward_prologue(a, mis, a, a, None, 4, 8, 64, a, a, 512, None) == 3   # s misaligned
     assert lib.sq_forward_prologue(a, a, a, a, None, 4, 8, 16400, a, a, 1 << 20, None) == 2  # K above 16384
     assert lib.sq_gemm_s32(a, a, 4, 0, 64, a, None) == 2

@@ -24,7 +24,7 @@ __all__ = [
     "sq_version", "sq_calibrate", "sq_calibrate_workspace_bytes", "sq_calibrate_noalloc", "sq_prepare_weight",
     "sq_quantize_act", "sq_quantize_per_tensor", "sq_quantize_per_tensor_workspace_bytes", "sq_linear_weight_only", "sq_ste_backward",
     "sq_ste_backward_workspace_bytes", "sq_linear", "sq_workspace_bytes", "sq_forward",
-    "sq_forward_workspace_bytes", "sq_forward_prologue", "sq_forward_prologue_workspace_bytes", "sq_gemm_s32", "sq_device_status", "sq_debug_fail_after",
+    "sq_forward_workspace_bytes", "sq_forward_prologue", "sq_rel_mse", "sq_rel_mse_workspace_bytes", "sq_forward_prologue_workspace_bytes", "sq_gemm_s32", "sq_device_status", "sq_debug_fail_after",
     "sq_debug_pipeline_stall",
     "STATUS",
 ]
@@ -55,6 +55,8 @@ _SIGNATURES = [
     ("sq_quantize_per_tensor", ctypes.c_int, (_P, _I64, _I64, _P, _P, _P, _SZ, _P)),
     ("sq_linear_weight_only", ctypes.c_int, (_P, _I64, _P, _P, _P, _I64, _I64, _P, _P)),
     ("sq_ste_backward_workspace_bytes", _SZ, (_I64, _I64, _I64)),
+    ("sq_rel_mse_workspace_bytes", _SZ, ()),
+    ("sq_rel_mse", ctypes.c_int, (_P, _P, _I64, _I64, ctypes.c_double, _P, _P, _P, _P, _SZ, _P)),
     ("sq_ste_backward", ctypes.c_int, (_P, _P, _P, _P, _P, ctypes.c_float, _P, _P, _P, _P, _I64, _I64, _I64,
                                        _P, _P, _P, _P, _P, _P, _SZ, _P)),
     ("sq_workspace_bytes", _SZ, (_I64, _I64, _I64)),
@@ -371,6 +373,36 @@ def sq_forward(X: torch.Tensor, s: torch.Tensor, Wq: torch.Tensor, w_scale: torc
     _check(_load().sq_forward(_ptr(X), _ptr(s), _ptr(Wq), _ptr(w_scale), _ptr(bias), M, N, K, _ptr(Y), _ptr(ws),
                           ws.numel(), _stream(stream)))
     return Y
+
+
+def sq_rel_mse_workspace_bytes() -> int:
+    return int(_load().sq_rel_mse_workspace_bytes())
+
+
+def sq_rel_mse(Y_fp: torch.Tensor, Y_q: torch.Tensor, lam: float = 0.0, G_in: Optional[torch.Tensor] = None,
+               G_out: Optional[torch.Tensor] = None, loss: Optional[torch.Tensor] = None,
+               workspace: Optional[torch.Tensor] = None, stream=None):
+    """The relative-MSE auxiliary loss ||Y_fp - Y_q||^2 / ||Y_fp||^2 (a
+    float64 tensor of one element, on the device) and, given G_in (bf16
+    [M, N]), G_out = bf16(G_in + lam * d aux / d Y_q).  Returns (loss, G_out);
+    G_out is None without G_in.  G_out may be G_in (in place)."""
+    _want(Y_fp, "Y_fp", torch.bfloat16, 2)
+    _want(Y_q, "Y_q", torch.bfloat16, 2)
+    M, N = Y_fp.shape
+    if tuple(Y_q.shape) != (M, N):
+        raise ValueError("Y_fp and Y_q must have the same shape")
+    if G_in is not None:
+        _want(G_in, "G_in", torch.bfloat16, 2)
+        if tuple(G_in.shape) != (M, N):
+            raise ValueError("G_in must be [M, N]")
+        G_out = _out(G_out, (M, N), torch.bfloat16, Y_fp.device, "G_out")
+    elif G_out is not None:
+        raise ValueError("G_out without G_in")
+    loss = _out(loss, (1,), torch.float64, Y_fp.device, "loss")
+    ws = _workspace(workspace, sq_rel_mse_workspace_bytes(), Y_fp.device)
+    _check(_load().sq_rel_mse(_ptr(Y_fp), _ptr(Y_q), M, N, float(lam), _ptr(G_in), _ptr(G_out), _ptr(loss),
+                          _ptr(ws), ws.numel(), _stream(stream)))
+    return loss, G_out
 
 
 def sq_forward_prologue_workspace_bytes(M: int, K: int) -> int:

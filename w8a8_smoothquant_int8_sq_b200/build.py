@@ -17,7 +17,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libsq.so")
-SOURCES = ["sq_api.cu", "sq_quant.cu", "sq_gemm.cu", "sq_weight_only.cu", "sq_ste.cu"]
+SOURCES = ["sq_api.cu", "sq_quant.cu", "sq_gemm.cu", "sq_weight_only.cu", "sq_ste.cu", "sq_aux.cu"]
 HEADERS = ["sq_device.cuh", "sq_internal.h", "sq_gemm_small.cuh", "sq_gemm_splitk.cuh", "sq_gemm_pair.cuh", "sq_gemm_prologue.cuh", os.path.join("..", "..", "include", "sq.h")]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -376,6 +376,33 @@ sq_status sq_linear(const int8_t* Xq, const float* x_scale, const int8_t* Wq, co
                      workspace, workspace == nullptr ? 0 : workspace_bytes);
 }
 
+// ------------------------------------------------ auxiliary loss (learnable alpha)
+size_t sq_rel_mse_workspace_bytes(void) { return round_up(sq::rel_mse_workspace_bytes(), 256); }
+
+sq_status sq_rel_mse(const sq_bf16* Y_fp, const sq_bf16* Y_q, int64_t M, int64_t N, double lambda,
+                     const sq_bf16* G_in, sq_bf16* G_out, double* loss_out, void* workspace, size_t workspace_bytes,
+                     void* stream) {
+  SQ_TRY(check_rows(M, "M"));
+  SQ_TRY(check_rows(N, "N"));
+  SQ_NONNULL(Y_fp);
+  SQ_NONNULL(Y_q);
+  if (loss_out == nullptr) return fail(SQ_ERR_NULL, "loss_out is NULL");
+  if ((reinterpret_cast<uintptr_t>(loss_out) & 7u) != 0) return fail(SQ_ERR_ALIGN, "loss_out is not 8-byte aligned");
+  if ((G_in == nullptr) != (G_out == nullptr)) return fail(SQ_ERR_ARG, "G_in and G_out must both be given or both be NULL");
+  if (G_in != nullptr && (!aligned16(G_in) || !aligned16(G_out)))
+    return fail(SQ_ERR_ALIGN, "G_in / G_out are not 16-byte aligned");
+  if (!std::isfinite(lambda)) return fail(SQ_ERR_ARG, "lambda is not finite");
+  if (workspace == nullptr || workspace_bytes < sq_rel_mse_workspace_bytes())
+    return fail(SQ_ERR_WORKSPACE, "workspace must hold sq_rel_mse_workspace_bytes() = " +
+                                      std::to_string(sq_rel_mse_workspace_bytes()) + " bytes");
+  if (!aligned16(workspace)) return fail(SQ_ERR_ALIGN, "workspace is not 16-byte aligned");
+  sq::DeviceInfo dev;
+  SQ_TRY(prologue(&dev));
+  return cuda_status(sq::launch_rel_mse(Y_fp, Y_q, M * N, lambda, G_in, G_out, loss_out, workspace,
+                                        static_cast<cudaStream_t>(stream), dev),
+                     "relative-MSE loss launch");
+}
+
 // ----------------------------------------------------------- fused forward
 static size_t forward_xq_bytes(int64_t M, int64_t K) { return round_up(static_cast<size_t>(M * K), 256); }
 

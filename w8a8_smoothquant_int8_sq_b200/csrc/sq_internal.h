@@ -190,6 +190,15 @@ void debug_pipeline_stall(bool enable, unsigned long long timeout_ns);
 // Device status word (bit 0: pipeline wait timeout).
 cudaError_t read_device_status(uint32_t* flags, bool clear);
 
+// ---- relative-MSE auxiliary loss (sq_aux.cu)
+// loss = sum (Y_fp - Y_q)^2 / max(sum Y_fp^2, 1e-24) over n elements (float64);
+// with g_out != null also g_out = bf16(g_in + lambda * 2 (Y_q - Y_fp) / den)
+// (g_in and g_out may be the same array).  ws: rel_mse_workspace_bytes(),
+// 16-byte aligned.
+size_t rel_mse_workspace_bytes();
+cudaError_t launch_rel_mse(const uint16_t* yfp, const uint16_t* yq, int64_t n, double lambda, const uint16_t* g_in,
+                           uint16_t* g_out, double* loss, void* ws, cudaStream_t st, const DeviceInfo& dev);
+
 // ---- straight-through backward of the learnable-alpha layer (sq_ste.cu)
 struct SteArgs {
   const uint16_t* G;      // [M][N] bf16, dL/dY
