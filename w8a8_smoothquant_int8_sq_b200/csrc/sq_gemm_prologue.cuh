@@ -120,7 +120,7 @@ struct PrologueParams {
 // per CTA rank: converter warp 0 lane 0 at 0 stage free, 1 first slot landed,
 // 2 first slot converted, 3 second slot landed, 4 second slot converted,
 // 5 codes published; 6 the MMA's full wait done (even CTA); 7 the Wq producer's
-// empty wait done; 8 past the proxy fence; 9 converter warp 7 at 5.  X producer issue times
+// empty wait done; 8 past the proxy fence; 9 the last converter warp at 5.  X producer issue times
 // per slot in g_pro_xtrace.
 __device__ unsigned long long g_pro_trace[2][64][10];
 __device__ unsigned long long g_pro_xtrace[2][128];
@@ -436,9 +436,9 @@ __global__ void __launch_bounds__(kFThreads, 1)
     uint32_t phase = 0, xphase = 0;
     bool ok = true;
     int cseq = 0;  // stages converted (trace index)
-    const bool tr0 = cw == 0 && lane == 0, tr7 = cw == kFConvWarps - 1 && lane == 0;
+    const bool tr0 = cw == 0 && lane == 0, trl = cw == kFConvWarps - 1 && lane == 0;
     (void)tr0;
-    (void)tr7;
+    (void)trl;
     for (int tile = pair; ok && tile < num_tiles; tile += num_pairs) {
       int m_blk, n_blk;
       tile_coords(tile, p.num_m_blocks, p.num_n_blocks, p.group_m, m_blk, n_blk);
@@ -518,7 +518,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(rank == 0 ? &full[stage] : &cfull[stage]);
         if (tr0) SQ_PRO_MARK(cseq, 5);
-        if (tr7) SQ_PRO_MARK(cseq, 9);
+        if (trl) SQ_PRO_MARK(cseq, 9);
         ++cseq;
         if (++stage == kFStages) {
           stage = 0;
