@@ -224,6 +224,25 @@ struct SteGemmParams {
   unsigned int* mwbits;    // DW: [I] max |W| as fp32 bits
 };
 
+#ifdef SQ_TRACE
+// Optional per-tile timestamps (build with -DSQ_TRACE), CTAs 0..3, first 16
+// tiles of each: MMA thread at 0 accumulator free, 1 last MMA issued;
+// epilogue warp 0 (lane 0) at 2 block loads issued, 3 accumulator ready,
+// 4 first 32 columns done, 5 tile done.  [EPI][cta][tile][mark]
+__device__ unsigned long long g_ste_trace[2][4][16][6];
+#define SQ_STE_MARK(t, i)                                                                              \
+  do {                                                                                                 \
+    if (blockIdx.x < 4 && (t) < 16) g_ste_trace[EPI][blockIdx.x][(t)][(i)] = globaltimer_ns();         \
+  } while (0)
+extern "C" __attribute__((visibility("default"))) int sq_trace_read_ste(unsigned long long* host) {
+  return cudaMemcpyFromSymbol(host, g_ste_trace, sizeof(g_ste_trace)) == cudaSuccess ? 0 : 1;
+}
+#else
+#define SQ_STE_MARK(t, i) \
+  do {                    \
+  } while (0)
+#endif
+
 __device__ __forceinline__ void ste_flag_timeout(volatile int* abort_flag) {
   *abort_flag = 1;
   atomicOr(&g_sq_ste_status, 1u);
@@ -347,6 +366,7 @@ __global__ void __launch_bounds__(kSThreads, 1)
           if (!*abort_flag) ste_flag_timeout(abort_flag);
           break;
         }
+        SQ_STE_MARK(it, 0);
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kSAccCols);
         for (int kb = 0; kb < nk; ++kb) {
@@ -371,6 +391,7 @@ __global__ void __launch_bounds__(kSThreads, 1)
           }
         }
         if (!ok) break;
+        SQ_STE_MARK(it, 1);
         mma_commit(&tfull[acc]);
       }
       mma_commit(drain);
@@ -428,12 +449,14 @@ __global__ void __launch_bounds__(kSThreads, 1)
           }
         }
       }
+      if (ew == 0 && lane == 0) SQ_STE_MARK(it, 2);
       const bool mine = !*abort_flag && mbar_wait_bounded(&tfull[acc], acc_phase, kSWaitNs);
       if (!__all_sync(0xFFFFFFFFu, mine)) {
         if (lane == 0 && !*abort_flag) ste_flag_timeout(abort_flag);
         break;
       }
       tc_fence_after();
+      if (ew == 0 && lane == 0) SQ_STE_MARK(it, 3);
       const uint32_t t_base =
           tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * kSAccCols);
       float tsum = 0.0f;
@@ -481,9 +504,11 @@ __global__ void __launch_bounds__(kSThreads, 1)
             o += p.I;
           }
         }
+        if (cc == 0 && ew == 0 && lane == 0) SQ_STE_MARK(it, 4);
       }
       tc_fence_before();
       __syncwarp();
+      if (ew == 0 && lane == 0) SQ_STE_MARK(it, 5);
       if (lane == 0) mbar_arrive(&tempty[acc]);
       if (row_ok) {
         atomicAdd(p.tsum + i, tsum);
