@@ -81,6 +81,15 @@ constexpr unsigned long long kSWaitNs = 2000000000ull;
 constexpr int kEpiDX = 0;
 constexpr int kEpiDW = 1;
 
+// Warp-wide load of 8 consecutive 32-bit TMEM columns; lane i of the warp gets
+// TMEM lane (warp quarter * 32 + i).
+__device__ __forceinline__ void tmem_ld_8cols(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr)
+               : "memory");
+}
+
 __device__ __forceinline__ uint16_t bf16_bits_rn(float v) { return __bfloat16_as_ushort(__float2bfloat16_rn(v)); }
 
 // store the first min(4, n) of v0..v3 at dst (8-byte aligned when n >= 4)
@@ -406,6 +415,45 @@ __global__ void __launch_bounds__(kSThreads, 1)
     int8_t* stg_q = reinterpret_cast<int8_t*>(stg + 32 * kStgSrcPitch);  // [32 j][kStgQPitch bytes]
     float* stg_qs = reinterpret_cast<float*>(stg + 32 * (kStgSrcPitch + kStgQPitch));  // [32 j]
     constexpr int kChunks = kSBN / 32 / 2;  // 32-column chunks per warp and tile
+    // this warp's 32 x 64 block of src and q of a tile and its column scales:
+    // lane l holds row j_blk * 128 + 64 half + 32 cc + l, the warp's 32
+    // columns from i0 (those that exist; the rest stay zero).  A tile's blocks
+    // are fetched while the previous tile's last chunk is processed (the
+    // first tile's before its accumulator is ready), so the loads overlap the
+    // epilogue and the MMAs.
+    uint4 ra[kChunks][4], rb[kChunks][2];
+    float rq[kChunks];
+    auto load_blocks = [&](int t) {
+      const int ib = t % p.num_i_blocks;
+      const int jb = t / p.num_i_blocks;
+      const int r0 = ib * kSBM + quarter * 32;
+      // rows of this warp that exist: 0, 16 or 32 (I % 16 == 0, r0 % 32 == 0)
+      const int nr = max(0, min(32, p.I - r0));
+#pragma unroll
+      for (int cc = 0; cc < kChunks; ++cc) {
+        const int j = jb * kSBN + half * 64 + cc * 32 + lane;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) ra[cc][u] = make_uint4(0u, 0u, 0u, 0u);
+        rb[cc][0] = rb[cc][1] = make_uint4(0u, 0u, 0u, 0u);
+        rq[cc] = 0.0f;
+        if (j < p.J) {
+          rq[cc] = __ldg(p.qscale + j);
+          if (nr > 0) {
+            const int64_t e = static_cast<int64_t>(j) * p.I + r0;
+            const uint4* sv = reinterpret_cast<const uint4*>(p.src + e);
+            const uint4* qv = reinterpret_cast<const uint4*>(p.q + e);
+            ra[cc][0] = sv[0];
+            ra[cc][1] = sv[1];
+            rb[cc][0] = qv[0];
+            if (nr > 16) {
+              ra[cc][2] = sv[2];
+              ra[cc][3] = sv[3];
+              rb[cc][1] = qv[1];
+            }
+          }
+        }
+      }
+    };
     int it = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
       const int acc = it & 1;
@@ -415,40 +463,9 @@ __global__ void __launch_bounds__(kSThreads, 1)
       const int i0 = i_blk * kSBM + quarter * 32;  // this warp's first row
       const int i = i0 + lane;
       const bool row_ok = i < p.I;
-      // rows of this warp that exist: 0, 16 or 32 (I % 16 == 0, i0 % 32 == 0)
-      const int ni = max(0, min(32, p.I - i0));
       const float s_i = row_ok ? __ldg(p.s + i) : 1.0f;
       const float rs_i = __frcp_rn(s_i);
-      // this warp's 32 x 64 block of src and q and its column scales, fetched
-      // before the accumulator is ready so that the loads overlap the tile's
-      // MMAs: lane l holds row j_blk * 128 + 64 half + 32 cc + l, columns
-      // i0 .. i0 + ni - 1
-      uint4 ra[kChunks][4], rb[kChunks][2];
-      float rq[kChunks];
-#pragma unroll
-      for (int cc = 0; cc < kChunks; ++cc) {
-        const int j = j_blk * kSBN + half * 64 + cc * 32 + lane;
-#pragma unroll
-        for (int u = 0; u < 4; ++u) ra[cc][u] = make_uint4(0u, 0u, 0u, 0u);
-        rb[cc][0] = rb[cc][1] = make_uint4(0u, 0u, 0u, 0u);
-        rq[cc] = 0.0f;
-        if (j < p.J) {
-          rq[cc] = __ldg(p.qscale + j);
-          if (ni > 0) {
-            const int64_t e = static_cast<int64_t>(j) * p.I + i0;
-            const uint4* sv = reinterpret_cast<const uint4*>(p.src + e);
-            const uint4* qv = reinterpret_cast<const uint4*>(p.q + e);
-            ra[cc][0] = sv[0];
-            ra[cc][1] = sv[1];
-            rb[cc][0] = qv[0];
-            if (ni > 16) {
-              ra[cc][2] = sv[2];
-              ra[cc][3] = sv[3];
-              rb[cc][1] = qv[1];
-            }
-          }
-        }
-      }
+      if (it == 0) load_blocks(tile);
       if (ew == 0 && lane == 0) SQ_STE_MARK(it, 2);
       const bool mine = !*abort_flag && mbar_wait_bounded(&tfull[acc], acc_phase, kSWaitNs);
       if (!__all_sync(0xFFFFFFFFu, mine)) {
@@ -464,9 +481,6 @@ __global__ void __launch_bounds__(kSThreads, 1)
 #pragma unroll
       for (int cc = 0; cc < kChunks; ++cc) {
         const int c0 = half * 64 + cc * 32;
-        uint32_t r[32], rl[32];
-        tmem_ld_32cols(t_base + static_cast<uint32_t>(c0), r);           // A Bh^T
-        tmem_ld_32cols(t_base + static_cast<uint32_t>(kSBN + c0), rl);   // A Bl^T
         const int j0 = j_blk * kSBN + c0;
         const int jn = min(32, p.J - j0);
         __syncwarp();  // the previous chunk's reads of the staging area are done
@@ -479,29 +493,51 @@ __global__ void __launch_bounds__(kSThreads, 1)
           dq[1] = rb[cc][1];
           stg_qs[lane] = rq[cc];
         }
-        tmem_ld_wait();
+        // the blocks of this warp's next tile, in flight while this chunk and
+        // the tile hand-over run
+        if (cc == kChunks - 1 && tile + static_cast<int>(gridDim.x) < num_tiles)
+          load_blocks(tile + static_cast<int>(gridDim.x));
         __syncwarp();
-        if (j0 < p.J && row_ok) {
-          float* o = p.out + static_cast<int64_t>(j0) * p.I + i;
+        // Columns past J and rows past I hold zeros in every operand (TMA
+        // fills the boxes past the matrix with zeros, and the staged blocks
+        // start from zero), so they add nothing to the sums; only the stores
+        // are predicated, and the loop has no early exit.  Eight columns at a
+        // time: each group's TMEM loads end in a wait, which also bounds how
+        // far the compiler hoists the staging reads (register pressure).
+        const bool st_ok = row_ok && j0 < p.J;
+        float* op = p.out + (static_cast<int64_t>(j0) * p.I + i);  // advanced by a row per column
 #pragma unroll
-          for (int jj = 0; jj < 32; ++jj) {
-            if (jj >= jn) break;
-            const float v = __fadd_rn(__uint_as_float(r[jj]), __uint_as_float(rl[jj]));
-            const uint16_t xb = *reinterpret_cast<const uint16_t*>(reinterpret_cast<const uint8_t*>(stg_src) +
-                                                                  jj * kStgSrcPitch + lane * 2);
+        for (int g = 0; g < 4; ++g) {
+          uint32_t r[8], rl[8];
+          tmem_ld_8cols(t_base + static_cast<uint32_t>(c0 + 8 * g), r);          // A Bh^T
+          tmem_ld_8cols(t_base + static_cast<uint32_t>(kSBN + c0 + 8 * g), rl);  // A Bl^T
+          tmem_ld_wait();
+          // an opaque copy of the staging pointer: the group's staging reads
+          // cannot be hoisted above this point
+          const uint8_t* sg = stg;
+          asm volatile("" : "+l"(sg));
+          const float* sqs = reinterpret_cast<const float*>(sg + 32 * (kStgSrcPitch + kStgQPitch));
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const int jj = 8 * g + u;
+            const float v = __fadd_rn(__uint_as_float(r[u]), __uint_as_float(rl[u]));
+            const uint16_t xb = *reinterpret_cast<const uint16_t*>(sg + jj * kStgSrcPitch + lane * 2);
             const float x = __uint_as_float(static_cast<uint32_t>(xb) << 16);
-            const float dq = static_cast<float>(stg_q[jj * kStgQPitch + lane]);
+            const float dq = static_cast<float>(*reinterpret_cast<const int8_t*>(sg + 32 * kStgSrcPitch +
+                                                                                 jj * kStgQPitch + lane));
+            float o;
             if (EPI == kEpiDX) {
-              *o = __fmul_rn(v, rs_i);                                          // dXs / s
-              const float err = __fmaf_rn(-dq, stg_qs[jj], __fmul_rn(x, rs_i));  // X/s - Xdq
+              o = __fmul_rn(v, rs_i);                                           // dXs / s
+              const float err = __fmaf_rn(-dq, sqs[jj], __fmul_rn(x, rs_i));  // X/s - Xdq
               tsum = __fmaf_rn(v, err, tsum);
             } else {
-              *o = __fmul_rn(v, s_i);                                           // dWs * s
-              const float err = __fmaf_rn(-dq, stg_qs[jj], __fmul_rn(x, s_i));   // W*s - Wdq
+              o = __fmul_rn(v, s_i);                                            // dWs * s
+              const float err = __fmaf_rn(-dq, sqs[jj], __fmul_rn(x, s_i));   // W*s - Wdq
               tsum = __fmaf_rn(v, err, tsum);
               mbits = max(mbits, static_cast<uint32_t>(xb & 0x7FFFu) << 16);
             }
-            o += p.I;
+            if (st_ok && jj < jn) *op = o;
+            op += p.I;
           }
         }
         if (cc == 0 && ew == 0 && lane == 0) SQ_STE_MARK(it, 4);
