@@ -100,6 +100,13 @@ __device__ __forceinline__ void st_async_f32(uint32_t remote_addr, float v, uint
                "r"(__float_as_uint(v)), "r"(remote_bar)
                : "memory");
 }
+// The same for 16 bytes (16-byte aligned destination).
+__device__ __forceinline__ void st_async_v4(uint32_t remote_addr, uint4 v, uint32_t remote_bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
+                   remote_addr),
+               "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w), "r"(remote_bar)
+               : "memory");
+}
 __device__ __forceinline__ uint32_t map_cluster_rank(uint32_t smem_addr, uint32_t rank) {
   uint32_t d;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(d) : "r"(smem_addr), "r"(rank));
@@ -268,6 +275,7 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
   uint64_t* drain = b_ready + 2;
   uint64_t* x_in = b_ready + 3;  // fused: every quantisation warp holds its slice of X
   uint64_t* xchg = b_ready + 4;  // fused: the slice maxima of every rank have landed in recv
+  uint64_t* red_bar = b_ready + 5;  // every rank's partial sums of the rows this rank reduces have landed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + p.misc_off);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + p.misc_off + 4);
 
@@ -298,14 +306,20 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
       mbar_init(xchg, 1);
       mbar_arrive_expect_tx(xchg, static_cast<uint32_t>(S * NT * 4));
     }
+    // the partial sums arrive by st.async: S senders x (256 / S) rows x the
+    // token quads that hold real tokens x 16 bytes
+    mbar_init(red_bar, 1);
+    mbar_arrive_expect_tx(red_bar, static_cast<uint32_t>(kSmallRows * ((p.M + 3) / 4) * 16));
     *abort_flag = 0;
     fence_mbar_init();
     fence_proxy_async_smem();
   }
-  // fused, asynchronous exchange: a cluster phase that says every rank's
-  // exchange barrier is initialised; arrived now, waited for just before the
-  // first remote store (warps 0 and 1 wait for it at the end)
-  if (kFused && SQ_SMALL_XCHG_ASYNC) cluster_arrive_relaxed();
+  // A cluster phase that says every rank's barriers are initialised: arrived
+  // now, waited for just before a thread's first remote store (the fused
+  // kernel's exchange, or the partial sums), or at the end by the warps that
+  // store nothing remotely.  (The fused kernel with the exchange by cluster
+  // barrier has its quantisation warps take that barrier instead.)
+  if (!kFused || SQ_SMALL_XCHG_ASYNC) cluster_arrive_relaxed();
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmW);
     if (!kFused) tma_prefetch_desc(&tmX);
@@ -578,6 +592,7 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
     // ------------------------------------------------- accumulators to shared memory (warps 2..5)
     if (warp < 6) {
       const int quarter = warp & 3;
+      if (!kFused) cluster_wait();  // every rank's red_bar is initialised
       bool have = my_nkb > 0;
       if (have) {
         const bool mine = !*abort_flag && mbar_wait_bounded(acc_full, 0, kWaitTimeoutNs);
@@ -605,32 +620,38 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
           }
         }
         // push the row's partial sums to the rank that reduces this row, into
-        // that rank's slot for this sender (fire-and-forget stores; the
-        // cluster barrier below waits for them)
+        // that rank's slot for this sender, by st.async: the bytes count on
+        // the owner's red_bar, which the owner waits for (no cluster barrier)
         const int rpr = kSmallRows / S;
         const int owner = n_local / rpr;
         const uint32_t dst = map_cluster_rank(
             smem_u32(part + (static_cast<int>(rank) * rpr + (n_local - owner * rpr)) * NT), static_cast<uint32_t>(owner));
+        const uint32_t dst_bar = map_cluster_rank(smem_u32(red_bar), static_cast<uint32_t>(owner));
         const int nq = (p.M + 3) / 4;  // token quads that hold real tokens
 #pragma unroll
         for (int i = 0; i < NT / 4; ++i)
-          if (i < nq) st_cluster_v4(dst + 16u * i, make_uint4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]));
+          if (i < nq)
+            st_async_v4(dst + 16u * i, make_uint4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]), dst_bar);
       }
     }
   }
 
   // ------------------------------------------- split-K reduction over the cluster
-  // Rank q reduces rows [q*256/S, (q+1)*256/S): every rank has pushed its
-  // partial sums of those rows into rank q's shared memory (one slot per
-  // sender), so after the cluster barrier the S partials of a row are local
-  // loads; the sum is dequantised and stored.  Token quads past M are skipped.
-  // No CTA reads another's shared memory after the barrier, so none has to
-  // wait for the others before leaving.
+  // Rank q reduces rows [q*256/S, (q+1)*256/S): every rank pushes its partial
+  // sums of those rows into rank q's shared memory (one slot per sender) with
+  // st.async, counted on rank q's red_bar; once its phase completes the S
+  // partials of a row are local loads; the sum is dequantised and stored.
+  // Token quads past M are skipped.  A rank leaves only after every byte
+  // addressed to it has landed, and no rank reads another's shared memory,
+  // so no cluster barrier is needed at the end.
   tc_fence_before();
-  __syncthreads();
-  if (kFused && warp < 2) cluster_wait();  // completes the phase these warps arrived at early
-  cluster_sync_all();  // every rank's pushes have landed
-  if (threadIdx.x == 0) SQ_TRACE_MARK(5);
+  __syncthreads();  // w_scale, bias and the token scales staged above
+  // completes the start phase for the warps that stored nothing remotely
+  if (kFused ? warp < 2 : (warp < 2 || warp >= 6)) cluster_wait();
+  if (warp >= 2) {
+    if (!mbar_wait_bounded(red_bar, 0, kWaitTimeoutNs) && lane == 0) flag_timeout(abort_flag);
+  }
+  if (threadIdx.x == 64) SQ_TRACE_MARK(5);
   if (warp >= 2) {
     const int rpr = kSmallRows / S;
     const int r_lo = static_cast<int>(rank) * rpr;
