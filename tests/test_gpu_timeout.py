@@ -130,3 +130,41 @@ def test_fused_prologue_wait_timeout_is_reported_and_the_context_survives(sq):
     torch.cuda.synchronize()
     assert torch.equal(Y.view(torch.int16), Y_l.view(torch.int16))
     assert sq.sq_device_status() == 0
+
+
+def test_few_token_wait_timeout_is_reported_and_the_context_survives(sq):
+    """The same failure in the few-token GEMM (decode shape: K split over a
+    cluster of 8, partial sums pushed to the reducing rank by st.async and
+    counted on its mbarrier): every producer skips its first stage, so the MMA
+    waits give up; every rank still sends its (zero) partial sums, so no rank
+    waits for another.  Both the quantising forward and the product on
+    prequantised codes are stalled, then run again and checked."""
+    rng = np.random.default_rng(95)
+    M, N, K = 8, 2048, 8192  # 8 row blocks x 8 K ranks, 8 k-blocks each: more than the ring holds
+    X = torch.randn(M, K, device="cuda").to(torch.bfloat16)
+    s = (torch.rand(K, device="cuda") + 0.5).float()
+    Wq_h = rng.integers(-127, 128, (N, K), dtype=np.int64).astype(np.int8)
+    ws_h = (rng.random(N, dtype=np.float32) * 1e-3 + 1e-4).astype(np.float32)
+    Wq, ws = dev(Wq_h), dev(ws_h)
+    Xq, xs = sq.sq_quantize_act(X, s)
+    torch.cuda.synchronize()
+    assert sq.sq_device_status(clear=True) == 0
+    for run in (lambda: sq.sq_forward(X, s, Wq, ws), lambda: sq.sq_linear(Xq, xs, Wq, ws)):
+        try:
+            sq.sq_debug_pipeline_stall(True, 50_000_000)
+            t0 = time.perf_counter()
+            run()
+            torch.cuda.synchronize()
+            elapsed = time.perf_counter() - t0
+        finally:
+            sq.sq_debug_pipeline_stall(False)
+        flags = sq.sq_device_status(clear=True)
+        assert flags & 1, "the stalled few-token pipeline was not reported"
+        assert elapsed < 5.0
+    Y_f = sq.sq_forward(X, s, Wq, ws)
+    Y_l = sq.sq_linear(Xq, xs, Wq, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(Y_f.view(torch.int16), Y_l.view(torch.int16)), "fused forward != quantise + product"
+    assert_y_close(host_bf16_bits(Y_l), O.int8_gemm(host(Xq), Wq_h), host(xs), ws_h, None,
+                   "few-token GEMM after a timeout")
+    assert sq.sq_device_status() == 0

@@ -582,6 +582,8 @@ cudaError_t run_small(const SmallArgs& a, cudaStream_t st, const DeviceInfo& dev
   p.x_scale = a.x_scale;
   p.w_scale = a.w_scale;
   p.bias = a.bias;
+  p.timeout_ns = g_debug_stall.load() ? g_debug_timeout_ns.load() : kWaitTimeoutNs;
+  p.skip_first_load = g_debug_stall.load() ? 1 : 0;
   p.Y = a.Y;
   p.b_off = stages * stage_bytes;
   p.part_off = p.b_off + b_bytes;

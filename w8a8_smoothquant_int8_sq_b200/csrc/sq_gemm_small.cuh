@@ -78,6 +78,8 @@ struct SmallParams {
   uint16_t* Y;           // [M][N]
   // shared-memory layout (bytes from the 1024-aligned base)
   int b_off, part_off, xs_off, red_off, wsb_off, bar_off, misc_off;
+  unsigned long long timeout_ns;  // limit of every mbarrier wait
+  int skip_first_load;            // test hook: the producer never loads its first stage
 };
 
 __device__ __forceinline__ uint32_t cluster_rank() {
@@ -351,30 +353,33 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
       // returned; issued behind a full ring of weight boxes they would wait for
       // the whole ring to drain from HBM, and the MMAs wait for their codes
       if (kFused && SQ_SMALL_GATE > 0 &&
-          (*abort_flag || !mbar_wait_bounded(SQ_SMALL_GATE == 3 ? b_ready : x_in, 0, kWaitTimeoutNs))) {
+          (*abort_flag || !mbar_wait_bounded(SQ_SMALL_GATE == 3 ? b_ready : x_in, 0, p.timeout_ns))) {
         if (!*abort_flag) flag_timeout(abort_flag);
         ok = false;
       }
       for (int kb = kb0; ok && kb < kb1; ++kb) {
-        if (*abort_flag || !mbar_wait_bounded(&empty[stage], phase ^ 1u, kWaitTimeoutNs)) {
+        if (*abort_flag || !mbar_wait_bounded(&empty[stage], phase ^ 1u, p.timeout_ns)) {
           if (!*abort_flag) flag_timeout(abort_flag);
           ok = false;
           break;
         }
         uint8_t* dst = smem + stage * p.stage_bytes;
-        mbar_arrive_expect_tx(&full[stage], static_cast<uint32_t>(p.stage_bytes));
-        tma_load_2d(dst, &tmW, kb * kBK, rb * kSmallRows, &full[stage]);
-        if (!kFused) tma_load_2d(dst + kSmallABytes, &tmX, kb * kBK, 0, &full[stage]);
+        if (!(p.skip_first_load && kb == kb0)) {  // test hook: the first stage never fills
+          mbar_arrive_expect_tx(&full[stage], static_cast<uint32_t>(p.stage_bytes));
+          tma_load_2d(dst, &tmW, kb * kBK, rb * kSmallRows, &full[stage]);
+          if (!kFused) tma_load_2d(dst + kSmallABytes, &tmX, kb * kBK, 0, &full[stage]);
+        }
         ++issued;
         if (++stage == stages) {
           stage = 0;
           phase ^= 1u;
         }
       }
-      if (!ok) {  // drain the copies in flight (the last min(issued, stages) loads)
+      if (!ok) {  // drain the copies in flight (the last min(issued, stages) loads; a skipped one never completes)
         for (int i = 0; i < min(issued, stages); ++i) {
           const int q = issued - 1 - i;
-          (void)mbar_wait_bounded(&full[q % stages], static_cast<uint32_t>((q / stages) & 1), kWaitTimeoutNs);
+          if (p.skip_first_load && q == 0) continue;
+          (void)mbar_wait_bounded(&full[q % stages], static_cast<uint32_t>((q / stages) & 1), p.timeout_ns);
         }
       }
     }
@@ -384,14 +389,14 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
       constexpr uint32_t idesc = idesc_i8(kBM, NT);
       bool ok = true;
       if (kFused) {
-        ok = !*abort_flag && mbar_wait_bounded(b_ready, 0, kWaitTimeoutNs);
+        ok = !*abort_flag && mbar_wait_bounded(b_ready, 0, p.timeout_ns);
         if (!ok && !*abort_flag) flag_timeout(abort_flag);
       }
       SQ_TRACE_MARK(1);
       int stage = 0;
       uint32_t phase = 0;
       for (int j = 0; ok && j < my_nkb; ++j) {
-        if (*abort_flag || !mbar_wait_bounded(&full[stage], phase, kWaitTimeoutNs)) {
+        if (*abort_flag || !mbar_wait_bounded(&full[stage], phase, p.timeout_ns)) {
           if (!*abort_flag) flag_timeout(abort_flag);
           ok = false;
           break;
@@ -418,7 +423,7 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
       SQ_TRACE_MARK(3);
       if (ok) mma_commit(acc_full);
       mma_commit(drain);
-      (void)mbar_wait_bounded(drain, 0, kWaitTimeoutNs);
+      (void)mbar_wait_bounded(drain, 0, p.timeout_ns);
     }
   } else {
     // ------------------------------------------------- quantisation (warps 2..9)
@@ -508,7 +513,7 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
             st_async_f32(map_cluster_rank(slot, static_cast<uint32_t>(r)), cmax[qt],
                          map_cluster_rank(bar, static_cast<uint32_t>(r)));
         }
-        if (!mbar_wait_bounded(xchg, 0, kWaitTimeoutNs) && lane == 0) flag_timeout(abort_flag);
+        if (!mbar_wait_bounded(xchg, 0, p.timeout_ns) && lane == 0) flag_timeout(abort_flag);
       } else {  // warps 0, 1 arrived early
         asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
       }
@@ -595,7 +600,7 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
       if (!kFused) cluster_wait();  // every rank's red_bar is initialised
       bool have = my_nkb > 0;
       if (have) {
-        const bool mine = !*abort_flag && mbar_wait_bounded(acc_full, 0, kWaitTimeoutNs);
+        const bool mine = !*abort_flag && mbar_wait_bounded(acc_full, 0, p.timeout_ns);
         have = __all_sync(0xFFFFFFFFu, mine);
         if (!have && lane == 0 && !*abort_flag) flag_timeout(abort_flag);
       }
@@ -649,7 +654,7 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
   // completes the start phase for the warps that stored nothing remotely
   if (kFused ? warp < 2 : (warp < 2 || warp >= 6)) cluster_wait();
   if (warp >= 2) {
-    if (!mbar_wait_bounded(red_bar, 0, kWaitTimeoutNs) && lane == 0) flag_timeout(abort_flag);
+    if (!mbar_wait_bounded(red_bar, 0, p.timeout_ns) && lane == 0) flag_timeout(abort_flag);
   }
   if (threadIdx.x == 64) SQ_TRACE_MARK(5);
   if (warp >= 2) {
