@@ -168,3 +168,34 @@ def test_few_token_wait_timeout_is_reported_and_the_context_survives(sq):
     assert_y_close(host_bf16_bits(Y_l), O.int8_gemm(host(Xq), Wq_h), host(xs), ws_h, None,
                    "few-token GEMM after a timeout")
     assert sq.sq_device_status() == 0
+
+
+def test_backward_wait_timeout_is_reported_and_the_context_survives(sq):
+    """The same failure in the straight-through backward's two tcgen05 GEMMs
+    (dX and dW): their producers skip the first stage, the waits give up, the
+    kernels report and return; then the whole backward runs again and matches
+    its oracle within the derived bounds."""
+    from tests.helpers import dev_bf16
+    from tests.test_gpu_ste import _inputs, _run
+    from oracle import ste_backward as STE
+    G, X, W, mx = _inputs(64, 264, 640, seed=7)
+    alpha = float(STE.alpha_from_logit(0.5))
+    Wd, Xd = dev_bf16(W), dev_bf16(X)
+    mx_d = dev(np.asarray(mx, np.float32).copy())
+    s = sq.sq_calibrate(None, Wd, alpha, mx_inout=mx_d)
+    Wq, ws = sq.sq_prepare_weight(Wd, s)
+    Xq, xs = sq.sq_quantize_act(Xd, s)
+    torch.cuda.synchronize()
+    assert sq.sq_device_status(clear=True) == 0
+    try:
+        sq.sq_debug_pipeline_stall(True, 50_000_000)
+        t0 = time.perf_counter()
+        sq.sq_ste_backward(dev_bf16(G), Xd, Wd, s, mx_d, alpha, Xq, xs, Wq, ws)
+        torch.cuda.synchronize()
+        elapsed = time.perf_counter() - t0
+    finally:
+        sq.sq_debug_pipeline_stall(False)
+    flags = sq.sq_device_status(clear=True)
+    assert flags & 1, "the stalled backward was not reported"
+    assert elapsed < 5.0
+    _run(sq, G, X, W, mx, 0.5, "backward after a timeout")

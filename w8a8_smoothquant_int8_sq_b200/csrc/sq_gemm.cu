@@ -873,6 +873,12 @@ void debug_pipeline_stall(bool enable, unsigned long long timeout_ns) {
   g_debug_stall.store(enable ? 1 : 0);
 }
 
+bool debug_stall_state(unsigned long long* timeout_ns) {
+  const bool on = g_debug_stall.load() != 0;
+  *timeout_ns = on ? g_debug_timeout_ns.load() : kWaitTimeoutNs;
+  return on;
+}
+
 cudaError_t read_device_status(uint32_t* flags, bool clear) {
   cudaError_t e = cudaDeviceSynchronize();
   if (e != cudaSuccess) return e;

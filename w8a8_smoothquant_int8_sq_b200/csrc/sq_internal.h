@@ -183,9 +183,12 @@ struct PrologueArgs {
 };
 cudaError_t launch_forward_prologue(const PrologueArgs& a, cudaStream_t st, const DeviceInfo& dev, const char** why);
 
-// Test hook: while enabled, the general GEMM's producer skips its first stage
-// and every wait gives up after timeout_ns (the kernel then reports bit 0).
+// Test hook: while enabled, the GEMMs' producers skip their first stage and
+// every wait gives up after timeout_ns (the kernel then reports bit 0).
 void debug_pipeline_stall(bool enable, unsigned long long timeout_ns);
+// Whether that hook is on; *timeout_ns receives the wait limit to use (the
+// hook's while it is on, the normal one otherwise).
+bool debug_stall_state(unsigned long long* timeout_ns);
 
 // Device status word (bit 0: pipeline wait timeout).
 cudaError_t read_device_status(uint32_t* flags, bool clear);

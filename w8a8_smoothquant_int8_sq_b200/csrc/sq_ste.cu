@@ -77,7 +77,6 @@ constexpr int kSMiscOffset = kSStgOffset + kSEpiWarps * kStgBytes;
 constexpr int kSAlloc = kSMiscOffset + 16 + 1024;
 constexpr int kSAccCols = 2 * kSBN;         // one accumulator: A Bh^T in columns [0, 128), A Bl^T in [128, 256)
 constexpr uint32_t kSTmemCols = 2 * kSAccCols;
-constexpr unsigned long long kSWaitNs = 2000000000ull;
 constexpr int kEpiDX = 0;
 constexpr int kEpiDW = 1;
 
@@ -231,6 +230,8 @@ struct SteGemmParams {
   float* out;              // dX or dW: element (j, i) at out[j * I + i]
   float* tsum;             // [I] sum over j of dXs * dX_q (or dWs * dW_q)
   unsigned int* mwbits;    // DW: [I] max |W| as fp32 bits
+  unsigned long long timeout_ns;  // limit of every mbarrier wait
+  int skip_first_load;            // test hook: the producer never loads its first stage
 };
 
 #ifdef SQ_TRACE
@@ -336,19 +337,21 @@ __global__ void __launch_bounds__(kSThreads, 1)
         tma_prefetch_l2_2d(&tmSrc, i_blk * kSBM, j_blk * kSBN);
         tma_prefetch_l2_2d(&tmQ, i_blk * kSBM, j_blk * kSBN);
         for (int kb = 0; kb < nk; ++kb) {
-          if (*abort_flag || !mbar_wait_bounded(&empty[stage], phase ^ 1u, kSWaitNs)) {
+          if (*abort_flag || !mbar_wait_bounded(&empty[stage], phase ^ 1u, p.timeout_ns)) {
             if (!*abort_flag) ste_flag_timeout(abort_flag);
             ok = false;
             break;
           }
           uint8_t* sa = smem + stage * kSStageBytes;
           uint8_t* sb = sa + kSABytes;
-          mbar_arrive_expect_tx(&full[stage], kSStageBytes);
-          tma_load_2d(sa, &tmA, kb * kSBK, i_blk * kSBM, &full[stage]);
-          tma_load_2d(sb, &tmBh, kb * kSBK, j_blk * kSBN, &full[stage]);
-          tma_load_2d(sb + kSBBytes, &tmBl, kb * kSBK, j_blk * kSBN, &full[stage]);
-          issued[stage] = 1;
-          issued_phase[stage] = phase;
+          if (!(p.skip_first_load && tile == static_cast<int>(blockIdx.x) && kb == 0)) {
+            mbar_arrive_expect_tx(&full[stage], kSStageBytes);
+            tma_load_2d(sa, &tmA, kb * kSBK, i_blk * kSBM, &full[stage]);
+            tma_load_2d(sb, &tmBh, kb * kSBK, j_blk * kSBN, &full[stage]);
+            tma_load_2d(sb + kSBBytes, &tmBl, kb * kSBK, j_blk * kSBN, &full[stage]);
+            issued[stage] = 1;  // (test hook: a skipped stage is not waited for)
+            issued_phase[stage] = phase;
+          }
           if (++stage == kSStages) {
             stage = 0;
             phase ^= 1u;
@@ -358,7 +361,7 @@ __global__ void __launch_bounds__(kSThreads, 1)
       if (!ok) {
 #pragma unroll
         for (int i = 0; i < kSStages; ++i)
-          if (issued[i]) (void)mbar_wait_bounded(&full[i], issued_phase[i], kSWaitNs);
+          if (issued[i]) (void)mbar_wait_bounded(&full[i], issued_phase[i], p.timeout_ns);
       }
     }
   } else if (warp == 1) {
@@ -371,7 +374,7 @@ __global__ void __launch_bounds__(kSThreads, 1)
       for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x, ++it) {
         const int acc = it & 1;
         const uint32_t acc_phase = (it >> 1) & 1;
-        if (*abort_flag || !mbar_wait_bounded(&tempty[acc], acc_phase ^ 1u, kSWaitNs)) {
+        if (*abort_flag || !mbar_wait_bounded(&tempty[acc], acc_phase ^ 1u, p.timeout_ns)) {
           if (!*abort_flag) ste_flag_timeout(abort_flag);
           break;
         }
@@ -379,7 +382,7 @@ __global__ void __launch_bounds__(kSThreads, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kSAccCols);
         for (int kb = 0; kb < nk; ++kb) {
-          if (*abort_flag || !mbar_wait_bounded(&full[stage], phase, kSWaitNs)) {
+          if (*abort_flag || !mbar_wait_bounded(&full[stage], phase, p.timeout_ns)) {
             if (!*abort_flag) ste_flag_timeout(abort_flag);
             ok = false;
             break;
@@ -404,7 +407,7 @@ __global__ void __launch_bounds__(kSThreads, 1)
         mma_commit(&tfull[acc]);
       }
       mma_commit(drain);
-      (void)mbar_wait_bounded(drain, 0, kSWaitNs);
+      (void)mbar_wait_bounded(drain, 0, p.timeout_ns);
     }
   } else {
     const int quarter = warp & 3;          // TMEM lanes 32 quarter .. + 31
@@ -467,7 +470,7 @@ __global__ void __launch_bounds__(kSThreads, 1)
       const float rs_i = __frcp_rn(s_i);
       if (it == 0) load_blocks(tile);
       if (ew == 0 && lane == 0) SQ_STE_MARK(it, 2);
-      const bool mine = !*abort_flag && mbar_wait_bounded(&tfull[acc], acc_phase, kSWaitNs);
+      const bool mine = !*abort_flag && mbar_wait_bounded(&tfull[acc], acc_phase, p.timeout_ns);
       if (!__all_sync(0xFFFFFFFFu, mine)) {
         if (lane == 0 && !*abort_flag) ste_flag_timeout(abort_flag);
         break;
@@ -652,6 +655,7 @@ cudaError_t run_ste_gemm(const void* A, const void* Bh, const void* Bl, int64_t 
     return cudaErrorInvalidValue;
   }
   SteGemmParams p = base;
+  p.skip_first_load = debug_stall_state(&p.timeout_ns) ? 1 : 0;
   p.I = static_cast<int>(I);
   p.J = static_cast<int>(J);
   p.C = static_cast<int>(C);
