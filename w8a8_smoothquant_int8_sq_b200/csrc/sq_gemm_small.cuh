@@ -48,6 +48,12 @@ namespace {
 // Build-time knob: when the fused kernel's producer starts streaming the
 // weight (0 at once, 1 once the activation loads have returned, 2 once the row
 // scales are known, 3 once the codes are written).
+// Build-time knob: weight boxes (k-blocks) per CTA prefetched into L2 before
+// the wait for the previous kernel (in a stream of calls, the CTAs that start
+// while the previous call's last CTAs finish get their first stages early).
+#ifndef SQ_SMALL_EARLY_L2
+#define SQ_SMALL_EARLY_L2 2
+#endif
 #ifndef SQ_SMALL_GATE
 #define SQ_SMALL_GATE 0
 #endif
@@ -325,6 +331,11 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmW);
     if (!kFused) tma_prefetch_desc(&tmX);
+    // the first weight boxes of this CTA into L2 while the previous kernel may
+    // still run (a hint only: writes land in L2, so the loads after the wait
+    // read current data)
+    for (int kb = kb0; kb < min(kb1, kb0 + SQ_SMALL_EARLY_L2); ++kb)
+      tma_prefetch_l2_2d(&tmW, kb * kBK, rb * kSmallRows);
   }
   if (warp == 1) {
     __syncwarp();
