@@ -658,7 +658,7 @@ def run_ours(args, wl, rank, world, local_rank):
             "sq_rel_mse": Call(lambda T: sq.sq_rel_mse(T["Yfp"], T["Y"], AUX_WEIGHT, G_in=T["G"], G_out=T["Gt"],
                                                        loss=T["aux_loss"], workspace=T["ws_aux"]),
                                ["Yfp", "Y", "G"], 2),
-            "sq_ste_backward": Call(bwd, ["Gt", "X", "W", "Xq", "Wq"], 7),
+            "sq_ste_backward": Call(bwd, ["Gt", "X", "W", "Xq", "Wq"], 6),
         }
         stages = [["sq_calibrate(mx)"], ["sq_prepare_weight", "sq_quantize_act"], ["sq_linear"], ["sq_rel_mse"],
                   ["sq_ste_backward"]]

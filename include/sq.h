@@ -240,7 +240,7 @@ SQ_API sq_status sq_linear_weight_only(const sq_bf16* X, int64_t M, const int8_t
  * 2^-16 + 2^-23 + 2C * 2^-22 of the sum of its absolute products (C the
  * contraction length).  ds is formed from the quantisation errors W*s - Wdq
  * and X/s - Xdq, so it carries that relative error without cancellation.
- * Launches 7 kernels; reads G once.
+ * Launches 6 kernels; reads G once.
  */
 SQ_API size_t sq_ste_backward_workspace_bytes(int64_t M, int64_t N, int64_t K);
 SQ_API sq_status sq_ste_backward(const sq_bf16* G, const sq_bf16* X, const sq_bf16* W, const float* s,

@@ -28,10 +28,11 @@
 // that cancels heavily.
 //
 // Kernels (all chained with programmatic dependent launch):
-//   ste_init_kernel         zero the per-channel sums and db
+//   transpose_codes_kernel  Wt[k][n] = Wq[n][k], Xt[k][m] = Xq[m][k] as bf16;
+//                           the first launch also zeroes the per-channel sums,
+//                           db and the finish counter
 //   split_g_kernel          Ghi/Glo[m][n] from G w_scale, Gthi/Gtlo[n][m] from
 //                           G x_scale (transposed), db[n] += sum_m G[m][n]
-//   transpose_codes_kernel  Wt[k][n] = Wq[n][k], Xt[k][m] = Xq[m][k] as bf16
 //   ste_gemm_kernel<DX>     dXs^T on the tensor cores (bf16 in, fp32 in TMEM);
 //                           epilogue writes dX and adds lane k's
 //                           sum_m dXs (X/s - Xdq)
@@ -103,32 +104,43 @@ __device__ __forceinline__ void store4(uint16_t* dst, int n, uint16_t v0, uint16
   }
 }
 
-__global__ void ste_init_kernel(float* tx, float* tw, unsigned int* mwbits, int K, float* db, int N,
-                                unsigned int* counter) {
-  griddep_wait();
-  griddep_launch_dependents();
-  if (blockIdx.x == 0 && threadIdx.x == 0) *counter = 0u;
-  const int stride = gridDim.x * blockDim.x;
-  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < K; i += stride) {
-    tx[i] = 0.0f;
-    tw[i] = 0.0f;
-    mwbits[i] = 0u;
-  }
-  if (db != nullptr)
-    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < N; i += stride) db[i] = 0.0f;
-}
+// Per-call sums that the later kernels accumulate into, zeroed by the first
+// transpose (before the split of G adds to db and the GEMMs to tx, tw, mw).
+struct SteZero {
+  float* tx;
+  float* tw;
+  unsigned int* mwbits;
+  int K;
+  float* db;  // may be null
+  int N;
+  unsigned int* counter;
+};
 
 // out[c][r] = in[r][c] as bf16 (exact for int8 codes) for r < R, c < C.  in:
 // int8, row pitch C (C % 4 == 0); out: row pitch ldo elements (ldo % 8 == 0).
 // Thread (ty, tx) of a 16 x 16 block loads 4 codes of rows ty + 16i and
-// stores 4 outputs of rows ty + 16i of the transposed tile.
+// stores 4 outputs of rows ty + 16i of the transposed tile.  With zero.tx not
+// null the grid also zeroes the words of `zero`.
 __global__ void __launch_bounds__(kTThreads) transpose_codes_kernel(const int8_t* in, int R, int C, uint16_t* out,
-                                                                     int ldo) {
+                                                                     int ldo, SteZero zero) {
   __shared__ uint16_t tile[kTT][kTT + 2];
   const int c0 = blockIdx.x * kTT, r0 = blockIdx.y * kTT;
   const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
   griddep_wait();
   griddep_launch_dependents();
+  if (zero.tx != nullptr) {
+    const int nb = gridDim.x * gridDim.y;
+    const int b = blockIdx.y * gridDim.x + blockIdx.x;
+    const int stride = nb * kTThreads;
+    for (int i = b * kTThreads + threadIdx.x; i < zero.K; i += stride) {
+      zero.tx[i] = 0.0f;
+      zero.tw[i] = 0.0f;
+      zero.mwbits[i] = 0u;
+    }
+    if (zero.db != nullptr)
+      for (int i = b * kTThreads + threadIdx.x; i < zero.N; i += stride) zero.db[i] = 0.0f;
+    if (b == 0 && threadIdx.x == 0) *zero.counter = 0u;
+  }
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int rl = ty + 16 * i, r = r0 + rl, c = c0 + 4 * tx;
@@ -567,7 +579,7 @@ __global__ void __launch_bounds__(kSThreads, 1)
 // sum_k ds_k raw_k (ln mx_k + ln mw_k) over the channels whose raw_k =
 // mx_k^alpha / mw_k^(1-alpha) (both clamped at 1e-8) is not below 1e-8.
 // float64; one channel per thread, block sums in `partial`, and the last
-// block to finish (arrival counter, zeroed by ste_init_kernel) adds the block
+// block to finish (arrival counter, zeroed by the first transpose) adds the block
 // sums in block order and writes d eta.
 constexpr int kFinishThreads = 256;
 __global__ void __launch_bounds__(kFinishThreads) ste_finish_kernel(const float* tx, const float* tw,
@@ -713,18 +725,19 @@ cudaError_t launch_ste_backward(const SteArgs& a, cudaStream_t st, const DeviceI
   const int M = static_cast<int>(a.M), N = static_cast<int>(a.N), K = static_cast<int>(a.K);
   const int Mp = static_cast<int>(L.Mp);
 
-  cudaError_t e = launch_pdl(ste_init_kernel, dim3(std::max(1, std::min(dev.sm_count, (std::max(K, N) + 255) / 256))),
-                             dim3(256), 0, st, tx, tw, mw, K, a.db, N, fin_counter);
-  if (e != cudaSuccess) return *why = "init launch", e;
+  // the codes transposed first: the first transpose also zeroes the sums that
+  // the split of G (db) and the GEMMs (tx, tw, mw) accumulate into
+  const SteZero zero{tx, tw, mw, K, a.db, N, fin_counter};
+  const SteZero no_zero{nullptr, nullptr, nullptr, 0, nullptr, 0, nullptr};
+  cudaError_t e = launch_pdl(transpose_codes_kernel, dim3((K + kTT - 1) / kTT, (N + kTT - 1) / kTT), dim3(kTThreads),
+                             0, st, a.Wq, N, K, Wt, N, zero);
+  if (e != cudaSuccess) return *why = "transpose of Wq", e;
+  e = launch_pdl(transpose_codes_kernel, dim3((K + kTT - 1) / kTT, (M + kTT - 1) / kTT), dim3(kTThreads), 0, st, a.Xq,
+                 M, K, Xt, Mp, no_zero);
+  if (e != cudaSuccess) return *why = "transpose of Xq", e;
   e = launch_pdl(split_g_kernel, dim3((N + kTT - 1) / kTT, (M + kTT - 1) / kTT), dim3(kTThreads), 0, st, a.G, M, N,
                  a.w_scale, a.x_scale, Gh, Gl, Gth, Gtl, Mp, a.db);
   if (e != cudaSuccess) return *why = "split of G", e;
-  e = launch_pdl(transpose_codes_kernel, dim3((K + kTT - 1) / kTT, (N + kTT - 1) / kTT), dim3(kTThreads), 0, st, a.Wq,
-                 N, K, Wt, N);
-  if (e != cudaSuccess) return *why = "transpose of Wq", e;
-  e = launch_pdl(transpose_codes_kernel, dim3((K + kTT - 1) / kTT, (M + kTT - 1) / kTT), dim3(kTThreads), 0, st, a.Xq,
-                 M, K, Xt, Mp);
-  if (e != cudaSuccess) return *why = "transpose of Xq", e;
 
   SteGemmParams p{};
   p.s = a.s;
