@@ -199,3 +199,32 @@ def test_backward_wait_timeout_is_reported_and_the_context_survives(sq):
     assert flags & 1, "the stalled backward was not reported"
     assert elapsed < 5.0
     _run(sq, G, X, W, mx, 0.5, "backward after a timeout")
+
+
+def test_weight_only_wait_timeout_is_reported_and_the_context_survives(sq):
+    """The same failure in the int8 weight-only comparison kernel (K split
+    over a cluster, partial sums pushed to rank 0): the first stage never
+    fills, the waits give up, every CTA lets the copies it issued land and
+    still meets its cluster at the reduction; the next call is exact."""
+    from tests.helpers import dev_bf16
+    from tests.test_gpu_weight_only import _check
+    import workloads
+    X = workloads.random_bf16((8, 4096), seed=12, scale=1.0)
+    W = workloads.random_bf16((1024, 4096), seed=13, scale=0.02)
+    Wq, ws = sq.sq_prepare_weight(dev_bf16(W), torch.ones(4096, dtype=torch.float32, device="cuda"))
+    Xd = dev_bf16(X)
+    torch.cuda.synchronize()
+    assert sq.sq_device_status(clear=True) == 0
+    try:
+        sq.sq_debug_pipeline_stall(True, 50_000_000)
+        t0 = time.perf_counter()
+        sq.sq_linear_weight_only(Xd, Wq, ws, None)
+        torch.cuda.synchronize()
+        elapsed = time.perf_counter() - t0
+    finally:
+        sq.sq_debug_pipeline_stall(False)
+    flags = sq.sq_device_status(clear=True)
+    assert flags & 1, "the stalled weight-only pipeline was not reported"
+    assert elapsed < 5.0
+    _check(sq, X, W, None, "weight-only after a timeout")
+    assert sq.sq_device_status() == 0

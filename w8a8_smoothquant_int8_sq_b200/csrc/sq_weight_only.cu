@@ -60,7 +60,6 @@ constexpr int kWoMaxRecvSplit = 4;                              // K splits whos
 constexpr int kWoRecvBytes = kWoMaxRecvSplit * kWoTok * kWoRows * 4;  // 16 KB
 constexpr int kWoBarOffset = kWoRecvOffset + kWoRecvBytes;
 constexpr int kWoSmemBytes = kWoBarOffset + kWoStages * 8 + 16 + 1024;
-constexpr unsigned long long kWoWaitNs = 2000000000ull;
 static_assert(kWoStageCols == kWoWarps * kWoStep, "one 16-column step per warp per stage");
 static_assert(kWoRedBytes <= kWoXBytes, "the warp sums reuse the X area");
 static_assert(kWoMaxSplit <= kWoMaxRecvSplit, "every split's partial has a slot");
@@ -74,6 +73,8 @@ struct WoParams {
   uint16_t* Y;           // [M][N] bf16
   int M, N, K;
   int kc;  // columns per K split (a multiple of kWoStageCols)
+  unsigned long long timeout_ns;  // limit of every mbarrier wait
+  int skip_first_load;            // test hook: the first stage is never loaded
 };
 
 __device__ unsigned int g_sq_wo_status = 0u;
@@ -140,9 +141,13 @@ __global__ void __launch_bounds__(kWoThreads, 1) weight_only_kernel(const __grid
   __syncthreads();
   griddep_wait();
   griddep_launch_dependents();
+  int issued = 0;  // thread 0: stages issued so far (0 .. issued - 1)
   auto issue_stage = [&](int j) {  // thread 0 only
-    mbar_arrive_expect_tx(&full[j % kWoStages], kWoStageBytes);
-    tma_load_2d(ring + (j % kWoStages) * kWoStageBytes, &tmW, k_lo + j * kWoStageCols, row0, &full[j % kWoStages]);
+    if (!(p.skip_first_load && j == 0)) {  // test hook: the first stage never fills
+      mbar_arrive_expect_tx(&full[j % kWoStages], kWoStageBytes);
+      tma_load_2d(ring + (j % kWoStages) * kWoStageBytes, &tmW, k_lo + j * kWoStageCols, row0, &full[j % kWoStages]);
+    }
+    issued = j + 1;
   };
   if (threadIdx.x == 0)
     for (int j = 0; j < min(kWoStages, nstages); ++j) issue_stage(j);
@@ -199,7 +204,7 @@ __global__ void __launch_bounds__(kWoThreads, 1) weight_only_kernel(const __grid
     for (int q = 0; q < kWoTok / 2; ++q) acc[r][q] = 0ull;
   for (int j = 0; j < nstages; ++j) {
     const int st = j % kWoStages;
-    const bool ok = !*abort_flag && mbar_wait_bounded(&full[st], static_cast<uint32_t>((j / kWoStages) & 1), kWoWaitNs);
+    const bool ok = !*abort_flag && mbar_wait_bounded(&full[st], static_cast<uint32_t>((j / kWoStages) & 1), p.timeout_ns);
     if (!__all_sync(0xFFFFFFFFu, ok)) {
       if (lane == 0) {
         *abort_flag = 1;
@@ -260,9 +265,11 @@ __global__ void __launch_bounds__(kWoThreads, 1) weight_only_kernel(const __grid
     }
   }
   if (*abort_flag && threadIdx.x == 0) {
-    // let the copies already issued land before the block exits
-    for (int j = max(0, nstages - kWoStages); j < nstages; ++j)
-      (void)mbar_wait_bounded(&full[j % kWoStages], static_cast<uint32_t>((j / kWoStages) & 1), kWoWaitNs);
+    // let the copies issued and not yet consumed land before the block exits
+    // (the last kWoStages issued; a skipped first stage never completes)
+    for (int j = max(0, issued - kWoStages); j < issued; ++j)
+      if (!(p.skip_first_load && j == 0))
+        (void)mbar_wait_bounded(&full[j % kWoStages], static_cast<uint32_t>((j / kWoStages) & 1), p.timeout_ns);
   }
 
   // ---- the eight warps' sums -> one per (token, row)
@@ -346,6 +353,7 @@ cudaError_t launch_weight_only(const uint16_t* X, int64_t M, const int8_t* Wq, c
   p.N = static_cast<int>(N);
   p.K = static_cast<int>(K);
   p.kc = static_cast<int>(kc);
+  p.skip_first_load = debug_stall_state(&p.timeout_ns) ? 1 : 0;
   CUtensorMap tmW;
   if (!make_tmap_2d(&tmW, Wq, N, K, 1, kWoStageCols, kWoRows, 128)) return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(weight_only_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kWoSmemBytes);
