@@ -372,8 +372,9 @@ SQ_API void sq_debug_fail_after(int n);
 /* sq_debug_pipeline_stall -- device-side failure test: while enabled
  * (enable != 0), the GEMM kernels used by sq_linear / sq_forward / sq_gemm_s32
  * (any M), by sq_forward_prologue, by sq_ste_backward and by
- * sq_linear_weight_only never load their first pipeline stage and every
- * pipeline wait gives up after timeout_ns (<= 0: the normal 2 s).  The kernel then sets bit 0 of
+ * sq_linear_weight_only, and the column-max kernel of sq_calibrate, never
+ * load their first pipeline stage and every pipeline wait gives up after
+ * timeout_ns (<= 0: the normal 2 s).  The kernel then sets bit 0 of
  * the device status word, drains its copies in flight, frees its tensor memory
  * and returns: the call's output is invalid, the CUDA context stays usable and
  * sq_device_status() reports SQ_ERR_TIMEOUT.  No GPU fault is involved.

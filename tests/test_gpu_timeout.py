@@ -228,3 +228,34 @@ def test_weight_only_wait_timeout_is_reported_and_the_context_survives(sq):
     assert elapsed < 5.0
     _check(sq, X, W, None, "weight-only after a timeout")
     assert sq.sq_device_status() == 0
+
+
+def test_calibration_wait_timeout_is_reported_and_the_context_survives(sq):
+    """The same failure in the calibration (column max-abs over C and W by a
+    TMA ring per block): the first box of every block never fills, the waits
+    give up, every block still merges what it has and takes part in its
+    stripe's arrival count, so the workspace is left zero; the next call
+    equals the oracle's s."""
+    from tests.helpers import assert_scales_close, dev_bf16
+    import workloads
+    C = workloads.random_bf16((512, 4096), seed=21, scale=1.0, outlier_cols=[7, 900], outlier_scale=40.0)
+    W = workloads.random_bf16((1024, 4096), seed=22, scale=0.02)
+    Cd, Wd = dev_bf16(C), dev_bf16(W)
+    torch.cuda.synchronize()
+    assert sq.sq_device_status(clear=True) == 0
+    try:
+        sq.sq_debug_pipeline_stall(True, 50_000_000)
+        t0 = time.perf_counter()
+        sq.sq_calibrate(Cd, Wd, 0.5)
+        torch.cuda.synchronize()
+        elapsed = time.perf_counter() - t0
+    finally:
+        sq.sq_debug_pipeline_stall(False)
+    flags = sq.sq_device_status(clear=True)
+    assert flags & 1, "the stalled calibration was not reported"
+    assert elapsed < 5.0
+    s = sq.sq_calibrate(Cd, Wd, 0.5)
+    torch.cuda.synchronize()
+    s_o, _ = O.calibrate(C, W, np.float32(0.5))
+    assert_scales_close(host(s), s_o, "calibration after a timeout")
+    assert sq.sq_device_status() == 0

@@ -25,7 +25,6 @@ namespace sq {
 // Latched by a wait in these kernels that ran out of time (bit 0), like the
 // GEMM's status word; read and cleared through read_device_status.
 __device__ unsigned int g_sq_quant_status = 0u;
-constexpr unsigned long long kQuantWaitTimeoutNs = 2000000000ull;  // 2 s per wait
 
 
 
@@ -111,6 +110,7 @@ struct ColmaxParams {
   float* mx_inout;
   float* s;
   unsigned long long timeout_ns;
+  int skip_first_load;  // test hook: the first box of every block is never loaded
 };
 
 __device__ __forceinline__ float smoothing_factor(float mx, float mw, double alpha) {
@@ -173,13 +173,16 @@ __global__ void __launch_bounds__(kColThreads) colmax_kernel(const __grid_consta
           atomicOr(&g_sq_quant_status, 1u);
           break;
         }
+        if (p.skip_first_load && j == 0) continue;  // test hook: this box never fills
         mbar_arrive_expect_tx(&full[st], box_bytes);
         tma_load_2d(smem + st * kColStageBytes, map, stripe * p.box_cols, r0 + j * kColBoxRows, &full[st]);
       }
       if (j < nbox) {
         // gave up: let the copies already issued land before the block exits
+        // (a skipped box never completes)
         for (int q = max(0, j - kColStages); q < j; ++q)
-          (void)mbar_wait_bounded(&full[q % kColStages], static_cast<uint32_t>((q / kColStages) & 1), p.timeout_ns);
+          if (!(p.skip_first_load && q == 0))
+            (void)mbar_wait_bounded(&full[q % kColStages], static_cast<uint32_t>((q / kColStages) & 1), p.timeout_ns);
       }
     }
   } else {
@@ -324,7 +327,7 @@ cudaError_t launch_calibrate(const uint16_t* C, int64_t R, int64_t K, const uint
   p.alpha = static_cast<double>(alpha);
   p.mx_inout = mx_inout;
   p.s = s;
-  p.timeout_ns = kQuantWaitTimeoutNs;
+  p.skip_first_load = debug_stall_state(&p.timeout_ns) ? 1 : 0;  // the normal limit: 2 s
   const int64_t grid = static_cast<int64_t>(stripes) * (p.chunks_c + p.chunks_w);
   return launch_pdl(colmax_kernel, dim3(static_cast<unsigned>(grid)), dim3(kColThreads),
                     static_cast<size_t>(kColSmemBytes), st, tmC, tmW, p);
