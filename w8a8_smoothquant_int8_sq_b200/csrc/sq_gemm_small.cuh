@@ -18,9 +18,10 @@
 //   * split-K over a thread-block cluster of S CTAs: each CTA streams its
 //     share of the row block's K; at the end every CTA pushes its partial
 //     int32 sums of each row (real tokens only) into the shared memory of the
-//     rank that reduces that row, and after one cluster barrier each rank adds
-//     the S partials of its rows from its own shared memory (exact, no global
-//     scratch, no remote load on the critical path).
+//     rank that reduces that row with st.async, whose bytes count on that
+//     rank's mbarrier, and once its phase completes each rank adds the S
+//     partials of its rows from its own shared memory (exact, no global
+//     scratch, no remote load and no cluster barrier at the end).
 //   * prequantised codes (sq_linear): the codes travel by TMA in the same
 //     stage as the weight box (NT-row box, rows past M zero-filled), so the
 //     first MMA waits only for the first stage.
@@ -40,7 +41,9 @@
 //
 // Warps: 0 TMA producer, 1 TMEM owner + MMA issuer, 2..9 quantisation and
 // reduction (2..5 also drain TMEM: lane quarters 2, 3, 0, 1).  Every mbarrier
-// wait is bounded; every thread reaches every cluster barrier.
+// wait is bounded; every thread takes part in the one cluster phase (arrived
+// after the barrier set-up, waited for before its first remote store or at
+// the end).
 
 namespace sq {
 namespace {
